@@ -1,0 +1,417 @@
+"""CPU oracle for the 4-bit paged KV cache and its decode attention.
+
+TEST INFRASTRUCTURE.  Only the test suite, the smoke check in
+``__graft_entry__.smoke()`` and the CPU-baseline / reference leg of
+``bench.py`` may import or run this module.  The product path never does:
+the CUDA library has no CPU fallback and shares no code, constant or table
+with this file.
+
+What it computes, step by step, and where each step comes from:
+
+  [AMBP]  "Agent Memory Below the Prompt: Persistent Q4 KV Cache for
+          Multi-Agent LLM Inference on Edge Devices" (gist.science summary of
+          arXiv 2603.04428).  Section 2.1, item 1: the cache is cut into
+          256-token blocks.  Section 2.1, item 2: 4-bit codes packed into
+          uint32 words with one 16-bit scale and one 16-bit bias per group,
+          read directly by attention ("direct restore"), about 72 % smaller
+          than FP16.  Section 2.1, item 3: attention batched over several
+          agents' quantised caches.  Section 2.2: GQA models.
+  [UQ]    UltraQuant news item (poko-everyday.com, arXiv 2606.20474),
+          section "technology / business": a Walsh-Hadamard rotation before
+          4-bit quantisation, with keys and values treated asymmetrically.
+  [IKV]   IntentKV article (Qiita), section "invalidate instead of
+          compacting": an evicted slot is re-pointed to a sentinel slot
+          whose key is -1e4, so its softmax weight collapses to zero while
+          every surviving slot keeps its position.
+  [QKVS]  QKVShare (gist.science summary of arXiv 2605.03884),
+          "Methodologie": bit widths drawn from {2, 4, 8, FP16}; the
+          receiver dequantises the shared cache before use.
+
+Readings taken where the pages leave a step open (each is restated in the
+design notes):
+  * groups are 64 consecutive values along head_dim of one (token, head)
+    vector; scale s and zero z are fp16 (binary16), z is an additive offset;
+  * the rotation is the orthonormal Sylvester-ordered Walsh-Hadamard
+    transform c*H_D, c = binary32 nearest to 1/sqrt(D), butterflies applied
+    in ascending stride order h = 1, 2, ..., D/2; K is rotated, V is not;
+    the query is rotated by the same transform inside attention;
+  * codes are computed from the *stored* fp16 s and z with binary32
+    subtraction and division, rounded half to even, then clamped;
+    min and max have +0.0 added so a signed zero never reaches the
+    stored parameters;
+  * nibble order: value 2i in the low nibble of byte i, so element j of a
+    little-endian uint32 word sits at bits 4*(j mod 8);
+  * an evicted slot's *logit* is -1e4 and its value is 0; its stored bytes
+    stay where they are; one 256-bit mask per physical block, shared by
+    all KV heads; writing a token into a slot makes the slot live again;
+  * 8-bit blocks use the same steps with 255 levels, one code per byte.
+
+Precision: the encoding steps (rotation, min/max, scale/zero, codes,
+dequantisation) are binary32/binary16 by definition, so they are written
+with numpy float32/float16 scalars-arrays, one IEEE operation per step and
+no fused multiply-add.  Attention is fp64 over the dequantised cache.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+BLOCK_TOKENS = 256          # [AMBP] 2.1 item 1
+GROUP = 64                  # values sharing one (scale, zero) pair
+SENTINEL_LOGIT = -1.0e4     # [IKV]
+MASK_WORDS = BLOCK_TOKENS // 32
+
+
+def levels(bits: int) -> int:
+    """Largest code of a `bits`-wide unsigned code (15 for Q4, 255 for Q8)."""
+    return (1 << bits) - 1
+
+
+# ---------------------------------------------------------------------------
+# input conversion (exact)
+# ---------------------------------------------------------------------------
+
+def to_f32(a: np.ndarray, dtype: str) -> np.ndarray:
+    """fp16 / bf16 input -> binary32, exactly.
+
+    fp16 arrives as np.float16; bf16 arrives as its raw uint16 bit pattern
+    (numpy has no bfloat16), which is the upper half of a binary32.
+    """
+    if dtype == "fp16":
+        return np.asarray(a, dtype=np.float16).astype(np.float32)
+    if dtype == "bf16":
+        bits = np.asarray(a, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+        return bits.view(np.float32)
+    if dtype == "fp32":
+        return np.asarray(a, dtype=np.float32)
+    raise ValueError(dtype)
+
+
+# ---------------------------------------------------------------------------
+# Walsh-Hadamard rotation [UQ]
+# ---------------------------------------------------------------------------
+
+def rotation_constant(d: int) -> np.float32:
+    """c = binary32 nearest to 1/sqrt(d) for d a power of two.
+
+    1/sqrt(2^k) is 2^(-k/2) for even k and sqrt(2) * 2^(-(k+1)/2) for odd k;
+    both are formed from the correctly rounded double sqrt(2), then rounded
+    once to binary32.
+    """
+    k = int(round(math.log2(d)))
+    assert 1 << k == d, "head_dim must be a power of two"
+    if k % 2 == 0:
+        return np.float32(2.0 ** (-k // 2))
+    return np.float32(math.sqrt(2.0) * 2.0 ** (-(k + 1) // 2))
+
+
+def fwht(x: np.ndarray, dtype=np.float32) -> np.ndarray:
+    """Unnormalised Sylvester-ordered Walsh-Hadamard transform, last axis.
+
+    Stages run with stride h = 1, 2, 4, ..., n/2.  In each stage every pair
+    (i, i+h) with bit h of i clear becomes (x_i + x_{i+h}, x_i - x_{i+h}),
+    each sum and difference one IEEE operation in `dtype`.  The result is
+    H_n x with H_n[i, j] = (-1)^popcount(i & j).
+    """
+    y = np.array(x, dtype=dtype, copy=True)
+    n = y.shape[-1]
+    h = 1
+    while h < n:
+        v = y.reshape(y.shape[:-1] + (n // (2 * h), 2, h))
+        a = v[..., 0, :].copy()
+        b = v[..., 1, :].copy()
+        v[..., 0, :] = a + b
+        v[..., 1, :] = a - b
+        h *= 2
+    return y
+
+
+def rotate_f32(x: np.ndarray) -> np.ndarray:
+    """c * H x in binary32: the butterflies, then one multiply by c."""
+    d = x.shape[-1]
+    return fwht(x, np.float32) * rotation_constant(d)
+
+
+def rotate_f64(x: np.ndarray) -> np.ndarray:
+    """(1/sqrt(D)) * H x in fp64 (used for the query inside attention)."""
+    d = x.shape[-1]
+    return fwht(x, np.float64) * (1.0 / math.sqrt(d))
+
+
+# ---------------------------------------------------------------------------
+# group quantisation [AMBP 2.1 item 2], [UQ], [QKVS]
+# ---------------------------------------------------------------------------
+
+def quantize_groups(x: np.ndarray, bits: int):
+    """Quantise binary32 vectors x[..., D] group by group.
+
+    Returns (codes uint8 [..., D], scale fp16 [..., D/64], zero fp16 [..., D/64]).
+    Per group of 64 values:
+      mn = min + 0, mx = max + 0                  (exact)
+      s  = fl(fl(mx - mn) / L)                    L = 2^bits - 1
+      s_h = fp16(s), z_h = fp16(mn)               round to nearest even
+      code = 0 if s_h == 0 else clamp(rne(fl(fl(x - z_h) / s_h)), 0, L)
+    """
+    x = np.asarray(x, dtype=np.float32)
+    d = x.shape[-1]
+    assert d % GROUP == 0
+    L = np.float32(levels(bits))
+    g = x.reshape(x.shape[:-1] + (d // GROUP, GROUP))
+    zero = np.float32(0.0)
+    mn = g.min(axis=-1) + zero
+    mx = g.max(axis=-1) + zero
+    s = (mx - mn) / L
+    s_h = s.astype(np.float16)
+    z_h = mn.astype(np.float16)
+    sf = s_h.astype(np.float32)[..., None]
+    zf = z_h.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (g - zf) / sf
+    q = np.clip(np.rint(t), zero, L)
+    q = np.where(sf == zero, zero, q)
+    return q.astype(np.uint8).reshape(x.shape), s_h, z_h
+
+
+def dequantize_groups(codes: np.ndarray, s_h: np.ndarray, z_h: np.ndarray) -> np.ndarray:
+    """x_hat = fl(code * s_h + z_h) in binary32 (code * s_h is exact)."""
+    codes = np.asarray(codes)
+    d = codes.shape[-1]
+    c = codes.astype(np.float32).reshape(codes.shape[:-1] + (d // GROUP, GROUP))
+    sf = np.asarray(s_h, dtype=np.float16).astype(np.float32)[..., None]
+    zf = np.asarray(z_h, dtype=np.float16).astype(np.float32)[..., None]
+    return (c * sf + zf).reshape(codes.shape)
+
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """Two 4-bit codes per byte: element 2i low nibble, 2i+1 high nibble."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << np.uint8(4))).astype(np.uint8)
+
+
+def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    packed = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = packed & np.uint8(0x0F)
+    out[..., 1::2] = packed >> np.uint8(4)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the paged pool [AMBP 2.1 items 1-2], eviction mask [IKV]
+# ---------------------------------------------------------------------------
+
+class OraclePool:
+    """Host model of the paged cache.
+
+    Unified block ids: [0, n_q4) are 4-bit blocks, [n_q4, n_q4 + n_q8) are
+    8-bit blocks.  Per block and KV head: codes [256][D/2] (4-bit) or
+    [256][D] (8-bit) and params [256][D/64][2] fp16 as (scale, zero).
+    mask[block][8] uint32: bit (slot mod 32) of word (slot / 32) set means
+    the slot has been remapped to the sentinel.
+    """
+
+    def __init__(self, n_kv_heads: int, head_dim: int, n_q4: int, n_q8: int = 0,
+                 k_rotated: bool = True):
+        self.hkv = n_kv_heads
+        self.d = head_dim
+        self.n_q4 = n_q4
+        self.n_q8 = n_q8
+        self.k_rotated = k_rotated
+        ng = head_dim // GROUP
+        T = BLOCK_TOKENS
+        self.codes4 = {s: np.zeros((n_q4, n_kv_heads, T, head_dim // 2), np.uint8) for s in "kv"}
+        self.params4 = {s: np.zeros((n_q4, n_kv_heads, T, ng, 2), np.float16) for s in "kv"}
+        self.codes8 = {s: np.zeros((n_q8, n_kv_heads, T, head_dim), np.uint8) for s in "kv"}
+        self.params8 = {s: np.zeros((n_q8, n_kv_heads, T, ng, 2), np.float16) for s in "kv"}
+        self.mask = np.zeros((n_q4 + n_q8, MASK_WORDS), np.uint32)
+
+    @property
+    def n_blocks(self) -> int:
+        return self.n_q4 + self.n_q8
+
+    def bits(self, blk: int) -> int:
+        if not 0 <= blk < self.n_blocks:
+            raise IndexError(f"block id {blk} outside [0, {self.n_blocks})")
+        return 4 if blk < self.n_q4 else 8
+
+    # -- writes ------------------------------------------------------------
+    def quantize_blocks(self, k: np.ndarray, v: np.ndarray, dtype: str,
+                        block_ids: Sequence[int]) -> None:
+        """Encode tokens k/v [n][Hkv][D] into the pool.
+
+        Token i goes to block block_ids[i // 256], slot i % 256; the slot's
+        mask bit is cleared (a freshly written slot is live).
+        """
+        kf = to_f32(k, dtype)
+        vf = to_f32(v, dtype)
+        n = kf.shape[0]
+        assert kf.shape == (n, self.hkv, self.d) and vf.shape == kf.shape
+        for c in range(-(-n // BLOCK_TOKENS)):
+            t0, t1 = c * BLOCK_TOKENS, min(n, (c + 1) * BLOCK_TOKENS)
+            blk = int(block_ids[c])
+            bits = self.bits(blk)
+            kk = kf[t0:t1]
+            if self.k_rotated:
+                kk = rotate_f32(kk)
+            for name, x in (("k", kk), ("v", vf[t0:t1])):
+                codes, s_h, z_h = quantize_groups(x, bits)       # [cnt][Hkv][D]
+                codes = codes.transpose(1, 0, 2)                  # [Hkv][cnt][D]
+                par = np.stack([s_h, z_h], axis=-1).transpose(1, 0, 2, 3)
+                if bits == 4:
+                    self.codes4[name][blk, :, : t1 - t0] = pack_nibbles(codes)
+                    self.params4[name][blk, :, : t1 - t0] = par
+                else:
+                    i8 = blk - self.n_q4
+                    self.codes8[name][i8, :, : t1 - t0] = codes
+                    self.params8[name][i8, :, : t1 - t0] = par
+            for slot in range(t1 - t0):
+                self.mask[blk, slot // 32] &= np.uint32(~(1 << (slot % 32)) & 0xFFFFFFFF)
+
+    def invalidate_slots(self, slot_ids: Sequence[int]) -> None:
+        """Remap physical slots (block*256 + offset) to the sentinel [IKV]."""
+        for sid in slot_ids:
+            sid = int(sid)
+            blk, slot = divmod(sid, BLOCK_TOKENS)
+            self.bits(blk)
+            self.mask[blk, slot // 32] |= np.uint32(1 << (slot % 32))
+
+    # -- reads -------------------------------------------------------------
+    def masked(self, blk: int) -> np.ndarray:
+        """bool [256]: slot remapped to the sentinel."""
+        words = self.mask[blk]
+        return np.array([(int(words[t // 32]) >> (t % 32)) & 1 for t in range(BLOCK_TOKENS)],
+                        dtype=bool)
+
+    def codes_params(self, blk: int, name: str):
+        """(codes uint8 [Hkv][256][D], scale fp16 [Hkv][256][ng], zero fp16)."""
+        if self.bits(blk) == 4:
+            codes = unpack_nibbles(self.codes4[name][blk])
+            par = self.params4[name][blk]
+        else:
+            codes = self.codes8[name][blk - self.n_q4]
+            par = self.params8[name][blk - self.n_q4]
+        return codes, par[..., 0], par[..., 1]
+
+    def dequantize_block(self, blk: int, unrotate_k: bool = False):
+        """Binary32 K_hat, V_hat [Hkv][256][D] with the sentinel applied.
+
+        K is in the stored (rotated) domain unless `unrotate_k`; the inverse
+        of c*H is c*H itself (H symmetric, H H^T = D I), applied with the
+        same butterfly order.  Remapped slots read K = -1e4, V = 0.
+        """
+        out = []
+        for name in "kv":
+            codes, s_h, z_h = self.codes_params(blk, name)
+            x = dequantize_groups(codes, s_h, z_h)
+            if name == "k" and unrotate_k and self.k_rotated:
+                x = rotate_f32(x)
+            out.append(x)
+        k_hat, v_hat = out
+        m = self.masked(blk)
+        k_hat[:, m, :] = np.float32(SENTINEL_LOGIT)
+        v_hat[:, m, :] = np.float32(0.0)
+        return k_hat, v_hat
+
+
+# ---------------------------------------------------------------------------
+# decode attention [AMBP 2.1 items 2-3, 2.2], [IKV]
+# ---------------------------------------------------------------------------
+
+def decode_attention(pool: OraclePool, q: np.ndarray, q_dtype: str,
+                     block_tables: np.ndarray, seq_lens: Sequence[int],
+                     softmax_scale: Optional[float] = None,
+                     heads: Optional[Sequence[tuple]] = None) -> np.ndarray:
+    """fp64 single-token GQA attention over the paged quantised cache.
+
+    For sequence b and query head h (KV head h // g): token t of the
+    sequence lives in block block_tables[b][t // 256], slot t % 256.  Its
+    logit is scale * <q_rot, K_hat_t> (q_rot = (1/sqrt D) H q when K is
+    stored rotated), or -1e4 if the slot is remapped, in which case its
+    value is 0.  Output = softmax(logits) . V_hat, softmax max-subtracted.
+    A sequence with no tokens yields 0.
+
+    `heads` optionally restricts the work to a list of (b, h) pairs; the
+    other rows of the result stay 0.
+    """
+    qf = to_f32(q, q_dtype).astype(np.float64)
+    B, Hq, D = qf.shape
+    g = Hq // pool.hkv
+    assert g * pool.hkv == Hq and D == pool.d
+    if softmax_scale is None or softmax_scale <= 0:
+        softmax_scale = 1.0 / math.sqrt(D)
+    want = None if heads is None else {}
+    if heads is not None:
+        for b, h in heads:
+            want.setdefault(int(b), []).append(int(h))
+    out = np.zeros((B, Hq, D), np.float64)
+    for b in range(B):
+        if want is not None and b not in want:
+            continue
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        ks, vs, ms = [], [], []
+        for c in range(-(-n // BLOCK_TOKENS)):
+            cnt = min(BLOCK_TOKENS, n - c * BLOCK_TOKENS)
+            blk = int(block_tables[b][c])
+            k_hat, v_hat = pool.dequantize_block(blk)
+            ks.append(k_hat[:, :cnt])
+            vs.append(v_hat[:, :cnt])
+            ms.append(pool.masked(blk)[:cnt])
+        K = np.concatenate(ks, axis=1).astype(np.float64)    # [Hkv][n][D]
+        V = np.concatenate(vs, axis=1).astype(np.float64)
+        M = np.concatenate(ms)
+        for h in (range(Hq) if want is None else want[b]):
+            kv = h // g
+            qv = rotate_f64(qf[b, h]) if pool.k_rotated else qf[b, h]
+            s = softmax_scale * (K[kv] @ qv)
+            s[M] = SENTINEL_LOGIT          # V_hat of these rows is already 0
+            p = np.exp(s - s.max())
+            out[b, h] = (p @ V[kv]) / p.sum()
+    return out
+
+
+# ---------------------------------------------------------------------------
+# mixed 4/8-bit block selection [QKVS]
+# ---------------------------------------------------------------------------
+
+def block_absmean(k: np.ndarray, dtype: str) -> np.ndarray:
+    """fp64 mean |K| of each 256-token chunk of raw (unrotated) keys [n][Hkv][D]."""
+    kf = to_f32(k, dtype).astype(np.float64)
+    n = kf.shape[0]
+    out = []
+    for c in range(-(-n // BLOCK_TOKENS)):
+        chunk = np.abs(kf[c * BLOCK_TOKENS: (c + 1) * BLOCK_TOKENS])
+        out.append(chunk.sum() / chunk.size)
+    return np.array(out, dtype=np.float64)
+
+
+def mixed_block_ids(absmean: np.ndarray, n_q8: int, q4_first: int, q8_first: int) -> np.ndarray:
+    """Block id per chunk: the n_q8 chunks of highest mean |K| go 8-bit.
+
+    Ranking is descending mean |K| with ties to the lower chunk index.  The
+    k-th 8-bit chunk in chunk order gets id q8_first + k, the k-th 4-bit
+    chunk gets q4_first + k.
+    """
+    n = len(absmean)
+    order = sorted(range(n), key=lambda i: (-float(absmean[i]), i))
+    chosen = set(order[:n_q8])
+    ids = np.empty(n, np.int32)
+    n8 = n4 = 0
+    for i in range(n):
+        if i in chosen:
+            ids[i] = q8_first + n8
+            n8 += 1
+        else:
+            ids[i] = q4_first + n4
+            n4 += 1
+    return ids
+
+
+def bytes_per_token_head(head_dim: int, bits: int) -> int:
+    """Stored bytes for one (token, KV head): K and V codes plus fp16 (s, z)."""
+    code_bytes = head_dim * bits // 8
+    param_bytes = (head_dim // GROUP) * 2 * 2
+    return 2 * (code_bytes + param_bytes)

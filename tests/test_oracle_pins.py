@@ -1,0 +1,443 @@
+"""Pins for the CPU oracle against facts outside the oracle itself.
+
+Each test checks the oracle against something the pages print (fixtures in
+tests/golden), a closed form, a textbook identity, a library routine that
+computes the same mathematics by another route, or brute force on tiny
+inputs.  A dropped term, a wrong sign or index, a transposed operand or a
+wrong rounding rule in the oracle fails at least one of them.
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.special
+
+from conftest import read_golden
+from oracle import q4kv_oracle as O
+
+
+def _hexf(s):
+    return np.float32(float.fromhex(s))
+
+
+# ---------------------------------------------------------------------------
+# Walsh-Hadamard rotation
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64, 128, 256])
+def test_fwht_is_sylvester_matrix(n):
+    # transform of each basis vector gives one column of H (exact integers)
+    H = O.fwht(np.eye(n), np.float64).T
+    i = np.arange(n)
+    popc = np.vectorize(lambda a: bin(a).count("1"))(i[:, None] & i[None, :])
+    assert np.array_equal(H, (-1.0) ** popc)
+    Hi = H.astype(np.int64)
+    assert np.array_equal(Hi @ Hi.T, n * np.eye(n, dtype=np.int64))
+    # textbook Sylvester construction (library routine)
+    assert np.array_equal(Hi, scipy.linalg.hadamard(n))
+
+
+def test_fwht_h2():
+    assert np.array_equal(O.fwht(np.array([3.0, 5.0]), np.float64), [8.0, -2.0])
+
+
+@pytest.mark.parametrize("n", [128, 256])
+def test_fwht_matches_matrix_product(n):
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((5, n))
+    Hs = scipy.linalg.hadamard(n).astype(np.float64)
+    assert np.allclose(O.fwht(x, np.float64), x @ Hs.T, rtol=0, atol=1e-11)
+    # integer inputs are exact in binary32 as well
+    xi = rng.integers(-1000, 1000, size=(5, n)).astype(np.float32)
+    exact = xi.astype(np.int64) @ scipy.linalg.hadamard(n).T
+    assert np.array_equal(O.fwht(xi, np.float32).astype(np.int64), exact)
+
+
+@pytest.mark.parametrize("n", [64, 128, 256, 512])
+def test_rotation_constant_is_nearest_binary32(n):
+    c = O.rotation_constant(n)
+    lo = np.nextafter(c, np.float32(0))
+    hi = np.nextafter(c, np.float32(1))
+    C, L, Hh = Fraction(float(c)), Fraction(float(lo)), Fraction(float(hi))
+    target_sq = Fraction(1, n)                       # (1/sqrt n)^2
+    assert ((L + C) / 2) ** 2 < target_sq < ((C + Hh) / 2) ** 2
+    if n == 256:
+        assert c == np.float32(0.0625)
+    if n == 128:
+        assert float(c) == float.fromhex("0x1.6a09e6p-4")
+
+
+@pytest.mark.parametrize("n", [128, 256])
+def test_rotation_special_vectors(n):
+    c = O.rotation_constant(n)
+    e0 = np.zeros(n, np.float32)
+    e0[0] = 1
+    assert np.array_equal(O.rotate_f32(e0), np.full(n, c, np.float32))
+    ones = np.ones(n, np.float32)
+    want = np.zeros(n, np.float32)
+    want[0] = np.float32(n) * c
+    assert np.array_equal(O.rotate_f32(ones), want)
+
+
+def test_rotation_preserves_norm():
+    rng = np.random.default_rng(2)
+    for n in (128, 256):
+        x = rng.standard_normal((64, n)).astype(np.float32)
+        y = O.rotate_f32(x)
+        r = np.linalg.norm(y.astype(np.float64), axis=1) / np.linalg.norm(x.astype(np.float64), axis=1)
+        assert np.all(np.abs(r - 1) < 8 * math.log2(n) * 2.0 ** -24)
+
+
+def test_stage_order_worked_example():
+    g = read_golden("fwht_stage_order.txt")
+    x = np.array([_hexf(s) for s in g["input_hex"].split()], np.float32)
+    out = O.fwht(x, np.float32)
+    assert out[0] == _hexf(g["ascending_out0_hex"])
+    assert out[0] != _hexf(g["descending_out0_hex"])
+
+
+def test_rotation_is_self_inverse():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((16, 128))
+    assert np.allclose(O.rotate_f64(O.rotate_f64(x)), x, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# group quantiser and packing
+# ---------------------------------------------------------------------------
+
+def test_ramp_gives_exact_codes():
+    g = read_golden("quantizer_cases.txt")
+    z, s = float(g["ramp_z"]), float(g["ramp_s"])
+    j = np.arange(64)
+    x = (z + (j % 16) * s).astype(np.float32)[None, :]
+    codes, s_h, z_h = O.quantize_groups(x, 4)
+    assert s_h[0, 0] == np.float16(s) and z_h[0, 0] == np.float16(z)
+    assert np.array_equal(codes[0], j % 16)
+    assert np.array_equal(O.dequantize_groups(codes, s_h, z_h), x)
+
+
+def test_ties_round_to_even():
+    g = read_golden("quantizer_cases.txt")
+    want = [int(v) for v in g["ties_expected"].split(",")]
+    z, s = -1.5, 0.25
+    vals = [z, z + 15 * s] + [z + (k + 0.5) * s for k in range(15)]
+    x = np.array(vals + [z] * (64 - len(vals)), np.float32)[None, :]
+    codes, s_h, z_h = O.quantize_groups(x, 4)
+    assert s_h[0, 0] == np.float16(0.25) and z_h[0, 0] == np.float16(-1.5)
+    assert codes[0, 0] == 0 and codes[0, 1] == 15
+    assert list(codes[0, 2:17]) == want
+
+
+def test_constant_group():
+    g = read_golden("quantizer_cases.txt")
+    v = float(g["constant_value"])
+    x = np.full((1, 128), v, np.float32)
+    codes, s_h, z_h = O.quantize_groups(x, 4)
+    assert np.all(codes == 0) and np.all(s_h == 0)
+    assert np.all(z_h.view(np.uint16) == int(g["constant_zero_fp16_bits"], 16))
+    assert np.all(O.dequantize_groups(codes, s_h, z_h) == np.float32(np.float16(v)))
+
+
+def test_signed_zero_never_reaches_params():
+    for x in (np.full((1, 64), -0.0, np.float32), np.zeros((1, 64), np.float32)):
+        x[0, 1::2] = -0.0
+        codes, s_h, z_h = O.quantize_groups(x, 4)
+        assert s_h.view(np.uint16)[0, 0] == 0 and z_h.view(np.uint16)[0, 0] == 0
+        assert np.all(codes == 0)
+
+
+def test_fp16_rounding_of_scale_is_ties_to_even():
+    assert np.float16(np.float32(1 + 2.0 ** -11)) == np.float16(1.0)
+    assert np.float16(np.float32(1 + 3 * 2.0 ** -11)) == np.float16(1 + 2.0 ** -9)
+
+
+def test_scale_and_zero_definition():
+    # mx - mn = 1.0 -> s = fl(1/15) -> fp16; zero = fp16(mn)
+    x = np.linspace(0.3, 1.3, 64).astype(np.float32)
+    x[0], x[-1] = np.float32(0.3), np.float32(1.3)
+    codes, s_h, z_h = O.quantize_groups(x[None, :], 4)
+    s32 = (np.float32(1.3) - np.float32(0.3)) / np.float32(15)
+    assert s_h[0, 0] == np.float16(s32)
+    assert z_h[0, 0] == np.float16(np.float32(0.3))
+    # 8-bit uses 255 levels
+    c8, s8, z8 = O.quantize_groups(x[None, :], 8)
+    assert s8[0, 0] == np.float16((np.float32(1.3) - np.float32(0.3)) / np.float32(255))
+    assert c8.max() == 255 and c8.min() == 0
+
+
+def _roundtrip_bound(x, codes, s_h, z_h, bits):
+    L = O.levels(bits)
+    d = x.shape[-1]
+    xs = x.reshape(x.shape[:-1] + (d // 64, 64)).astype(np.float64)
+    sf = s_h.astype(np.float64)[..., None]
+    zf = z_h.astype(np.float64)[..., None]
+    xh = O.dequantize_groups(codes, s_h, z_h).reshape(xs.shape).astype(np.float64)
+    err = np.abs(xs - xh)
+    inner = np.maximum(0.5 * sf, np.maximum(zf - xs, xs - zf - L * sf))
+    slack = 2.0 ** -18 * sf + np.spacing(np.abs(xh).astype(np.float32)).astype(np.float64)
+    return err, inner + slack
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_roundtrip_error_bound_random(bits):
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((300, 128)) * rng.choice([0.01, 1, 30], size=(300, 1))).astype(np.float32)
+    codes, s_h, z_h = O.quantize_groups(x, bits)
+    err, bound = _roundtrip_bound(x, codes, s_h, z_h, bits)
+    assert np.all(err <= bound)
+
+
+def test_roundtrip_half_scale_when_params_exact():
+    # values on an fp16-friendly grid: mn and s exact in fp16 -> |x - x_hat| <= s/2
+    rng = np.random.default_rng(5)
+    z = np.float32(-2.0)
+    s = np.float32(0.25)
+    inner = rng.uniform(0, 15, size=(200, 62)).astype(np.float32) * s + z
+    x = np.concatenate([np.full((200, 1), z), np.full((200, 1), z + 15 * s), inner], axis=1)
+    codes, s_h, z_h = O.quantize_groups(x.astype(np.float32), 4)
+    assert np.all(s_h == np.float16(s)) and np.all(z_h == np.float16(z))
+    xh = O.dequantize_groups(codes, s_h, z_h)
+    assert np.all(np.abs(x - xh) <= s / 2)
+
+
+def test_pack_order():
+    g = read_golden("quantizer_cases.txt")
+    assert O.pack_nibbles(np.array([1, 2], np.uint8))[0] == 0x21
+    word = O.pack_nibbles(np.arange(8, dtype=np.uint8)).view("<u4")[0]
+    assert word == int(g["packed_word_0to7"], 16)
+    rng = np.random.default_rng(6)
+    c = rng.integers(0, 16, size=(7, 128)).astype(np.uint8)
+    assert np.array_equal(O.unpack_nibbles(O.pack_nibbles(c)), c)
+
+
+def test_memory_saving_matches_page_figure():
+    g = read_golden("page_figures.txt")
+    fp16 = 2 * 128 * 2
+    q4 = O.bytes_per_token_head(128, 4)
+    assert q4 == 144
+    saving = 100.0 * (1 - q4 / fp16)
+    assert saving == 71.875
+    assert abs(saving - float(g["q4_memory_saving_percent_approx"])) < 0.5
+    assert int(g["q4_scale_bits"]) == 16 and int(g["q4_bias_bits"]) == 16
+    assert O.BLOCK_TOKENS == int(g["block_tokens"])
+    assert O.SENTINEL_LOGIT == float(g["sentinel_key"])
+    assert 4 in [int(b) for b in g["mixed_bit_widths"].split(",")]
+    assert 8 in [int(b) for b in g["mixed_bit_widths"].split(",")]
+
+
+# ---------------------------------------------------------------------------
+# pool and attention
+# ---------------------------------------------------------------------------
+
+def _pool_with(k, v, dtype="fp16", n_q4=None, n_q8=0, ids=None, rotated=True):
+    n, hkv, d = k.shape
+    nb = -(-n // 256)
+    if n_q4 is None:
+        n_q4 = nb
+    pool = O.OraclePool(hkv, d, n_q4, n_q8, k_rotated=rotated)
+    pool.quantize_blocks(k, v, dtype, list(range(nb)) if ids is None else ids)
+    return pool
+
+
+def _rand_kv(n, hkv, d, seed):
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    v = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    return k, v
+
+
+def test_attention_matches_explicit_brute_force():
+    """Independent route: explicit Hadamard matrix, scipy softmax, fp64."""
+    d, hkv, hq, n = 128, 2, 8, 300
+    k, v = _rand_kv(n, hkv, d, 7)
+    pool = _pool_with(k, v)
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((1, hq, d)).astype(np.float16)
+    tables = np.array([[0, 1]], np.int32)
+    out = O.decode_attention(pool, q, "fp16", tables, [n])
+    H = scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d)
+    kh = np.concatenate([pool.dequantize_block(b)[0] for b in (0, 1)], axis=1)[:, :n].astype(np.float64)
+    vh = np.concatenate([pool.dequantize_block(b)[1] for b in (0, 1)], axis=1)[:, :n].astype(np.float64)
+    for h in range(hq):
+        kv = h // (hq // hkv)
+        logits = (kh[kv] @ (H @ q[0, h].astype(np.float64))) / math.sqrt(d)
+        want = scipy.special.softmax(logits) @ vh[kv]
+        assert np.allclose(out[0, h], want, rtol=0, atol=1e-12)
+
+
+def test_attention_rotation_consistency():
+    """<Hq, Hk> = <q, k>: attending in the unrotated domain gives the same result."""
+    d, n = 128, 256
+    k, v = _rand_kv(n, 1, d, 9)
+    pool = _pool_with(k, v)
+    q = np.random.default_rng(10).standard_normal((1, 2, d)).astype(np.float16)
+    out = O.decode_attention(pool, q, "fp16", np.array([[0]]), [n])
+    k_un = pool.dequantize_block(0, unrotate_k=True)[0][0].astype(np.float64)
+    vh = pool.dequantize_block(0)[1][0].astype(np.float64)
+    for h in range(2):
+        s = (k_un @ q[0, h].astype(np.float64)) / math.sqrt(d)
+        want = scipy.special.softmax(s) @ vh
+        assert np.allclose(out[0, h], want, atol=2e-5)
+
+
+def test_single_live_slot_returns_its_value():
+    d, n = 128, 200
+    k, v = _rand_kv(n, 1, d, 11)
+    pool = _pool_with(k, v)
+    pool.invalidate_slots([t for t in range(n) if t != 57])
+    q = np.random.default_rng(12).standard_normal((1, 4, d)).astype(np.float16)
+    out = O.decode_attention(pool, q, "fp16", np.array([[0]]), [n])
+    codes, s_h, z_h = pool.codes_params(0, "v")
+    want = O.dequantize_groups(codes[0, 57], s_h[0, 57], z_h[0, 57]).astype(np.float64)
+    for h in range(4):
+        assert np.array_equal(out[0, h], want)
+
+
+def test_sentinel_weight_is_exactly_zero():
+    # exp(-1e4 - m) underflows to +0 in fp64 once m > -1e4 + 745
+    assert np.exp(np.float64(O.SENTINEL_LOGIT) - (-9000.0)) == 0.0
+    assert np.exp(np.float32(O.SENTINEL_LOGIT) - np.float32(-9000.0)) == 0.0
+    d, n = 128, 512
+    k, v = _rand_kv(n, 1, d, 13)
+    pool = _pool_with(k, v)
+    masked = list(range(0, n, 3))
+    pool.invalidate_slots(masked)
+    q = np.random.default_rng(14).standard_normal((1, 4, d)).astype(np.float16)
+    out = O.decode_attention(pool, q, "fp16", np.array([[0, 1]]), [n])
+    # same tokens with the masked ones removed: a fresh pool holding only live rows
+    live = [t for t in range(n) if t not in set(masked)]
+    pool2 = _pool_with(k[live], v[live])
+    # the live rows quantise identically (per-vector groups), so values agree
+    out2 = O.decode_attention(pool2, q, "fp16", np.array([[0, 1]]), [len(live)])
+    assert np.allclose(out, out2, rtol=0, atol=1e-13)
+
+
+def test_dequantize_applies_sentinel():
+    d, n = 128, 256
+    k, v = _rand_kv(n, 2, d, 25)
+    pool = _pool_with(k, v)
+    pool.invalidate_slots([0, 77, 255])
+    for unrot in (False, True):
+        kh, vh = pool.dequantize_block(0, unrotate_k=unrot)
+        for t in (0, 77, 255):
+            assert np.all(kh[:, t] == np.float32(-1e4)) and np.all(vh[:, t] == 0)
+        assert np.all(vh[:, 1] != 0) or np.any(vh[:, 1] != 0)
+    # live rows: K dequantises to code*s + z in the rotated domain; unrotating
+    # brings it back within the quantiser's error of the raw key
+    kh, _ = pool.dequantize_block(0, unrotate_k=True)
+    assert np.abs(kh[:, 5] - k[5].astype(np.float32)).max() < 0.6
+
+
+def test_all_masked_and_empty_give_zero():
+    d, n = 128, 100
+    k, v = _rand_kv(n, 1, d, 15)
+    pool = _pool_with(k, v)
+    q = np.random.default_rng(16).standard_normal((2, 2, d)).astype(np.float16)
+    pool.invalidate_slots(range(n))
+    out = O.decode_attention(pool, q, "fp16", np.array([[0], [0]]), [n, 0])
+    assert np.all(out == 0)
+
+
+def test_zero_query_averages_live_values():
+    d, n = 128, 300
+    k, v = _rand_kv(n, 1, d, 17)
+    pool = _pool_with(k, v)
+    q = np.zeros((1, 1, d), np.float16)
+    out = O.decode_attention(pool, q, "fp16", np.array([[0, 1]]), [n])
+    vh = np.concatenate([pool.dequantize_block(b)[1][0] for b in (0, 1)])[:n].astype(np.float64)
+    assert np.allclose(out[0, 0], vh.mean(axis=0), atol=1e-13)
+
+
+def test_gqa_head_mapping():
+    # KV head j holds the constant value j + 1 in V; query head h must read j = h // g
+    d, hkv, g, n = 128, 4, 3, 64
+    rng = np.random.default_rng(18)
+    k = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    v = np.broadcast_to(np.arange(1, hkv + 1, dtype=np.float16)[None, :, None], (n, hkv, d)).copy()
+    pool = _pool_with(k, v)
+    q = rng.standard_normal((1, hkv * g, d)).astype(np.float16)
+    out = O.decode_attention(pool, q, "fp16", np.array([[0]]), [n])
+    for h in range(hkv * g):
+        assert np.allclose(out[0, h], h // g + 1, atol=1e-12)
+
+
+def test_block_table_indirection_and_permutation():
+    d, n = 128, 700
+    k, v = _rand_kv(n, 2, d, 19)
+    perm = [5, 2, 7]
+    pool = O.OraclePool(2, d, 8, 0)
+    pool.quantize_blocks(k, v, "fp16", perm)
+    ref = _pool_with(k, v)
+    q = np.random.default_rng(20).standard_normal((1, 4, d)).astype(np.float16)
+    a = O.decode_attention(pool, q, "fp16", np.array([perm]), [n])
+    b = O.decode_attention(ref, q, "fp16", np.array([[0, 1, 2]]), [n])
+    assert np.array_equal(a, b)
+    # a token's value is read from its own slot: the only live token at
+    # position 300 (block 1 of the table, slot 44) is returned verbatim
+    pool.invalidate_slots([blk * 256 + s for blk in perm for s in range(256)])
+    pool.mask[perm[1], 44 // 32] &= np.uint32(~(1 << (44 % 32)) & 0xFFFFFFFF)
+    c = O.decode_attention(pool, q, "fp16", np.array([perm]), [n])
+    codes, s_h, z_h = pool.codes_params(perm[1], "v")
+    want = O.dequantize_groups(codes[0, 44], s_h[0, 44], z_h[0, 44])
+    assert np.array_equal(c[0, 0], want.astype(np.float64))
+
+
+def test_softmax_scale_argument():
+    d, n = 128, 64
+    k, v = _rand_kv(n, 1, d, 21)
+    pool = _pool_with(k, v)
+    q = np.random.default_rng(22).standard_normal((1, 1, d)).astype(np.float16)
+    a = O.decode_attention(pool, q, "fp16", np.array([[0]]), [n], softmax_scale=0.25)
+    # doubling q (exact in fp16) and halving the scale leaves every logit unchanged
+    q2 = (q.astype(np.float32) * 2).astype(np.float16)
+    b = O.decode_attention(pool, q2, "fp16", np.array([[0]]), [n], softmax_scale=0.125)
+    assert np.array_equal(a, b)
+    # a non-positive scale selects 1/sqrt(D)
+    c = O.decode_attention(pool, q, "fp16", np.array([[0]]), [n], softmax_scale=0)
+    e = O.decode_attention(pool, q, "fp16", np.array([[0]]), [n], softmax_scale=1 / math.sqrt(d))
+    assert np.array_equal(c, e)
+
+
+def test_requantize_makes_slot_live():
+    d, n = 128, 256
+    k, v = _rand_kv(n, 1, d, 23)
+    pool = _pool_with(k, v)
+    pool.invalidate_slots([3, 4, 200])
+    assert pool.masked(0)[[3, 4, 200]].all()
+    pool.quantize_blocks(k, v, "fp16", [0])
+    assert not pool.masked(0).any()
+
+
+def test_q8_blocks_and_mixed_ids():
+    d, n = 128, 512
+    k, v = _rand_kv(n, 1, d, 24)
+    pool = O.OraclePool(1, d, 1, 1)
+    pool.quantize_blocks(k, v, "fp16", [1, 0])     # chunk 0 -> 8-bit block, chunk 1 -> 4-bit
+    kh8, _ = pool.dequantize_block(1, unrotate_k=True)
+    kh4, _ = pool.dequantize_block(0, unrotate_k=True)
+    e8 = np.abs(kh8[0] - k[:256, 0].astype(np.float32)).max()
+    e4 = np.abs(kh4[0] - k[256:, 0].astype(np.float32)).max()
+    assert e8 < e4 / 8
+    am = np.array([0.5, 2.0, 1.0, 2.0, 0.1])
+    ids = O.mixed_block_ids(am, 2, q4_first=0, q8_first=100)
+    # ranking: chunk 1 (2.0), chunk 3 (2.0, tie -> lower index first), chunk 2 ...
+    assert list(ids) == [0, 100, 1, 101, 2]
+    # with one 8-bit slot the tie between chunks 1 and 3 goes to chunk 1
+    assert list(O.mixed_block_ids(am, 1, 0, 100)) == [0, 100, 1, 2, 3]
+
+
+def test_block_absmean_closed_form():
+    k = np.full((300, 2, 128), -1.5, np.float16)
+    k[256:] = 0.25
+    am = O.block_absmean(k, "fp16")
+    assert list(am) == [1.5, 0.25]
+
+
+def test_bf16_conversion_is_exact():
+    bits = np.array([0x3F80, 0xC000, 0x3E80, 0x0001], np.uint16)   # 1, -2, 0.25, tiny
+    f = O.to_f32(bits, "bf16")
+    assert list(f[:3]) == [1.0, -2.0, 0.25]
+    assert f[3] == np.float32(2.0 ** -133)
