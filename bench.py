@@ -1,0 +1,546 @@
+"""Throughput of the Q4 paged KV-cache path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl q4kv|reference]
+
+One step is one pass of the whole path over one batch of synthetic input:
+for every layer, quantise all K/V tokens into the paged 4-bit pool (K
+Walsh-Hadamard rotated), apply the workload's eviction / mixed-width steps,
+then run split-K paged GQA decode attention for the batch.  The default
+workload is the Gemma-3-12B-shaped 5-agent cache (48 layers, 16 query / 8
+KV heads, head_dim 256, 5 x 8192 tokens, bf16 input).
+
+Printed (rank 0, one JSON line): value = algorithmic HBM bytes of the whole
+step (quantise: read K/V, write codes + scale/zero; decode: read codes +
+scale/zero + mask of every live block) / step time, in GB/s, summed over
+ranks; per-kernel CUDA-event times; the roofline of the dominant kernel; an
+end-to-end number through host buffers; the CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Q4 paged decode-attn HBM GB/s (% of ~8 TB/s), KV tokens/s; quantize GB/s"
+
+
+# ---------------------------------------------------------------------------
+# workload description (shared by both arms)
+# ---------------------------------------------------------------------------
+
+def workload_by_name(name):
+    from decode_attention_q4kv_b200 import workloads as W
+    if name.startswith("sweep:"):
+        _, b, c = name.split(":")
+        return W.sweep_point(int(b), int(c))
+    aliases = {"gemma": W.GEMMA3_12B, "tiny": W.TINY, "mixed": W.LLAMA31_8B_MIXED,
+               "evict": W.QWEN25_14B_EVICT}
+    if name in aliases:
+        return aliases[name]
+    return W.WORKLOADS[name]
+
+
+def bytes_per_layer(w):
+    """Algorithmic HBM bytes of one layer: (quantise, decode)."""
+    in_elem = 2
+    vec = w.head_dim
+    ng = vec // 64
+    n_tok = w.prefill_tokens or w.n_tokens
+    q4_row = vec // 2 + ng * 4          # codes + (scale, zero) of one (token, head), one tensor
+    q8_row = vec + ng * 4
+    n_q8 = w.n_q8_blocks
+    n_blocks = w.n_blocks
+    frac8 = n_q8 / n_blocks if n_blocks else 0.0
+    row = (1 - frac8) * q4_row + frac8 * q8_row
+    quant = n_tok * w.n_kv_heads * (2 * vec * in_elem + 2 * row)
+    if w.q8_fraction:
+        quant += n_tok * w.n_kv_heads * vec * in_elem        # mean |K| pass reads K once more
+    dec_tok = w.batch * w.ctx
+    decode = dec_tok * w.n_kv_heads * 2 * row + n_blocks * 32 + w.batch * w.blocks_per_seq * 4
+    decode += w.batch * w.n_q_heads * vec * (in_elem + 4)
+    return quant, decode
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """Polls NVML during the timed region (SM clock, throttle reasons)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index, period_s=0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = None
+            props = torch.cuda.get_device_properties(index)
+            try:       # CUDA and NVML number devices differently: match by UUID
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:        # no NVML: report that instead of clocks
+            self.nvml, self.error = None, repr(e)
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def result(self):
+        if not self.nvml:
+            return {"error": self.error}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons)}
+
+
+class Job:
+    """All layers of one workload resident on one GPU, ready to step."""
+
+    def __init__(self, w, device, rank=0, layers=None):
+        import torch
+
+        import decode_attention_q4kv_b200 as q4
+        from decode_attention_q4kv_b200 import workloads as W
+
+        self.w, self.dev, self.torch, self.q4 = w, device, torch, q4
+        self.n_layers = layers or w.layers
+        n_tok = w.prefill_tokens or w.n_tokens
+        n_pool = max(w.n_blocks, n_tok // 256) if w.permuted_pool else w.n_blocks
+        self.n_q8 = w.n_q8_blocks
+        self.n_q4 = n_pool - self.n_q8
+        self.layers = []
+        for l in range(self.n_layers):
+            lid = l + 1000 * rank
+            k, v = W.kv_tokens(w, lid, n_tok, device)
+            q = W.query(w, lid, device)
+            pool = q4.Q4KVPool(w.n_kv_heads, w.head_dim, self.n_q4, self.n_q8, device=device)
+            self.layers.append(dict(k=k, v=v, q=q, pool=pool,
+                                    out=torch.empty((w.batch, w.n_q_heads, w.head_dim),
+                                                    dtype=torch.float16, device=device)))
+        if w.permuted_pool:
+            self.tables = W.permuted_tables(w).to(device)
+            self.prefill_ids = torch.arange(n_tok // 256, dtype=torch.int32, device=device)
+        else:
+            self.tables = W.identity_tables(w).to(device)
+            self.prefill_ids = None
+        self.ids = self.tables.reshape(-1).contiguous()
+        self.lens = W.seq_lens(w).to(device)
+        self.evict = W.evicted_slot_ids(w, W.identity_tables(w)).to(device) if w.evict_fraction else None
+        self.plan = q4.DecodePlan(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.blocks_per_seq)
+        self.ws = self.plan.workspace(device)
+        if w.permuted_pool:
+            # fill the whole pool once by tiling the quantised prefill (setup, not timed)
+            for L in self.layers:
+                L["pool"].quantize(L["k"], L["v"], self.prefill_ids)
+                self._tile(L["pool"], n_tok // 256)
+        self.quant_bytes, self.decode_bytes = bytes_per_layer(w)
+        self.launches_per_layer = 1 + 1 + (1 if self.plan.n_splits > 1 else 0)
+        if w.q8_fraction:
+            self.launches_per_layer += 3
+        if self.evict is not None:
+            self.launches_per_layer += 1
+
+    def _tile(self, pool, n_src):
+        for name in ("k_codes4", "v_codes4", "k_params4", "v_params4"):
+            t = getattr(pool, name)
+            for s in range(n_src, t.shape[0], n_src):
+                e = min(s + n_src, t.shape[0])
+                t[s:e].copy_(t[: e - s])
+
+    def quantize_layer(self, L):
+        w, q4 = self.w, self.q4
+        if w.q8_fraction:
+            am = q4.block_absmean(L["k"])
+            ids = q4.mixed_block_ids(am, self.n_q8, 0, self.n_q4)
+        elif self.prefill_ids is not None:
+            ids = self.prefill_ids
+        else:
+            ids = self.ids
+        L["pool"].quantize(L["k"], L["v"], ids)
+        if self.evict is not None:
+            L["pool"].invalidate(self.evict)
+
+    def decode_layer(self, L):
+        self.q4.decode_attention(L["pool"], L["q"], self.tables, self.lens, plan=self.plan,
+                                 workspace=self.ws, out=L["out"])
+
+    def step(self, events=None):
+        for L in self.layers:
+            if events is not None:
+                e0, e1, e2 = events.pop()
+                e0.record()
+            self.quantize_layer(L)
+            if events is not None:
+                e1.record()
+            self.decode_layer(L)
+            if events is not None:
+                e2.record()
+
+    @property
+    def bytes_per_step(self):
+        return self.n_layers * (self.quant_bytes + self.decode_bytes)
+
+
+def sources_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decode_attention_q4kv_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key, launches_scale=1.0):
+    """DRAM bytes per launch from the committed ncu summary, if the sources still match."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except OSError:
+        return None
+    ent = t.get(kernel_key)
+    if not ent or ent.get("sources") != sources_digest():
+        return None
+    return ent["dram_bytes_per_launch"] * launches_scale
+
+
+def measured_peak(key, fallback):
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            v = json.load(f).get(key)
+        if v:
+            return float(v), "measured"
+    except OSError:
+        pass
+    return fallback, "fallback"
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = workload_by_name(args.workload)
+    job = Job(w, dev, rank, args.layers)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        job.step()
+    torch.cuda.synchronize()
+
+    # timed region: K steps, events around every quantise and decode launch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+          for _ in range(args.steps * job.n_layers)]
+    todo = list(reversed(ev))
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for _ in range(args.steps):
+            job.step(todo)
+        stop.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = start.elapsed_time(stop) / 1e3
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    q_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    d_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+
+    # decode alone over all layers, cold (each layer's pool untouched for a full sweep)
+    reps = max(3, min(20, args.steps))
+    cold = []
+    for _ in range(reps):
+        for L in job.layers:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            job.decode_layer(L)
+            b.record()
+            cold.append((a, b))
+    torch.cuda.synchronize()
+    d_cold_ms = statistics.median(a.elapsed_time(b) for a, b in cold)
+
+    e2e = run_e2e(job, args, dev, world) if not args.no_e2e else None
+    if world > 1:
+        dist.barrier()
+
+    if rank == 0:
+        peak, peak_src = measured_peak("hbm_gbs", 6650.0)
+        q_gbps = job.quant_bytes / (q_ms * 1e-3) / 1e9
+        d_gbps = job.decode_bytes / (d_ms * 1e-3) / 1e9
+        d_cold_gbps = job.decode_bytes / (d_cold_ms * 1e-3) / 1e9
+        kv_tok = w.batch * w.ctx * w.n_kv_heads
+        dominant = "quantize" if q_ms >= d_ms else "decode"
+        if dominant == "quantize":
+            roof = dict(bound="hbm", achieved=round(q_gbps, 1), peak=peak, unit="GB/s",
+                        frac=round(q_gbps / peak, 4),
+                        traffic=traffic_for(f"quantize:{w.name}"),
+                        kernel="quantize_kernel", algorithmic_bytes_per_launch=job.quant_bytes,
+                        us_per_launch=round(q_ms * 1e3, 2), peak_source=f"{peak_src} hbm_gbs (burst copy)")
+        else:
+            roof = dict(bound="hbm", achieved=round(d_cold_gbps, 1), peak=peak, unit="GB/s",
+                        frac=round(d_cold_gbps / peak, 4),
+                        traffic=traffic_for(f"decode:{w.name}"),
+                        kernel="decode", algorithmic_bytes_per_launch=job.decode_bytes,
+                        us_per_launch=round(d_cold_ms * 1e3, 2), peak_source=f"{peak_src} hbm_gbs (burst copy)")
+        value = world * job.bytes_per_step * args.steps / elapsed / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "layers": job.n_layers, "batch": w.batch, "ctx": w.ctx,
+                       "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                       "input_dtype": w.dtype, "storage": "int4 codes, group 64, fp16 scale+zero, 256-token blocks",
+                       "q8_fraction": w.q8_fraction, "evict_fraction": w.evict_fraction,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "decode_splits": job.plan.n_splits,
+                       "l2": "step inputs larger than L2 (%.1f GB)" % (job.bytes_per_step / 1e9)},
+            "kernels": {
+                "quantize": {"gbps": round(q_gbps, 1), "us_per_launch": round(q_ms * 1e3, 2),
+                             "bytes_per_launch": job.quant_bytes},
+                "decode": {"gbps_in_step": round(d_gbps, 1), "us_per_launch_in_step": round(d_ms * 1e3, 2),
+                           "gbps_cold": round(d_cold_gbps, 1), "us_per_launch_cold": round(d_cold_ms * 1e3, 2),
+                           "bytes_per_launch": job.decode_bytes,
+                           "kv_tokens_per_s": round(kv_tok / (d_cold_ms * 1e-3), 1),
+                           "frac_cold": round(d_cold_gbps / peak, 4)},
+            },
+            "roofline": roof,
+            "gpu_launches": job.launches_per_layer * job.n_layers * args.steps,
+            "clocks": clk.result(),
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(job, args, dev, world):
+    """Same metric through the public API from pinned host buffers, copies timed."""
+    import torch
+
+    w = job.w
+    n_ring = min(2, job.n_layers)
+    host = []
+    for i in range(n_ring):
+        L = job.layers[i]
+        host.append(dict(k=L["k"].cpu().pin_memory(), v=L["v"].cpu().pin_memory(),
+                         q=L["q"].cpu().pin_memory(),
+                         out=torch.empty(L["out"].shape, dtype=L["out"].dtype).pin_memory()))
+    steps = max(1, min(args.steps, 5))
+
+    def one_step():
+        for li, L in enumerate(job.layers):
+            H = host[li % n_ring]
+            L["k"].copy_(H["k"], non_blocking=True)
+            L["v"].copy_(H["v"], non_blocking=True)
+            L["q"].copy_(H["q"], non_blocking=True)
+            job.quantize_layer(L)
+            job.decode_layer(L)
+            H["out"].copy_(L["out"], non_blocking=True)
+
+    one_step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one_step()
+    b.record()
+    torch.cuda.synchronize()
+    el = a.elapsed_time(b) / 1e3
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([el], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        el = float(t.item())
+    L0 = job.layers[0]
+    h2d = job.n_layers * sum(L0[x].numel() * L0[x].element_size() for x in ("k", "v", "q"))
+    d2h = job.n_layers * L0["out"].numel() * L0["out"].element_size()
+    return {"value": round(world * job.bytes_per_step * steps / el / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "note": "inputs copied from pinned host memory and the fp16 output read back, per layer, inside the timed region"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, kv_heads=1, layer=0):
+    """One bounded sample: one layer, `kv_heads` KV heads, all sessions, on the host.
+
+    Quantises every token of those heads and decodes every query head that
+    reads them, with the oracle as it stands.  Returns (seconds, algorithmic
+    bytes of the sample).
+    """
+    import numpy as np
+    import torch
+
+    from decode_attention_q4kv_b200 import workloads as W
+    from oracle import q4kv_oracle as O
+
+    n_tok = w.prefill_tokens or w.n_tokens
+    k, v = W.kv_tokens(w, layer, n_tok, "cpu")
+    q = W.query(w, layer, "cpu")
+    k, v = k[:, :kv_heads].contiguous(), v[:, :kv_heads].contiguous()
+    g = w.gqa
+    q = q[:, : kv_heads * g].contiguous()
+
+    def host(t):
+        if t.dtype == torch.float16:
+            return t.numpy(), "fp16"
+        return t.view(torch.int16).numpy().view(np.uint16), "bf16"
+
+    kh, dt = host(k)
+    vh, _ = host(v)
+    qh, _ = host(q)
+    nb = w.n_blocks
+    n_q8 = w.n_q8_blocks
+    t0 = time.perf_counter()
+    if w.q8_fraction:
+        ids = O.mixed_block_ids(O.block_absmean(kh, dt), n_q8, 0, nb - n_q8)
+    else:
+        ids = np.arange(-(-n_tok // 256))
+    pool = O.OraclePool(kv_heads, w.head_dim, nb - n_q8, n_q8)
+    pool.quantize_blocks(kh, vh, dt, ids)
+    if w.evict_fraction:
+        tabs = W.identity_tables(w)
+        slots = W.evicted_slot_ids(w, tabs)
+        pool.invalidate_slots(slots.tolist())
+    tables = np.asarray(ids, np.int64).reshape(w.batch, -1) if not w.permuted_pool else \
+        (W.permuted_tables(w).numpy() % (n_tok // 256))
+    O.decode_attention(pool, qh, dt, tables, [w.ctx] * w.batch)
+    secs = time.perf_counter() - t0
+    frac = kv_heads / w.n_kv_heads
+    qb, db = bytes_per_layer(w)
+    return secs, (qb + db) * frac
+
+
+def cpu_baseline(w, target_s=15.0):
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(limits=1):
+        secs, nbytes = oracle_sample(w, kv_heads=1)
+        heads, total_s, total_b = 1, secs, nbytes
+        while total_s < target_s * 0.5 and heads < w.n_kv_heads:
+            s2, b2 = oracle_sample(w, kv_heads=1, layer=heads)
+            total_s += s2
+            total_b += b2
+            heads += 1
+    return {"value": round(total_b / total_s / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{heads} x (one layer, one KV head of {w.n_kv_heads}: quantise all "
+                      f"{w.prefill_tokens or w.n_tokens} tokens + decode the {w.gqa} query heads "
+                      f"of all {w.batch} sessions); numpy/BLAS limited to 1 thread",
+            "seconds": round(total_s, 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_limits
+
+    w = workload_by_name(args.workload)
+    with threadpool_limits(limits=1):
+        for i in range(args.warmup):
+            oracle_sample(w, kv_heads=1, layer=i)
+        secs, nbytes = 0.0, 0.0
+        for i in range(args.steps):
+            s, b = oracle_sample(w, kv_heads=1, layer=args.warmup + i)
+            secs += s
+            nbytes += b
+    value = nbytes / secs / 1e9
+    line = {"metric": METRIC, "value": round(value, 5), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "layers": w.layers, "batch": w.batch, "ctx": w.ctx,
+                       "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                       "input_dtype": w.dtype},
+            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": "each step: one layer, one KV head (all tokens quantised, "
+                                       "its query heads decoded), numpy/BLAS limited to 1 thread"},
+            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="q4kv", choices=["q4kv", "reference"])
+    ap.add_argument("--workload", default="gemma")
+    ap.add_argument("--layers", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)      # timing rule: at least 3 untimed steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

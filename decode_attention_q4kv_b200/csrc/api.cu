@@ -1,0 +1,271 @@
+// Host side of the C ABI declared in include/q4kv.h: argument checks, launch
+// plans and dispatch to the kernels.  Every check happens before any CUDA
+// call, so a rejected call touches no device.
+#include <math.h>
+#include <string.h>
+
+#include "q4kv_internal.cuh"
+
+using namespace q4kv;
+
+namespace {
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+q4kv_status check_pool(const q4kv_pool* p) {
+  if (p == nullptr) return Q4KV_ERR_INVALID_ARG;
+  if (p->reserved != 0 || p->n_kv_heads < 1 || p->n_q4_blocks < 0 || p->n_q8_blocks < 0 ||
+      (p->k_rotated != 0 && p->k_rotated != 1))
+    return Q4KV_ERR_INVALID_ARG;
+  if (p->head_dim != 128 && p->head_dim != 256) return Q4KV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(p->n_q4_blocks) + p->n_q8_blocks > (int64_t{1} << 31) / kBlockTokens)
+    return Q4KV_ERR_INVALID_ARG;
+  if (p->n_q4_blocks > 0) {
+    const void* a[4] = {p->k_codes4, p->v_codes4, p->k_params4, p->v_params4};
+    for (const void* x : a)
+      if (x == nullptr || !aligned(x, 16)) return Q4KV_ERR_INVALID_ARG;
+  }
+  if (p->n_q8_blocks > 0) {
+    const void* a[4] = {p->k_codes8, p->v_codes8, p->k_params8, p->v_params8};
+    for (const void* x : a)
+      if (x == nullptr || !aligned(x, 16)) return Q4KV_ERR_INVALID_ARG;
+  }
+  if (p->n_q4_blocks + p->n_q8_blocks > 0 &&
+      (p->remap_mask == nullptr || !aligned(p->remap_mask, 16)))
+    return Q4KV_ERR_INVALID_ARG;
+  if (p->error_word != nullptr && !aligned(p->error_word, 4)) return Q4KV_ERR_INVALID_ARG;
+  return Q4KV_OK;
+}
+
+q4kv_status check_input(const void* x, int32_t dtype, int64_t n_tokens, int64_t stride,
+                        int32_t hkv, int32_t d) {
+  if (dtype != Q4KV_F16 && dtype != Q4KV_BF16) return Q4KV_ERR_INVALID_ARG;
+  if (n_tokens < 0 || stride < static_cast<int64_t>(hkv) * d) return Q4KV_ERR_INVALID_ARG;
+  if ((stride * 2) % 16 != 0) return Q4KV_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (x == nullptr || !aligned(x, 16))) return Q4KV_ERR_INVALID_ARG;
+  return Q4KV_OK;
+}
+
+q4kv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? Q4KV_OK : Q4KV_ERR_CUDA; }
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char* q4kv_status_string(q4kv_status s) {
+  switch (s) {
+    case Q4KV_OK: return "ok";
+    case Q4KV_ERR_INVALID_ARG: return "invalid argument";
+    case Q4KV_ERR_UNSUPPORTED: return "unsupported shape";
+    case Q4KV_ERR_CUDA: return "CUDA error";
+    case Q4KV_ERR_WORKSPACE: return "workspace missing or too small";
+    case Q4KV_ERR_DEVICE: return "device reported an error";
+  }
+  return "unknown status";
+}
+
+int32_t q4kv_abi_version(void) { return Q4KV_ABI_VERSION; }
+
+q4kv_status q4kv_pool_array_bytes(int32_t head_dim, int32_t n_kv_heads, int64_t n_blocks,
+                                  int32_t bits, size_t* codes_bytes, size_t* params_bytes) {
+  if (codes_bytes == nullptr || params_bytes == nullptr || n_kv_heads < 1 || n_blocks < 0 ||
+      (bits != 4 && bits != 8))
+    return Q4KV_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return Q4KV_ERR_UNSUPPORTED;
+  const size_t rows = static_cast<size_t>(n_blocks) * n_kv_heads * kBlockTokens;
+  *codes_bytes = rows * head_dim * bits / 8;
+  *params_bytes = rows * (head_dim / kGroup) * 4;
+  return Q4KV_OK;
+}
+
+q4kv_status q4kv_quantize_blocks(const q4kv_pool* pool, const void* k, const void* v,
+                                 int32_t in_dtype, int64_t n_tokens, int64_t token_stride,
+                                 const int32_t* block_ids, void* stream) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  st = check_input(k, in_dtype, n_tokens, token_stride, pool->n_kv_heads, pool->head_dim);
+  if (st != Q4KV_OK) return st;
+  st = check_input(v, in_dtype, n_tokens, token_stride, pool->n_kv_heads, pool->head_dim);
+  if (st != Q4KV_OK) return st;
+  if (n_tokens == 0) return Q4KV_OK;
+  if (block_ids == nullptr || !aligned(block_ids, 4)) return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_quantize(view_of(*pool), k, v, in_dtype, n_tokens, token_stride,
+                                   block_ids, as_stream(stream)));
+}
+
+q4kv_status q4kv_dequantize(const q4kv_pool* pool, const int32_t* block_ids, int32_t n_blocks,
+                            void* k_out, void* v_out, int32_t out_dtype, int32_t unrotate_k,
+                            void* stream) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  if (n_blocks < 0 || (out_dtype != Q4KV_F32 && out_dtype != Q4KV_F16) ||
+      (unrotate_k != 0 && unrotate_k != 1))
+    return Q4KV_ERR_INVALID_ARG;
+  if (n_blocks == 0) return Q4KV_OK;
+  if (block_ids == nullptr || k_out == nullptr || v_out == nullptr || !aligned(block_ids, 4) ||
+      !aligned(k_out, 16) || !aligned(v_out, 16))
+    return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_dequantize(view_of(*pool), block_ids, n_blocks, k_out, v_out,
+                                     out_dtype, unrotate_k, as_stream(stream)));
+}
+
+q4kv_status q4kv_invalidate_slots(const q4kv_pool* pool, const int64_t* slot_ids, int64_t n_slots,
+                                  void* stream) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  if (n_slots < 0) return Q4KV_ERR_INVALID_ARG;
+  if (n_slots == 0) return Q4KV_OK;
+  if (slot_ids == nullptr || !aligned(slot_ids, 8)) return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_invalidate(view_of(*pool), slot_ids, n_slots, as_stream(stream)));
+}
+
+q4kv_status q4kv_block_absmean(const void* k, int32_t in_dtype, int64_t n_tokens,
+                               int64_t token_stride, int32_t n_kv_heads, int32_t head_dim,
+                               double* out, void* stream) {
+  if (n_kv_heads < 1 || head_dim < 1 || (static_cast<int64_t>(n_kv_heads) * head_dim) % 8 != 0)
+    return Q4KV_ERR_INVALID_ARG;
+  q4kv_status st = check_input(k, in_dtype, n_tokens, token_stride, n_kv_heads, head_dim);
+  if (st != Q4KV_OK) return st;
+  if (n_tokens == 0) return Q4KV_OK;
+  if (out == nullptr || !aligned(out, 8)) return Q4KV_ERR_INVALID_ARG;
+  if ((n_tokens + kBlockTokens - 1) / kBlockTokens > 0x7fffffff) return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(
+      launch_absmean(k, in_dtype, n_tokens, token_stride, n_kv_heads, head_dim, out, as_stream(stream)));
+}
+
+q4kv_status q4kv_mixed_block_ids(const double* absmean, int32_t n_chunks, int32_t n_q8,
+                                 int32_t q4_first, int32_t q8_first, int32_t* block_ids,
+                                 void* stream) {
+  if (n_chunks < 0 || n_chunks > 65536 || n_q8 < 0 || n_q8 > n_chunks || q4_first < 0 ||
+      q8_first < 0)
+    return Q4KV_ERR_INVALID_ARG;
+  if (n_chunks == 0) return Q4KV_OK;
+  if (absmean == nullptr || block_ids == nullptr || !aligned(absmean, 8) || !aligned(block_ids, 4))
+    return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_mixed_ids(absmean, n_chunks, n_q8, q4_first, q8_first, block_ids,
+                                    as_stream(stream)));
+}
+
+q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                  int32_t head_dim, int32_t max_blocks_per_seq, int32_t n_splits,
+                                  int32_t num_sms, q4kv_decode_plan* plan) {
+  if (plan == nullptr || batch < 0 || n_q_heads < 1 || n_kv_heads < 1 ||
+      max_blocks_per_seq < 1 || n_splits < 0 || num_sms < 0 || n_q_heads % n_kv_heads != 0)
+    return Q4KV_ERR_INVALID_ARG;
+  if (batch > 65535 || n_kv_heads > 65535) return Q4KV_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens > 0x7fffffff)
+    return Q4KV_ERR_INVALID_ARG;
+  const int g = n_q_heads / n_kv_heads;
+  if (head_dim != 128 && head_dim != 256) return Q4KV_ERR_UNSUPPORTED;
+  if (g > 8 || g * head_dim / kGroup > 16) return Q4KV_ERR_UNSUPPORTED;
+  if (num_sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return Q4KV_ERR_CUDA;
+  }
+  const int64_t ctx = static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens;
+  const int64_t max_splits = (ctx + 63) / 64;
+  int64_t s = n_splits;
+  if (s == 0) {
+    const int64_t pairs = static_cast<int64_t>(batch > 0 ? batch : 1) * n_kv_heads;
+    const int64_t target = static_cast<int64_t>(num_sms) * 16;   // CTAs worth launching
+    s = (target + pairs - 1) / pairs;
+    const int64_t min_tokens = 256;                             // keep partials a small share
+    const int64_t cap = (ctx + min_tokens - 1) / min_tokens;
+    if (s > cap) s = cap;
+  }
+  if (s < 1) s = 1;
+  if (s > max_splits) s = max_splits;
+  if (s > 65535) s = 65535;
+  int64_t tps = (ctx + s - 1) / s;
+  tps = (tps + 63) / 64 * 64;
+  s = (ctx + tps - 1) / tps;
+  memset(plan, 0, sizeof(*plan));
+  plan->batch = batch;
+  plan->n_q_heads = n_q_heads;
+  plan->n_kv_heads = n_kv_heads;
+  plan->head_dim = head_dim;
+  plan->max_blocks_per_seq = max_blocks_per_seq;
+  plan->n_splits = static_cast<int32_t>(s);
+  plan->tokens_per_split = static_cast<int32_t>(tps);
+  plan->kernel = 0;
+  if (s > 1) {
+    const size_t rows = static_cast<size_t>(batch) * n_q_heads * s;
+    plan->workspace_bytes = round_up(rows * head_dim * sizeof(float), 256) + round_up(rows * 2 * sizeof(float), 256);
+  }
+  return Q4KV_OK;
+}
+
+q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan* plan,
+                                  const void* q, int32_t q_dtype, const int32_t* block_tables,
+                                  const int32_t* seq_lens, float softmax_scale, void* out,
+                                  int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  if (plan == nullptr) return Q4KV_ERR_INVALID_ARG;
+  // the plan must be one q4kv_decode_plan_make would produce for this pool
+  q4kv_decode_plan ref;
+  st = q4kv_decode_plan_make(plan->batch, plan->n_q_heads, plan->n_kv_heads, plan->head_dim,
+                             plan->max_blocks_per_seq, plan->n_splits, 1, &ref);
+  if (st != Q4KV_OK) return st;
+  if (plan->head_dim != pool->head_dim || plan->n_kv_heads != pool->n_kv_heads ||
+      ref.n_splits != plan->n_splits || ref.tokens_per_split != plan->tokens_per_split ||
+      ref.workspace_bytes != plan->workspace_bytes)
+    return Q4KV_ERR_INVALID_ARG;
+  if ((q_dtype != Q4KV_F16 && q_dtype != Q4KV_BF16) ||
+      (out_dtype != Q4KV_F32 && out_dtype != Q4KV_F16 && out_dtype != Q4KV_BF16) ||
+      !isfinite(softmax_scale))
+    return Q4KV_ERR_INVALID_ARG;
+  if (plan->batch == 0) return Q4KV_OK;
+  if (q == nullptr || block_tables == nullptr || seq_lens == nullptr || out == nullptr ||
+      !aligned(q, 16) || !aligned(block_tables, 16) || !aligned(seq_lens, 4) || !aligned(out, 16))
+    return Q4KV_ERR_INVALID_ARG;
+  if (pool->n_q4_blocks + pool->n_q8_blocks == 0) return Q4KV_ERR_INVALID_ARG;
+  if (plan->workspace_bytes > 0 &&
+      (workspace == nullptr || workspace_bytes < plan->workspace_bytes || !aligned(workspace, 256)))
+    return Q4KV_ERR_WORKSPACE;
+  DecodeArgs a;
+  a.pool = view_of(*pool);
+  a.plan = *plan;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(plan->head_dim));
+  a.out = out;
+  a.out_dtype = out_dtype;
+  const size_t rows = static_cast<size_t>(plan->batch) * plan->n_q_heads * plan->n_splits;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_ml = plan->workspace_bytes > 0
+                ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                           round_up(rows * plan->head_dim * sizeof(float), 256))
+                : nullptr;
+  return from_cuda(launch_decode(a, as_stream(stream)));
+}
+
+q4kv_status q4kv_read_device_error(const q4kv_pool* pool, uint32_t* bits, int32_t clear,
+                                   void* stream) {
+  if (pool == nullptr || bits == nullptr) return Q4KV_ERR_INVALID_ARG;
+  *bits = 0;
+  if (pool->error_word == nullptr) return Q4KV_OK;
+  cudaStream_t s = as_stream(stream);
+  uint32_t host = 0;
+  if (cudaMemcpyAsync(&host, pool->error_word, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return Q4KV_ERR_CUDA;
+  if (clear && host != 0) {
+    if (cudaMemsetAsync(pool->error_word, 0, sizeof(uint32_t), s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return Q4KV_ERR_CUDA;
+  }
+  *bits = host;
+  return host != 0 ? Q4KV_ERR_DEVICE : Q4KV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,325 @@
+// Split-K paged GQA decode attention over the packed 4/8-bit cache.
+//
+// "Agent Memory Below the Prompt" (arXiv 2603.04428 summary), sec. 2.1
+// item 2: attention reads the quantised cache directly ("direct restore");
+// item 3: one batched pass over many agents' caches; sec. 2.2: GQA.
+// IntentKV article (Qiita), "詰め直さずに「無効化」する": remapped slots
+// get logit -1e4 and contribute no value.
+//
+// Grid: (split, KV head, sequence).  A CTA owns the g query heads that share
+// one KV head and one token range of one sequence; it keeps a running max and
+// sum per head (online softmax) and writes either the final row (one split)
+// or a partial (o, max, sum) merged afterwards by log-sum-exp.
+#include <math.h>
+
+#include "q4kv_internal.cuh"
+
+namespace q4kv {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTile = 128;   // tokens per iteration: one token per thread in the key pass
+constexpr int kMaxG = 8;
+
+__device__ __forceinline__ float load_in(const void* p, int dtype, int64_t i) {
+  return dtype == Q4KV_F16 ? __half2float(static_cast<const __half*>(p)[i])
+                           : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+__device__ __forceinline__ void store_out(void* p, int dtype, int64_t i, float x) {
+  if (dtype == Q4KV_F32) static_cast<float*>(p)[i] = x;
+  else if (dtype == Q4KV_F16) static_cast<__half*>(p)[i] = __float2half_rn(x);
+  else static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(x);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_simple_kernel(const DecodeArgs a) {
+  constexpr int NG = D / kGroup;
+  constexpr int CP = D / 2;              // channel pairs, one per thread in the value pass
+  constexpr int NPH = kThreads / CP;     // token phases in the value pass (2 or 1)
+  __shared__ float qs[kMaxG][D];
+  __shared__ float lg[kMaxG][kTile];     // logits, then value weights
+  __shared__ int32_t tok_blk[kTile];     // unified block id of a live token, -1 otherwise
+  __shared__ int32_t tok_slot[kTile];
+  __shared__ float m_run[kMaxG], l_run[kMaxG], alpha[kMaxG];
+  __shared__ float ored[kMaxG][D];
+  __shared__ int poison;
+
+  const PoolView& P = a.pool;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int hq = a.plan.n_q_heads, g = hq / P.n_kv_heads;
+  const int S = a.plan.n_splits, tps = a.plan.tokens_per_split, mb = a.plan.max_blocks_per_seq;
+  const int seq = a.seq_lens[b];
+  const bool bad_seq = seq < 0 || seq > mb * kBlockTokens;
+  if (bad_seq && split == 0 && kvh == 0 && tid == 0) raise_error(P.error_word, Q4KV_DEVERR_SEQ_LEN);
+
+  for (int i = tid; i < g * D; i += kThreads) {
+    const int h = i / D, j = i % D;
+    qs[h][j] = load_in(a.q, a.q_dtype, (static_cast<int64_t>(b) * hq + kvh * g + h) * D + j);
+  }
+  if (tid < kMaxG) {
+    m_run[tid] = -INFINITY;
+    l_run[tid] = 0.0f;
+  }
+  if (tid == 0) poison = bad_seq ? 1 : 0;
+  __syncthreads();
+  if (P.k_rotated) {   // q_rot = c * H q, any summation order (fp32)
+    for (int hs = 1; hs < D; hs <<= 1) {
+      for (int i = tid; i < g * (D / 2); i += kThreads) {
+        const int h = i / (D / 2), p = i % (D / 2);
+        const int lo = (p / hs) * 2 * hs + (p % hs), hi = lo + hs;
+        const float x = qs[h][lo], y = qs[h][hi];
+        qs[h][lo] = x + y;
+        qs[h][hi] = x - y;
+      }
+      __syncthreads();
+    }
+    const float c = rotation_constant(D);
+    for (int i = tid; i < g * D; i += kThreads) qs[i / D][i % D] *= c;
+    __syncthreads();
+  }
+
+  const int t_begin = split * tps;
+  const int t_end = bad_seq ? t_begin : min(t_begin + tps, seq);
+  const int cp = tid % CP, ph = tid / CP;
+  float o0[kMaxG], o1[kMaxG];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) o0[h] = o1[h] = 0.0f;
+
+  for (int tile0 = t_begin; tile0 < t_end; tile0 += kTile) {
+    // ---- key pass: one token per thread ----
+    const int t = tile0 + tid;
+    bool present = t < t_end;
+    int32_t blk = -1;
+    int slot = t % kBlockTokens;
+    if (present) {
+      blk = a.tables[static_cast<int64_t>(b) * mb + t / kBlockTokens];
+      if (blk < 0 || blk >= P.n_q4 + P.n_q8) {
+        raise_error(P.error_word, Q4KV_DEVERR_BLOCK_ID);
+        poison = 1;
+        present = false;
+      }
+    }
+    bool masked = false;
+    if (present)
+      masked = (P.mask[static_cast<int64_t>(blk) * kMaskWords + slot / 32] >> (slot % 32)) & 1u;
+    if (present && !masked) {
+      float acc[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.0f;
+      const bool is8 = blk >= P.n_q4;
+      const int64_t phys = is8 ? blk - P.n_q4 : blk;
+      const int64_t row = (phys * P.n_kv_heads + kvh) * kBlockTokens + slot;
+      const __half2* par = (is8 ? P.k_params8 : P.k_params4) + row * NG;
+#pragma unroll 1
+      for (int gr = 0; gr < NG; ++gr) {
+        const float s = __low2float(par[gr]), z = __high2float(par[gr]);
+#pragma unroll 2
+        for (int j8 = 0; j8 < kGroup; j8 += 8) {
+          const int j0 = gr * kGroup + j8;
+          uint32_t w0, w1 = 0;
+          if (is8) {
+            const uint2 u = *reinterpret_cast<const uint2*>(P.k_codes8 + row * D + j0);
+            w0 = u.x;
+            w1 = u.y;
+          } else {
+            w0 = *reinterpret_cast<const uint32_t*>(P.k_codes4 + row * (D / 2) + j0 / 2);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t c = is8 ? ((e < 4 ? w0 : w1) >> (8 * (e % 4))) & 255u : (w0 >> (4 * e)) & 15u;
+            const float kv = __fmaf_rn(static_cast<float>(c), s, z);
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h)
+              if (h < g) acc[h] = fmaf(qs[h][j0 + e], kv, acc[h]);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h)
+        if (h < g) lg[h][tid] = acc[h] * a.scale;
+    } else {
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h)
+        if (h < g) lg[h][tid] = present ? Q4KV_SENTINEL_LOGIT : -INFINITY;
+    }
+    tok_blk[tid] = (present && !masked) ? blk : -1;
+    tok_slot[tid] = slot;
+    __syncthreads();
+
+    // ---- online softmax: warp w updates heads w, w+4 ----
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int h = warp; h < g; h += kThreads / 32) {
+        float v[kTile / 32];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kTile / 32; ++q) {
+          v[q] = lg[h][lane + 32 * q];
+          mx = fmaxf(mx, v[q]);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_old = m_run[h];
+        const float m_new = fmaxf(m_old, mx);
+        float al = 1.0f, sum = 0.0f;
+        if (m_new != -INFINITY) {
+          al = m_old == -INFINITY ? 0.0f : expf(m_old - m_new);
+#pragma unroll
+          for (int q = 0; q < kTile / 32; ++q) {
+            v[q] = v[q] == -INFINITY ? 0.0f : expf(v[q] - m_new);
+            sum += v[q];
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < kTile / 32; ++q) v[q] = 0.0f;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+#pragma unroll
+        for (int q = 0; q < kTile / 32; ++q)
+          lg[h][lane + 32 * q] = tok_blk[lane + 32 * q] >= 0 ? v[q] : 0.0f;
+        if (lane == 0) {
+          l_run[h] = l_run[h] * al + sum;
+          m_run[h] = m_new;
+          alpha[h] = al;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- value pass: one channel pair per thread ----
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < g) {
+        o0[h] *= alpha[h];
+        o1[h] *= alpha[h];
+      }
+    }
+    const int n_in_tile = min(kTile, t_end - tile0);
+    for (int tt = ph; tt < n_in_tile; tt += NPH) {
+      const int32_t vb = tok_blk[tt];
+      if (vb < 0) continue;
+      const bool is8 = vb >= P.n_q4;
+      const int64_t phys = is8 ? vb - P.n_q4 : vb;
+      const int64_t row = (phys * P.n_kv_heads + kvh) * kBlockTokens + tok_slot[tt];
+      const __half2 pr = (is8 ? P.v_params8 : P.v_params4)[row * NG + (2 * cp) / kGroup];
+      const float s = __low2float(pr), z = __high2float(pr);
+      uint32_t c0, c1;
+      if (is8) {
+        const uint32_t two = *reinterpret_cast<const uint16_t*>(P.v_codes8 + row * D + 2 * cp);
+        c0 = two & 255u;
+        c1 = two >> 8;
+      } else {
+        const uint32_t byte = P.v_codes4[row * (D / 2) + cp];
+        c0 = byte & 15u;
+        c1 = byte >> 4;
+      }
+      const float v0 = __fmaf_rn(static_cast<float>(c0), s, z);
+      const float v1 = __fmaf_rn(static_cast<float>(c1), s, z);
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h < g) {
+          const float w = lg[h][tt];
+          o0[h] = fmaf(w, v0, o0[h]);
+          o1[h] = fmaf(w, v1, o1[h]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // combine the token phases
+  if (NPH > 1) {
+    if (ph == 1) {
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h < g) {
+          ored[h][2 * cp] = o0[h];
+          ored[h][2 * cp + 1] = o1[h];
+        }
+      }
+    }
+    __syncthreads();
+    if (ph == 0) {
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h < g) {
+          o0[h] += ored[h][2 * cp];
+          o1[h] += ored[h][2 * cp + 1];
+        }
+      }
+    }
+  }
+  if (ph != 0) return;
+  const bool poisoned = poison != 0;
+  for (int h = 0; h < g; ++h) {
+    const int64_t qrow = static_cast<int64_t>(b) * hq + kvh * g + h;
+    if (S == 1) {
+      const float l = l_run[h];
+      const float inv = (!poisoned && l > 0.0f) ? 1.0f / l : 0.0f;
+      store_out(a.out, a.out_dtype, qrow * D + 2 * cp, poisoned ? 0.0f : o0[h] * inv);
+      store_out(a.out, a.out_dtype, qrow * D + 2 * cp + 1, poisoned ? 0.0f : o1[h] * inv);
+    } else {
+      float* po = a.ws_o + (qrow * S + split) * D;
+      po[2 * cp] = o0[h];
+      po[2 * cp + 1] = o1[h];
+      if (cp == 0) {
+        a.ws_ml[(qrow * S + split) * 2] = m_run[h];
+        a.ws_ml[(qrow * S + split) * 2 + 1] = poisoned ? -1.0f : l_run[h];
+      }
+    }
+  }
+}
+
+// Log-sum-exp merge of the splits of one (sequence, query head) row:
+//   M = max m_i, L = sum l_i e^(m_i - M), out = sum o_i e^(m_i - M) / L.
+// A poisoned split (l < 0) or an empty row (M = -inf) gives 0.
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
+  const int64_t row = blockIdx.x;
+  const int S = a.plan.n_splits;
+  const float* ml = a.ws_ml + row * S * 2;
+  float M = -INFINITY;
+  bool poisoned = false;
+  for (int i = 0; i < S; ++i) {
+    M = fmaxf(M, ml[2 * i]);
+    poisoned |= ml[2 * i + 1] < 0.0f;
+  }
+  for (int j = threadIdx.x; j < D; j += blockDim.x) {
+    float res = 0.0f;
+    if (!poisoned && M != -INFINITY) {
+      float num = 0.0f, den = 0.0f;
+      for (int i = 0; i < S; ++i) {
+        const float m = ml[2 * i];
+        if (m == -INFINITY) continue;
+        const float w = expf(m - M);
+        den = fmaf(ml[2 * i + 1], w, den);
+        num = fmaf(a.ws_o[(row * S + i) * D + j], w, num);
+      }
+      res = num / den;
+    }
+    store_out(a.out, a.out_dtype, row * D + j, res);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  const q4kv_decode_plan& p = a.plan;
+  const dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
+  if (p.head_dim == 128)
+    decode_simple_kernel<128><<<grid, kThreads, 0, stream>>>(a);
+  else
+    decode_simple_kernel<256><<<grid, kThreads, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_splits == 1) return e;
+  const unsigned rows = static_cast<unsigned>(p.batch) * p.n_q_heads;
+  if (p.head_dim == 128)
+    merge_kernel<128><<<rows, 128, 0, stream>>>(a);
+  else
+    merge_kernel<256><<<rows, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace q4kv

@@ -1,0 +1,107 @@
+// Internal declarations shared by the CUDA translation units of libq4kv.
+// Nothing here is part of the C ABI (include/q4kv.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "q4kv.h"
+
+namespace q4kv {
+
+constexpr int kBlockTokens = Q4KV_BLOCK_TOKENS;
+constexpr int kGroup = Q4KV_GROUP;
+constexpr int kMaskWords = Q4KV_MASK_WORDS;
+
+// Everything a kernel needs about the pool, passed by value.
+struct PoolView {
+  int32_t head_dim;
+  int32_t n_kv_heads;
+  int32_t k_rotated;
+  int32_t n_q4;
+  int32_t n_q8;
+  uint8_t* k_codes4;
+  uint8_t* v_codes4;
+  __half2* k_params4;
+  __half2* v_params4;
+  uint8_t* k_codes8;
+  uint8_t* v_codes8;
+  __half2* k_params8;
+  __half2* v_params8;
+  uint32_t* mask;
+  uint32_t* error_word;
+};
+
+inline PoolView view_of(const q4kv_pool& p) {
+  PoolView v;
+  v.head_dim = p.head_dim;
+  v.n_kv_heads = p.n_kv_heads;
+  v.k_rotated = p.k_rotated;
+  v.n_q4 = p.n_q4_blocks;
+  v.n_q8 = p.n_q8_blocks;
+  v.k_codes4 = p.k_codes4;
+  v.v_codes4 = p.v_codes4;
+  v.k_params4 = reinterpret_cast<__half2*>(p.k_params4);
+  v.v_params4 = reinterpret_cast<__half2*>(p.v_params4);
+  v.k_codes8 = p.k_codes8;
+  v.v_codes8 = p.v_codes8;
+  v.k_params8 = reinterpret_cast<__half2*>(p.k_params8);
+  v.v_params8 = reinterpret_cast<__half2*>(p.v_params8);
+  v.mask = p.remap_mask;
+  v.error_word = p.error_word;
+  return v;
+}
+
+__device__ __forceinline__ void raise_error(uint32_t* word, uint32_t bit) {
+  if (word != nullptr) atomicOr(word, bit);
+}
+
+// binary32 nearest to 1/sqrt(D) for the supported head sizes.
+__host__ __device__ __forceinline__ float rotation_constant(int d) {
+  return d == 256 ? 0.0625f : 0x1.6a09e6p-4f;   // 2^-4 and RN(2^-3.5)
+}
+
+// Load one element of an fp16/bf16 input as binary32 (exact).
+template <typename T>
+__device__ __forceinline__ float to_float(T x);
+template <>
+__device__ __forceinline__ float to_float<__half>(__half x) { return __half2float(x); }
+template <>
+__device__ __forceinline__ float to_float<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+// ---------------------------------------------------------------------------
+// launchers (each returns cudaGetLastError() of its launch)
+// ---------------------------------------------------------------------------
+cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, int in_dtype,
+                            int64_t n_tokens, int64_t token_stride, const int32_t* block_ids,
+                            cudaStream_t stream);
+cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,
+                              void* k_out, void* v_out, int out_dtype, int unrotate_k,
+                              cudaStream_t stream);
+cudaError_t launch_invalidate(const PoolView& pool, const int64_t* slot_ids, int64_t n,
+                              cudaStream_t stream);
+cudaError_t launch_absmean(const void* k, int in_dtype, int64_t n_tokens, int64_t token_stride,
+                           int n_kv_heads, int head_dim, double* out, cudaStream_t stream);
+cudaError_t launch_mixed_ids(const double* absmean, int32_t n, int32_t n_q8, int32_t q4_first,
+                             int32_t q8_first, int32_t* ids, cudaStream_t stream);
+
+struct DecodeArgs {
+  PoolView pool;
+  q4kv_decode_plan plan;
+  const void* q;
+  int q_dtype;
+  const int32_t* tables;
+  const int32_t* seq_lens;
+  float scale;
+  void* out;
+  int out_dtype;
+  float* ws_o;   // [B][Hq][S][D]
+  float* ws_ml;  // [B][Hq][S][2] (running max, running sum)
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace q4kv

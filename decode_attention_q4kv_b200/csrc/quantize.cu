@@ -1,0 +1,360 @@
+// Encoder and decoder of the paged 4/8-bit KV format.
+//
+// Format: "Agent Memory Below the Prompt" (arXiv 2603.04428 summary), sec. 2.1
+// item 2 -- codes packed into uint32 words, one 16-bit scale and one 16-bit
+// bias per group; keys rotated by a Walsh-Hadamard transform before coding,
+// values not (UltraQuant news item, arXiv 2606.20474, "技術/ビジネス面").
+//
+// Work mapping: a warp takes one KV head of 4 consecutive tokens (D = 128) or
+// 2 consecutive tokens (D = 256).  Each lane holds 16 consecutive channels of
+// one (token, head) vector, so the rotation runs as 4 butterfly stages inside
+// the lane followed by 3 (or 4) stages across lanes with warp shuffles, and a
+// 64-value group spans 4 lanes.  The warp's code rows are contiguous in the
+// pool (consecutive slots of one block and head), so its stores form one
+// 256-byte (Q4, D = 128) run.
+//
+// Bit-exactness: every arithmetic step is one IEEE binary32 operation written
+// with an _rn intrinsic (no contraction, no reassociation): butterflies in
+// ascending stride order, one multiply by c, exact min/max, subtraction and
+// division for the scale, fp16 round-to-nearest-even for scale and zero,
+// subtraction and division for each code, round-half-even to an integer,
+// clamp.  Dequantisation is fma(code, s, z), equal to code*s + z because the
+// product is exact.
+#include "q4kv_internal.cuh"
+
+namespace q4kv {
+namespace {
+
+constexpr int kEPL = 16;  // channels held by one lane
+
+template <int D>
+struct Shape {
+  static constexpr int LPV = D / kEPL;        // lanes per vector
+  static constexpr int VPW = 32 / LPV;        // vectors (tokens) per warp
+  static constexpr int NG = D / kGroup;       // groups per vector
+};
+
+// Unnormalised Walsh-Hadamard transform of a D-vector spread over LPV lanes
+// (lane j of the vector holds channels 16j .. 16j+15).  Stage order is
+// h = 1, 2, ..., D/2; in each stage the lower element of a pair becomes a+b
+// and the upper a-b.
+template <int D>
+__device__ __forceinline__ void fwht_vector(float (&x)[kEPL], int j) {
+#pragma unroll
+  for (int h = 1; h < kEPL; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < kEPL; ++i) {
+      if ((i & h) == 0) {
+        const float a = x[i], b = x[i + h];
+        x[i] = __fadd_rn(a, b);
+        x[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int h = kEPL; h < D; h <<= 1) {
+    const int lane_bit = h / kEPL;
+    const bool upper = (j & lane_bit) != 0;
+#pragma unroll
+    for (int i = 0; i < kEPL; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, x[i], lane_bit);
+      x[i] = upper ? __fsub_rn(other, x[i]) : __fadd_rn(x[i], other);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void rotate_vector(float (&x)[kEPL], int j) {
+  fwht_vector<D>(x, j);
+  const float c = rotation_constant(D);
+#pragma unroll
+  for (int i = 0; i < kEPL; ++i) x[i] = __fmul_rn(x[i], c);
+}
+
+template <typename T>
+__device__ __forceinline__ void load16(const T* __restrict__ src, bool valid, float (&x)[kEPL]) {
+  static_assert(sizeof(T) == 2, "16-bit inputs");
+  uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
+  if (valid) {
+    w0 = __ldg(reinterpret_cast<const uint4*>(src));
+    w1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+  }
+  const T* e0 = reinterpret_cast<const T*>(&w0);
+  const T* e1 = reinterpret_cast<const T*>(&w1);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[i] = to_float<T>(e0[i]);
+    x[8 + i] = to_float<T>(e1[i]);
+  }
+}
+
+// Encode the lane's 16 values (one quarter of a 64-value group) and store
+// codes and, from the group's first lane, its (scale, zero) pair.
+template <int BITS>
+__device__ __forceinline__ void encode_store(const float (&x)[kEPL], int j, bool valid,
+                                             uint8_t* __restrict__ code_dst,
+                                             __half2* __restrict__ param_dst) {
+  constexpr int L = (1 << BITS) - 1;
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < kEPL; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+  // the 4 lanes of a group are j = 4k .. 4k+3
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
+  mx = __fadd_rn(mx, 0.0f);
+  const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(L));
+  const __half sh = __float2half_rn(s);
+  const __half zh = __float2half_rn(mn);
+  const float sf = __half2float(sh);
+  const float zf = __half2float(zh);
+
+  uint32_t q[kEPL];
+#pragma unroll
+  for (int i = 0; i < kEPL; ++i) {
+    int r = 0;
+    if (sf != 0.0f) {
+      r = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], zf), sf));
+      r = min(max(r, 0), L);
+    }
+    q[i] = static_cast<uint32_t>(r);
+  }
+  if (!valid) return;
+  if (BITS == 4) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      lo |= q[i] << (4 * i);
+      hi |= q[8 + i] << (4 * i);
+    }
+    *reinterpret_cast<uint2*>(code_dst + j * 8) = make_uint2(lo, hi);
+  } else {
+    uint4 w;
+    w.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+    w.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
+    w.z = q[8] | (q[9] << 8) | (q[10] << 16) | (q[11] << 24);
+    w.w = q[12] | (q[13] << 8) | (q[14] << 16) | (q[15] << 24);
+    *reinterpret_cast<uint4*>(code_dst + j * 16) = w;
+  }
+  if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(sh, zh);
+}
+
+template <int D, typename InT>
+__global__ void __launch_bounds__(256) quantize_kernel(PoolView pool, const InT* __restrict__ k,
+                                                       const InT* __restrict__ v,
+                                                       int64_t n_tokens, int64_t stride,
+                                                       const int32_t* __restrict__ block_ids,
+                                                       int64_t n_items) {
+  using S = Shape<D>;
+  const int lane = threadIdx.x & 31;
+  const int r = lane / S::LPV;
+  const int j = lane % S::LPV;
+  const int hkv = pool.n_kv_heads;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+
+  for (int64_t item = warp0; item < n_items; item += n_warps) {
+    const int64_t group_of_tokens = item / hkv;
+    const int h = static_cast<int>(item - group_of_tokens * hkv);
+    const int64_t t0 = group_of_tokens * S::VPW;
+    const int64_t t = t0 + r;
+    const bool valid = t < n_tokens;
+    const int32_t blk = __ldg(block_ids + t0 / kBlockTokens);
+    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+      if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const int slot = static_cast<int>(t % kBlockTokens);
+    const bool is8 = blk >= pool.n_q4;
+    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+    const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
+
+    float x[kEPL];
+    const int64_t src = t * stride + static_cast<int64_t>(h) * D + j * kEPL;
+    // keys: rotate, then code
+    load16<InT>(k + (valid ? src : 0), valid, x);
+    if (pool.k_rotated) rotate_vector<D>(x, j);
+    if (is8)
+      encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
+    else
+      encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
+    // values: code unrotated
+    load16<InT>(v + (valid ? src : 0), valid, x);
+    if (is8)
+      encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+    else
+      encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+    // a freshly written slot is live
+    if (valid && h == 0 && j == 0)
+      atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32,
+                ~(1u << (slot % 32)));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dequantisation
+// ---------------------------------------------------------------------------
+
+template <int BITS>
+__device__ __forceinline__ void decode_lane(const uint8_t* __restrict__ codes,
+                                            const __half2* __restrict__ params, int j,
+                                            float (&x)[kEPL]) {
+  const __half2 p = params[j >> 2];
+  const float s = __low2float(p);
+  const float z = __high2float(p);
+  uint32_t w[4];
+  if (BITS == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(codes + j * 8);
+    w[0] = u.x;
+    w[1] = u.y;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[i] = __fmaf_rn(static_cast<float>((w[0] >> (4 * i)) & 15u), s, z);
+      x[8 + i] = __fmaf_rn(static_cast<float>((w[1] >> (4 * i)) & 15u), s, z);
+    }
+  } else {
+    const uint4 u = *reinterpret_cast<const uint4*>(codes + j * 16);
+    w[0] = u.x;
+    w[1] = u.y;
+    w[2] = u.z;
+    w[3] = u.w;
+#pragma unroll
+    for (int i = 0; i < kEPL; ++i)
+      x[i] = __fmaf_rn(static_cast<float>((w[i / 4] >> (8 * (i % 4))) & 255u), s, z);
+  }
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store16(OutT* dst, const float (&x)[kEPL]);
+template <>
+__device__ __forceinline__ void store16<float>(float* dst, const float (&x)[kEPL]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+template <>
+__device__ __forceinline__ void store16<__half>(__half* dst, const float (&x)[kEPL]) {
+  __align__(16) __half h[kEPL];
+#pragma unroll
+  for (int i = 0; i < kEPL; ++i) h[i] = __float2half_rn(x[i]);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = reinterpret_cast<const uint4*>(h)[0];
+  d[1] = reinterpret_cast<const uint4*>(h)[1];
+}
+
+template <int D, typename OutT>
+__global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
+                                                         const int32_t* __restrict__ block_ids,
+                                                         OutT* __restrict__ k_out,
+                                                         OutT* __restrict__ v_out, int unrotate_k,
+                                                         int64_t n_items) {
+  using S = Shape<D>;
+  const int lane = threadIdx.x & 31;
+  const int r = lane / S::LPV;
+  const int j = lane % S::LPV;
+  const int hkv = pool.n_kv_heads;
+  constexpr int kQuads = kBlockTokens / S::VPW;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+
+  for (int64_t item = warp0; item < n_items; item += n_warps) {
+    // item = ((list index * Hkv) + head) * kQuads + quad
+    const int quad = static_cast<int>(item % kQuads);
+    const int64_t bh = item / kQuads;
+    const int h = static_cast<int>(bh % hkv);
+    const int64_t li = bh / hkv;
+    const int slot = quad * S::VPW + r;
+    const int64_t out_row = (li * hkv + h) * kBlockTokens + slot;
+    OutT* kd = k_out + out_row * D + j * kEPL;
+    OutT* vd = v_out + out_row * D + j * kEPL;
+    const int32_t blk = __ldg(block_ids + li);
+    float x[kEPL];
+    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+      if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
+#pragma unroll
+      for (int i = 0; i < kEPL; ++i) x[i] = 0.0f;
+      store16<OutT>(kd, x);
+      store16<OutT>(vd, x);
+      continue;
+    }
+    const bool is8 = blk >= pool.n_q4;
+    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+    const int64_t row = (phys * hkv + h) * kBlockTokens + slot;
+    const bool masked =
+        (pool.mask[static_cast<int64_t>(blk) * kMaskWords + slot / 32] >> (slot % 32)) & 1u;
+
+    if (is8)
+      decode_lane<8>(pool.k_codes8 + row * D, pool.k_params8 + row * S::NG, j, x);
+    else
+      decode_lane<4>(pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG, j, x);
+    if (unrotate_k && pool.k_rotated) rotate_vector<D>(x, j);
+    if (masked) {
+#pragma unroll
+      for (int i = 0; i < kEPL; ++i) x[i] = Q4KV_SENTINEL_LOGIT;
+    }
+    store16<OutT>(kd, x);
+
+    if (is8)
+      decode_lane<8>(pool.v_codes8 + row * D, pool.v_params8 + row * S::NG, j, x);
+    else
+      decode_lane<4>(pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG, j, x);
+    if (masked) {
+#pragma unroll
+      for (int i = 0; i < kEPL; ++i) x[i] = 0.0f;
+    }
+    store16<OutT>(vd, x);
+  }
+}
+
+inline int grid_for(int64_t n_items) {
+  const int64_t warps_per_cta = 8;
+  int64_t g = (n_items + warps_per_cta - 1) / warps_per_cta;
+  if (g > (1 << 30)) g = 1 << 30;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, int in_dtype,
+                            int64_t n_tokens, int64_t token_stride, const int32_t* block_ids,
+                            cudaStream_t stream) {
+  const int d = pool.head_dim;
+  const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;
+  const int64_t n_items = ((n_tokens + vpw - 1) / vpw) * pool.n_kv_heads;
+  const dim3 grid(grid_for(n_items)), block(256);
+#define Q4KV_LAUNCH_Q(DD, T)                                                          \
+  quantize_kernel<DD, T><<<grid, block, 0, stream>>>(pool, static_cast<const T*>(k),  \
+                                                     static_cast<const T*>(v), n_tokens, \
+                                                     token_stride, block_ids, n_items)
+  if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(128, __half);
+  else if (d == 128) Q4KV_LAUNCH_Q(128, __nv_bfloat16);
+  else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(256, __half);
+  else Q4KV_LAUNCH_Q(256, __nv_bfloat16);
+#undef Q4KV_LAUNCH_Q
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,
+                              void* k_out, void* v_out, int out_dtype, int unrotate_k,
+                              cudaStream_t stream) {
+  const int d = pool.head_dim;
+  const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;
+  const int64_t n_items = static_cast<int64_t>(n_blocks) * pool.n_kv_heads * (kBlockTokens / vpw);
+  const dim3 grid(grid_for(n_items)), block(256);
+#define Q4KV_LAUNCH_D(DD, T)                                                            \
+  dequantize_kernel<DD, T><<<grid, block, 0, stream>>>(pool, block_ids, static_cast<T*>(k_out), \
+                                                       static_cast<T*>(v_out), unrotate_k, n_items)
+  if (d == 128 && out_dtype == Q4KV_F32) Q4KV_LAUNCH_D(128, float);
+  else if (d == 128) Q4KV_LAUNCH_D(128, __half);
+  else if (out_dtype == Q4KV_F32) Q4KV_LAUNCH_D(256, float);
+  else Q4KV_LAUNCH_D(256, __half);
+#undef Q4KV_LAUNCH_D
+  return cudaGetLastError();
+}
+
+}  // namespace q4kv

@@ -1,0 +1,262 @@
+/*
+ * q4kv.h -- C ABI of the B200 (sm_100a) 4-bit paged KV cache and its decode
+ * attention.
+ *
+ * Source pages (cited by title and section):
+ *   [AMBP] "Agent Memory Below the Prompt: Persistent Q4 KV Cache for
+ *          Multi-Agent LLM Inference on Edge Devices" (gist.science summary of
+ *          arXiv 2603.04428).  Sec. 2.1 item 1: 256-token blocks per agent.
+ *          Sec. 2.1 item 2: 4-bit codes packed in uint32 words, one 16-bit
+ *          scale and one 16-bit bias per group, read by attention directly
+ *          ("direct restore").  Sec. 2.1 item 3: attention batched over many
+ *          agents' quantised caches.  Sec. 2.2: GQA.
+ *   [UQ]   UltraQuant news item (poko-everyday.com, arXiv 2606.20474),
+ *          section "技術/ビジネス面": Walsh-Hadamard rotation before 4-bit
+ *          quantisation; keys and values treated asymmetrically.
+ *   [IKV]  IntentKV article (Qiita), section "詰め直さずに「無効化」する":
+ *          evicted slots are re-pointed to a sentinel slot with key -1e4,
+ *          whose softmax weight is zero; surviving slots do not move.
+ *   [QKVS] QKVShare (gist.science summary of arXiv 2605.03884),
+ *          "Méthodologie": per-token widths from {2, 4, 8, FP16}; the
+ *          receiver dequantises the shared cache before use.
+ *
+ * Format (fixed by this library):
+ *   - 256 tokens per block; one block holds every KV head of those tokens.
+ *   - Groups of 64 consecutive values along head_dim of one (token, head)
+ *     vector; per group an fp16 scale s and an fp16 zero z (additive offset);
+ *     value = code * s + z.
+ *   - K is stored rotated by c*H_D (Sylvester Walsh-Hadamard, c = binary32
+ *     nearest 1/sqrt(D), butterfly strides 1, 2, ..., D/2 in that order);
+ *     V is stored unrotated.  The query is rotated by the same transform
+ *     inside attention, so no inverse rotation is needed on the output.
+ *   - 4-bit codes: two per byte, element 2i in the low nibble of byte i
+ *     (element j of a little-endian uint32 word at bits 4*(j%8)).
+ *     8-bit codes: one per byte.
+ *   - Codes are computed from the stored fp16 s and z:
+ *       s = fl((max - min) / L), L = 15 or 255;  z = fp16(min)
+ *       code = 0 if fp16(s) == 0 else clamp(rne(fl(fl(x - z) / s)), 0, L)
+ *     with binary32 IEEE subtraction and division (bit-exact everywhere).
+ *   - An evicted slot is flagged in a per-block 256-bit mask shared by all
+ *     KV heads; its data stays in place.  Attention gives it logit -1e4 and
+ *     value 0, so its weight is exactly 0 whenever any live logit exceeds
+ *     -9896; a sequence whose every slot is evicted returns 0.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates or frees device memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns without waiting, except q4kv_read_device_error.
+ *   - Arguments are checked on the host first; on any failure the call
+ *     returns an error status and launches nothing.
+ *   - Faults found on the device (an out-of-range block id in a table or a
+ *     block-id list, an out-of-range slot id, a sequence length beyond its
+ *     table) never trap: the offending item is skipped, the affected output
+ *     row is written as 0, and a Q4KV_DEVERR_* bit is OR-ed into
+ *     pool->error_word when that pointer is non-NULL.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef Q4KV_H
+#define Q4KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define Q4KV_ABI_VERSION 1
+#define Q4KV_BLOCK_TOKENS 256
+#define Q4KV_GROUP 64
+#define Q4KV_MASK_WORDS 8            /* uint32 words of remap mask per block */
+#define Q4KV_SENTINEL_LOGIT (-1.0e4f)
+
+typedef enum {
+  Q4KV_OK = 0,
+  Q4KV_ERR_INVALID_ARG = 1,   /* NULL pointer, negative size, misaligned pointer or stride, bad dtype */
+  Q4KV_ERR_UNSUPPORTED = 2,   /* well-formed but outside what the kernels cover (head_dim, GQA ratio) */
+  Q4KV_ERR_CUDA = 3,          /* a CUDA runtime call or a kernel launch failed */
+  Q4KV_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than plan->workspace_bytes */
+  Q4KV_ERR_DEVICE = 5         /* q4kv_read_device_error found device error bits set */
+} q4kv_status;
+
+/* Bits of pool->error_word. */
+#define Q4KV_DEVERR_BLOCK_ID 1u  /* a block id outside [0, n_q4_blocks + n_q8_blocks) */
+#define Q4KV_DEVERR_SEQ_LEN 2u   /* seq_len < 0 or > max_blocks_per_seq * 256 */
+#define Q4KV_DEVERR_SLOT_ID 4u   /* a slot id outside [0, 256 * (n_q4_blocks + n_q8_blocks)) */
+#define Q4KV_DEVERR_TIMEOUT 8u   /* a bounded device-side wait gave up */
+
+typedef enum { Q4KV_F16 = 0, Q4KV_BF16 = 1, Q4KV_F32 = 2 } q4kv_dtype;
+
+/*
+ * The paged pool ([AMBP] sec. 2.1 items 1-2; 8-bit blocks: [QKVS]).
+ * Unified block ids: [0, n_q4_blocks) are 4-bit blocks, stored at index id
+ * of the *4 arrays; [n_q4_blocks, n_q4_blocks + n_q8_blocks) are 8-bit blocks,
+ * stored at index id - n_q4_blocks of the *8 arrays.
+ * Every array pointer must be 16-byte aligned.  Layouts (row-major):
+ *   k_codes4, v_codes4   uint8 [n_q4][Hkv][256][D/2]
+ *   k_params4, v_params4 half2 [n_q4][Hkv][256][D/64]   (.x = scale, .y = zero)
+ *   k_codes8, v_codes8   uint8 [n_q8][Hkv][256][D]      (may be NULL if n_q8 == 0)
+ *   k_params8, v_params8 half2 [n_q8][Hkv][256][D/64]
+ *   remap_mask           uint32 [n_q4 + n_q8][8]; bit (s % 32) of word s / 32
+ *                        set = slot s of that block is remapped to the sentinel
+ *   error_word           optional uint32 (NULL = do not report)
+ * The descriptor itself is read on the host during each call and may be
+ * reused or freed afterwards.
+ */
+typedef struct {
+  int32_t head_dim;     /* D: 128 or 256 */
+  int32_t n_kv_heads;   /* Hkv >= 1 */
+  int32_t k_rotated;    /* 1 = K stored Walsh-Hadamard rotated ([UQ]); 0 = raw */
+  int32_t n_q4_blocks;  /* >= 0 */
+  int32_t n_q8_blocks;  /* >= 0 */
+  int32_t reserved;     /* must be 0 */
+  uint8_t *k_codes4, *v_codes4;
+  void *k_params4, *v_params4;
+  uint8_t *k_codes8, *v_codes8;
+  void *k_params8, *v_params8;
+  uint32_t *remap_mask;
+  uint32_t *error_word;
+} q4kv_pool;
+
+/* Human-readable name of a status code (static storage). */
+const char *q4kv_status_string(q4kv_status status);
+
+/* Q4KV_ABI_VERSION of the loaded library. */
+int32_t q4kv_abi_version(void);
+
+/*
+ * Bytes of one codes array and of one params array for `n_blocks` blocks of
+ * width `bits` (4 or 8), so a caller can size the pool ([AMBP] sec. 2.1
+ * item 2: 144 bytes per token and KV head at D = 128, 4 bits, i.e. 71.875 %
+ * below fp16).  Host-only; touches no device.
+ */
+q4kv_status q4kv_pool_array_bytes(int32_t head_dim, int32_t n_kv_heads, int64_t n_blocks,
+                                  int32_t bits, size_t *codes_bytes, size_t *params_bytes);
+
+/*
+ * Quantise and store K/V of `n_tokens` tokens ([AMBP] sec. 2.1 item 2, [UQ]).
+ *   k, v         device, dtype in_dtype (Q4KV_F16 or Q4KV_BF16); element
+ *                (t, h, j) at index t*token_stride + h*D + j; 16-byte aligned;
+ *                token_stride >= Hkv*D and token_stride*elem_size % 16 == 0.
+ *                Values must be finite.
+ *   block_ids    device int32 [ceil(n_tokens/256)]: token t is written to
+ *                block block_ids[t/256], slot t % 256 (4- or 8-bit per the id).
+ *   Writing a slot clears its remap bit (a freshly written slot is live).
+ *   Codes, scales, zeros and packed bytes are bit-identical to the format's
+ *   definition above.  n_tokens == 0 is a no-op.  A block id out of range
+ *   skips its tokens and raises Q4KV_DEVERR_BLOCK_ID.
+ */
+q4kv_status q4kv_quantize_blocks(const q4kv_pool *pool, const void *k, const void *v,
+                                 int32_t in_dtype, int64_t n_tokens, int64_t token_stride,
+                                 const int32_t *block_ids, void *stream);
+
+/*
+ * Dequantise whole blocks ([QKVS] "Méthodologie": dequantise before use).
+ *   block_ids    device int32 [n_blocks]
+ *   k_out, v_out device [n_blocks][Hkv][256][D] of out_dtype (Q4KV_F32 or
+ *                Q4KV_F16), 16-byte aligned; value = fl(code*s + z), fp16
+ *                output rounds that to nearest even.
+ *   unrotate_k   1 = apply c*H (its own inverse) to K after dequantisation,
+ *                with the same butterfly order as the encoder (bit-exact).
+ *   Remapped slots read the sentinel: K = -1e4 in every channel, V = 0.
+ *   A block id out of range writes zeros for that block and raises
+ *   Q4KV_DEVERR_BLOCK_ID.
+ */
+q4kv_status q4kv_dequantize(const q4kv_pool *pool, const int32_t *block_ids, int32_t n_blocks,
+                            void *k_out, void *v_out, int32_t out_dtype, int32_t unrotate_k,
+                            void *stream);
+
+/*
+ * Remap slots to the sentinel ([IKV]): sets their remap bits; data stays in
+ * place and positions do not change.
+ *   slot_ids     device int64 [n_slots], slot = block_id*256 + offset.
+ *   Out-of-range ids are skipped and raise Q4KV_DEVERR_SLOT_ID.
+ */
+q4kv_status q4kv_invalidate_slots(const q4kv_pool *pool, const int64_t *slot_ids, int64_t n_slots,
+                                  void *stream);
+
+/*
+ * Mean |K| of each 256-token chunk of raw (unrotated) keys, accumulated in
+ * fp64 ([QKVS]: choose wider codes for the most demanding blocks).
+ *   k            as in q4kv_quantize_blocks (same layout and alignment rules)
+ *   out          device double [ceil(n_tokens/256)]; a short last chunk is
+ *                averaged over its own tokens.
+ */
+q4kv_status q4kv_block_absmean(const void *k, int32_t in_dtype, int64_t n_tokens,
+                               int64_t token_stride, int32_t n_kv_heads, int32_t head_dim,
+                               double *out, void *stream);
+
+/*
+ * Block ids for a mixed 4/8-bit cache: the n_q8 chunks of highest absmean
+ * (ties to the lower chunk index) get 8-bit ids, the rest 4-bit ids, each in
+ * chunk order: the k-th 8-bit chunk gets q8_first + k, the k-th 4-bit chunk
+ * q4_first + k.  absmean and block_ids are device arrays of n_chunks
+ * entries; 0 <= n_q8 <= n_chunks <= 65536.
+ */
+q4kv_status q4kv_mixed_block_ids(const double *absmean, int32_t n_chunks, int32_t n_q8,
+                                 int32_t q4_first, int32_t q8_first, int32_t *block_ids,
+                                 void *stream);
+
+/*
+ * Launch plan of one decode-attention shape.  The context of every sequence
+ * is cut into n_splits ranges of tokens_per_split tokens; each range yields a
+ * partial (max, sum, weighted value) per query head, merged by log-sum-exp.
+ */
+typedef struct {
+  int32_t batch;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t max_blocks_per_seq;  /* width of the block table */
+  int32_t n_splits;
+  int32_t tokens_per_split;    /* multiple of 64 */
+  int32_t kernel;              /* kernel variant chosen for this shape (informational) */
+  size_t workspace_bytes;      /* device scratch the call needs (0 when n_splits == 1) */
+} q4kv_decode_plan;
+
+/*
+ * Fill `plan` for a shape.  n_splits > 0 forces that split count (clamped to
+ * the context); 0 lets the library choose from num_sms.  num_sms > 0 is used
+ * as given; 0 queries the current CUDA device.  Host-only otherwise.
+ * Supported: head_dim 128 or 256, 1 <= n_q_heads / n_kv_heads <= 8 and
+ * (n_q_heads / n_kv_heads) * head_dim / 64 <= 16.
+ */
+q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                  int32_t head_dim, int32_t max_blocks_per_seq, int32_t n_splits,
+                                  int32_t num_sms, q4kv_decode_plan *plan);
+
+/*
+ * Single-token paged GQA decode attention over the quantised cache
+ * ([AMBP] sec. 2.1 items 2-3 and 2.2; [IKV] for remapped slots).
+ *   q            device [batch][n_q_heads][D], q_dtype Q4KV_F16 or Q4KV_BF16
+ *   block_tables device int32 [batch][max_blocks_per_seq]
+ *   seq_lens     device int32 [batch], 0 <= seq_len <= max_blocks_per_seq*256
+ *   softmax_scale  <= 0 selects 1/sqrt(D)
+ *   out          device [batch][n_q_heads][D] of out_dtype (F32, F16 or BF16)
+ *   workspace    device scratch of at least plan->workspace_bytes (may be
+ *                NULL when that is 0), 256-byte aligned, not shared with a
+ *                concurrent call.
+ * Query head h reads KV head h / (n_q_heads / n_kv_heads).  Logits are
+ * softmax_scale * <c*H q, K_hat> (or <q, K_hat> when K is stored raw); an
+ * empty or fully remapped sequence returns 0.
+ */
+q4kv_status q4kv_decode_attention(const q4kv_pool *pool, const q4kv_decode_plan *plan,
+                                  const void *q, int32_t q_dtype, const int32_t *block_tables,
+                                  const int32_t *seq_lens, float softmax_scale, void *out,
+                                  int32_t out_dtype, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
+ * Wait for `stream`, read pool->error_word into *bits, and zero it when
+ * `clear` is nonzero.  Returns Q4KV_ERR_DEVICE when any bit was set,
+ * Q4KV_OK otherwise (and *bits = 0 when pool->error_word is NULL).
+ */
+q4kv_status q4kv_read_device_error(const q4kv_pool *pool, uint32_t *bits, int32_t clear,
+                                   void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4KV_H */

@@ -1,0 +1,167 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports
+every function include/q4kv.h declares, sizes the pool as the format says,
+makes launch plans, and rejects bad arguments before touching a device."""
+import ctypes
+
+import pytest
+
+from decode_attention_q4kv_b200 import _lib
+
+L = _lib.lib()
+FAKE = 0x7F0000000000     # 4 KiB-aligned address never dereferenced: every call below is rejected first
+
+
+def _pool(**kw):
+    d = dict(head_dim=128, n_kv_heads=8, k_rotated=1, n_q4_blocks=4, n_q8_blocks=0, reserved=0,
+             k_codes4=FAKE, v_codes4=FAKE, k_params4=FAKE, v_params4=FAKE,
+             k_codes8=0, v_codes8=0, k_params8=0, v_params8=0, remap_mask=FAKE, error_word=0)
+    d.update(kw)
+    p = _lib.PoolDesc()
+    for k, v in d.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_exports_every_declared_function():
+    names = _lib.header_functions()
+    assert len(names) == 11
+    for n in names:
+        assert hasattr(L, n), n
+    # the binding declares a signature for each of them
+    assert set(names) == set(_lib._SIGNATURES)
+
+
+def test_abi_version_and_status_strings():
+    assert L.q4kv_abi_version() == 1
+    assert L.q4kv_status_string(0) == b"ok"
+    assert b"workspace" in L.q4kv_status_string(_lib.ERR_WORKSPACE)
+    assert L.q4kv_status_string(99) == b"unknown status"
+
+
+def test_struct_layouts():
+    assert ctypes.sizeof(_lib.PoolDesc) == 24 + 10 * 8
+    assert _lib.PoolDesc.k_codes4.offset == 24
+    assert ctypes.sizeof(_lib.DecodePlan) == 40
+
+
+def test_pool_array_bytes_give_144_bytes_per_token_head():
+    cb, pb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.q4kv_pool_array_bytes(128, 1, 1, 4, ctypes.byref(cb), ctypes.byref(pb)) == 0
+    assert (cb.value, pb.value) == (256 * 64, 256 * 2 * 4)
+    per_token_head = 2 * (cb.value + pb.value) / 256
+    assert per_token_head == 144
+    assert L.q4kv_pool_array_bytes(128, 1, 1, 8, ctypes.byref(cb), ctypes.byref(pb)) == 0
+    assert 2 * (cb.value + pb.value) / 256 == 272
+    assert L.q4kv_pool_array_bytes(256, 1, 1, 4, ctypes.byref(cb), ctypes.byref(pb)) == 0
+    assert 2 * (cb.value + pb.value) / 256 == 288
+    assert L.q4kv_pool_array_bytes(96, 1, 1, 4, ctypes.byref(cb), ctypes.byref(pb)) == _lib.ERR_UNSUPPORTED
+    assert L.q4kv_pool_array_bytes(128, 1, 1, 3, ctypes.byref(cb), ctypes.byref(pb)) == _lib.ERR_INVALID_ARG
+
+
+def _plan(*args):
+    p = _lib.DecodePlan()
+    st = L.q4kv_decode_plan_make(*args, ctypes.byref(p))
+    return st, p
+
+
+@pytest.mark.parametrize("B,hq,hkv,d,mb", [(1, 32, 8, 128, 16), (64, 32, 8, 128, 512),
+                                           (5, 16, 8, 256, 32), (32, 40, 8, 128, 64),
+                                           (256, 32, 8, 128, 512), (1, 8, 8, 128, 1)])
+def test_plan_covers_context(B, hq, hkv, d, mb):
+    st, p = _plan(B, hq, hkv, d, mb, 0, 148)
+    assert st == 0
+    ctx = mb * 256
+    assert p.tokens_per_split % 64 == 0 and p.tokens_per_split >= 64
+    assert p.n_splits * p.tokens_per_split >= ctx > (p.n_splits - 1) * p.tokens_per_split
+    if p.n_splits > 1:
+        assert p.workspace_bytes >= B * hq * p.n_splits * (d + 2) * 4
+    else:
+        assert p.workspace_bytes == 0
+    # forcing the plan's own split count reproduces it
+    st2, p2 = _plan(B, hq, hkv, d, mb, p.n_splits, 7)
+    assert st2 == 0 and (p2.n_splits, p2.tokens_per_split, p2.workspace_bytes) == \
+        (p.n_splits, p.tokens_per_split, p.workspace_bytes)
+
+
+def test_plan_rejects_bad_shapes():
+    assert _plan(1, 30, 8, 128, 4, 0, 148)[0] == _lib.ERR_INVALID_ARG      # Hq % Hkv != 0
+    assert _plan(1, 72, 8, 128, 4, 0, 148)[0] == _lib.ERR_UNSUPPORTED      # g = 9
+    assert _plan(1, 48, 8, 256, 4, 0, 148)[0] == _lib.ERR_UNSUPPORTED      # g*D/64 = 24
+    assert _plan(1, 32, 8, 64, 4, 0, 148)[0] == _lib.ERR_UNSUPPORTED       # D = 64
+    assert _plan(1, 32, 8, 128, 0, 0, 148)[0] == _lib.ERR_INVALID_ARG      # empty table
+    assert _plan(-1, 32, 8, 128, 4, 0, 148)[0] == _lib.ERR_INVALID_ARG
+    st, p = _plan(1, 32, 8, 128, 4, 100000, 148)                            # clamped to the context
+    assert st == 0 and p.n_splits == 16 and p.tokens_per_split == 64
+
+
+def test_quantize_rejects_bad_arguments_without_launching():
+    p = _pool()
+    q = L.q4kv_quantize_blocks
+    assert q(None, FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert q(ctypes.byref(_pool(head_dim=64)), FAKE, FAKE, 0, 10, 512, FAKE, None) == _lib.ERR_UNSUPPORTED
+    assert q(ctypes.byref(p), FAKE, FAKE, 2, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG       # fp32 input
+    assert q(ctypes.byref(p), FAKE + 2, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG   # misaligned
+    assert q(ctypes.byref(p), FAKE, FAKE, 0, 10, 1000, FAKE, None) == _lib.ERR_INVALID_ARG       # stride < Hkv*D
+    assert q(ctypes.byref(p), FAKE, FAKE, 0, 10, 1028, FAKE, None) == _lib.ERR_INVALID_ARG       # stride not 16 B
+    assert q(ctypes.byref(p), FAKE, FAKE, 0, -1, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert q(ctypes.byref(p), FAKE, FAKE, 0, 10, 1024, None, None) == _lib.ERR_INVALID_ARG       # no block ids
+    assert q(ctypes.byref(_pool(reserved=1)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert q(ctypes.byref(_pool(k_codes4=0)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert q(ctypes.byref(_pool(n_q8_blocks=2)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert q(ctypes.byref(_pool(remap_mask=FAKE + 4)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
+    # zero tokens is a no-op that succeeds
+    assert q(ctypes.byref(p), FAKE, FAKE, 0, 0, 1024, FAKE, None) == 0
+
+
+def test_other_entry_points_reject_bad_arguments():
+    p = _pool()
+    assert L.q4kv_dequantize(ctypes.byref(p), FAKE, 2, FAKE, FAKE, 1, 2, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_dequantize(ctypes.byref(p), FAKE, 2, FAKE, FAKE, 1, 0, None) == _lib.ERR_INVALID_ARG  # bf16 out
+    assert L.q4kv_dequantize(ctypes.byref(p), FAKE, 2, FAKE + 8, FAKE, 2, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_dequantize(ctypes.byref(p), FAKE, 0, FAKE, FAKE, 2, 0, None) == 0
+    assert L.q4kv_invalidate_slots(ctypes.byref(p), FAKE, -1, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_invalidate_slots(ctypes.byref(p), None, 3, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_invalidate_slots(ctypes.byref(p), FAKE, 0, None) == 0
+    assert L.q4kv_block_absmean(FAKE, 0, 10, 1000, 1, 3, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_block_absmean(FAKE, 0, 10, 1028, 8, 128, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_block_absmean(FAKE, 0, 0, 1024, 8, 128, FAKE, None) == 0
+    assert L.q4kv_mixed_block_ids(FAKE, 70000, 1, 0, 0, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_mixed_block_ids(FAKE, 10, 11, 0, 0, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_mixed_block_ids(FAKE, 0, 0, 0, 0, FAKE, None) == 0
+
+
+def test_decode_rejects_bad_arguments_without_launching():
+    p = _pool()
+    st, plan = _plan(2, 32, 8, 128, 4, 4, 148)
+    assert st == 0 and plan.workspace_bytes > 0
+    d = L.q4kv_decode_attention
+    args = lambda **kw: dict(dict(q=FAKE, qd=0, tab=FAKE, lens=FAKE, scale=0.0, out=FAKE, od=1,
+                                  ws=FAKE, wsb=plan.workspace_bytes), **kw)
+
+    def call(pool=p, pl=plan, **kw):
+        a = args(**kw)
+        return d(ctypes.byref(pool), ctypes.byref(pl), a["q"], a["qd"], a["tab"], a["lens"], a["scale"],
+                 a["out"], a["od"], a["ws"], a["wsb"], None)
+
+    assert call(ws=0) == _lib.ERR_WORKSPACE
+    assert call(wsb=plan.workspace_bytes - 1) == _lib.ERR_WORKSPACE
+    assert call(ws=FAKE + 16) == _lib.ERR_WORKSPACE
+    assert call(qd=2) == _lib.ERR_INVALID_ARG
+    assert call(od=7) == _lib.ERR_INVALID_ARG
+    assert call(q=FAKE + 2) == _lib.ERR_INVALID_ARG
+    assert call(scale=float("nan")) == _lib.ERR_INVALID_ARG
+    assert call(pool=_pool(n_kv_heads=4)) == _lib.ERR_INVALID_ARG       # plan and pool disagree
+    bad = _lib.DecodePlan.from_buffer_copy(plan)
+    bad.tokens_per_split += 64
+    assert call(pl=bad) == _lib.ERR_INVALID_ARG                          # not a plan the library made
+    st, empty = _plan(0, 32, 8, 128, 4, 0, 148)
+    assert st == 0
+    assert call(pl=empty, ws=0, wsb=0) == 0                              # batch 0: nothing to do
+
+
+def test_read_device_error_without_word():
+    p = _pool()
+    bits = ctypes.c_uint32(123)
+    assert L.q4kv_read_device_error(ctypes.byref(p), ctypes.byref(bits), 1, None) == 0
+    assert bits.value == 0
+    assert L.q4kv_read_device_error(None, ctypes.byref(bits), 1, None) == _lib.ERR_INVALID_ARG
