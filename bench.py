@@ -474,18 +474,18 @@ def oracle_sample(w, kv_heads=1, layer=0):
 
 
 def cpu_baseline(w, target_s=15.0):
+    """The oracle on a bounded sample: one-KV-head slices of successive layers until ~target_s."""
     from threadpoolctl import threadpool_limits
 
     with threadpool_limits(limits=1):
-        secs, nbytes = oracle_sample(w, kv_heads=1)
-        heads, total_s, total_b = 1, secs, nbytes
-        while total_s < target_s * 0.5 and heads < w.n_kv_heads:
-            s2, b2 = oracle_sample(w, kv_heads=1, layer=heads)
+        total_s, total_b, n = 0.0, 0.0, 0
+        while total_s < target_s and n < 4 * w.n_kv_heads:
+            s2, b2 = oracle_sample(w, kv_heads=1, layer=n)
             total_s += s2
             total_b += b2
-            heads += 1
+            n += 1
     return {"value": round(total_b / total_s / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{heads} x (one layer, one KV head of {w.n_kv_heads}: quantise all "
+            "sample": f"{n} x (one layer, one KV head of {w.n_kv_heads}: quantise all "
                       f"{w.prefill_tokens or w.n_tokens} tokens + decode the {w.gqa} query heads "
                       f"of all {w.batch} sessions); numpy/BLAS limited to 1 thread",
             "seconds": round(total_s, 2)}
