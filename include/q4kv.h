@@ -248,6 +248,38 @@ q4kv_status q4kv_decode_attention(const q4kv_pool *pool, const q4kv_decode_plan 
                                   void *stream);
 
 /*
+ * Decode attention for callers that cannot allocate device memory.
+ * (The source pages have no counterpart: this is an interface convenience.)
+ *
+ * Some callers cannot call cudaMalloc or hand the library a scratch buffer:
+ * runtimes whose device memory is owned by another allocator the library
+ * cannot reach, code with a fixed memory budget decided before it runs, or
+ * latency-critical loops where a fresh cudaMalloc would stall the device.
+ * For them this variant of q4kv_decode_attention takes the same arguments
+ * minus the workspace, and keeps its split partials in one file-scope device
+ * array of Q4KV_STATIC_SCRATCH_BYTES (16 MiB) instead.  Every GPU that loads
+ * the library holds that array until the process exits.
+ *   - A plan whose workspace_bytes exceeds Q4KV_STATIC_SCRATCH_BYTES is
+ *     rejected with Q4KV_ERR_WORKSPACE before anything runs; force fewer
+ *     splits (q4kv_decode_plan_make n_splits) or use q4kv_decode_attention.
+ *   - The first call on a device looks up the array's device address once
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - All calls share the array and it keeps the last call's contents; the
+ *     kernels overwrite every partial they later read, so nothing needs to
+ *     start at zero.  Calls that overlap on the GPU (other streams, other
+ *     host threads) race on the array and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Results equal those of q4kv_decode_attention with the same plan.
+ */
+#define Q4KV_STATIC_SCRATCH_BYTES (16u << 20)
+q4kv_status q4kv_decode_attention_static_scratch(const q4kv_pool *pool,
+                                                 const q4kv_decode_plan *plan, const void *q,
+                                                 int32_t q_dtype, const int32_t *block_tables,
+                                                 const int32_t *seq_lens, float softmax_scale,
+                                                 void *out, int32_t out_dtype, void *stream);
+
+/*
  * Wait for `stream`, read pool->error_word into *bits, and zero it when
  * `clear` is nonzero.  Returns Q4KV_ERR_DEVICE when any bit was set,
  * Q4KV_OK otherwise (and *bits = 0 when pool->error_word is NULL).

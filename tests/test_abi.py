@@ -24,7 +24,7 @@ def _pool(**kw):
 
 def test_exports_every_declared_function():
     names = _lib.header_functions()
-    assert len(names) == 11
+    assert len(names) == 12
     for n in names:
         assert hasattr(L, n), n
     # the binding declares a signature for each of them
