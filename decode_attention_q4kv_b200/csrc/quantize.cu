@@ -34,10 +34,246 @@ struct Shape {
   static constexpr int NG = D / kGroup;       // groups per vector
 };
 
-// Unnormalised Walsh-Hadamard transform of a D-vector spread over LPV lanes
-// (lane j of the vector holds channels 16j .. 16j+15).  Stage order is
-// h = 1, 2, ..., D/2; in each stage the lower element of a pair becomes a+b
-// and the upper a-b.
+// ---------------------------------------------------------------------------
+// Encoder.  A lane holds its 16 channels as 8 packed pairs: pair p = channels
+// (p, p + 8) of the lane's run, so the butterflies of strides 1, 2 and 4 pair
+// whole registers and run as packed f32x2 operations; stride 8 works inside a
+// pair.  Every packed operation is two independent binary32 operations with
+// round-to-nearest-even, identical to the scalar ones.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {   // a - b
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
+template <int D>
+__device__ __forceinline__ void fwht_pairs(float2 (&x)[8], int j) {
+  // stride 1, 2, 4: register pairs p and p + h (bit h of p clear)
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if ((p & h) == 0) {
+        const float2 a = x[p], b = x[p + h];
+        x[p] = add2(a, b);
+        x[p + h] = sub2(a, b);
+      }
+    }
+  }
+  // stride 8: channels p and p + 8 share a register pair
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const float a = x[p].x, b = x[p].y;
+    x[p].x = __fadd_rn(a, b);
+    x[p].y = __fsub_rn(a, b);
+  }
+  // strides 16 .. D/2: across lanes; fma(own, +-1, other) = other +- own exactly
+#pragma unroll
+  for (int h = kEPL; h < D; h <<= 1) {
+    const int lane_bit = h / kEPL;
+    const float sg = (j & lane_bit) ? -1.0f : 1.0f;
+    const float2 sgn = make_float2(sg, sg);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      float2 o;
+      o.x = __shfl_xor_sync(0xffffffffu, x[p].x, lane_bit);
+      o.y = __shfl_xor_sync(0xffffffffu, x[p].y, lane_bit);
+      x[p] = __ffma2_rn(x[p], sgn, o);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void rotate_pairs(float2 (&x)[8], int j) {
+  fwht_pairs<D>(x, j);
+  const float c = rotation_constant(D);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) x[p] = __fmul2_rn(x[p], make_float2(c, c));
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& w0, const uint4& w1, float2 (&x)[8]) {
+  static_assert(sizeof(T) == 2, "16-bit inputs");
+  const T* e0 = reinterpret_cast<const T*>(&w0);
+  const T* e1 = reinterpret_cast<const T*>(&w1);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) x[p] = make_float2(to_float<T>(e0[p]), to_float<T>(e1[p]));
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 1.5 * 2^23: adding it rounds |y| < 2^22 to an integer (ties to even) held in
+// the low mantissa bits.
+constexpr float kRoundMagic = 12582912.0f;
+
+// Encode the lane's 16 values (one quarter of a 64-value group) and store its
+// codes and, from the group's first lane, the group's (scale, zero).
+//
+// Codes are defined as clamp(rne(fl(fl(x - z) / s)), 0, L).  Fast path:
+// y = fl(x * r + (-z * r)) with r = fl(1/s), then k = rne(y).  With
+// |y - fl(fl(x - z)/s)| <= B = (4 (L + 1) + |z r|) 2^-24, k is the defined
+// code whenever y lies more than 2B away from a half-integer.  The fast path
+// is taken for a group only when |z r| <= 2^10 (so B < 2^-13) and every
+// value's quotient stays inside [-0.49, L + 0.49] (so no clamp is needed);
+// a lane whose values come within 2^-13 (4-bit) or 2^-12 (8-bit) of a
+// half-integer recomputes its codes with IEEE division.  Either way the codes
+// equal the definition.
+template <int BITS>
+__device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool valid,
+                                             uint8_t* __restrict__ code_dst,
+                                             __half2* __restrict__ param_dst) {
+  constexpr int L = (1 << BITS) - 1;
+  float mn = min3(min3(min3(x[0].x, x[0].y, x[1].x), min3(x[1].y, x[2].x, x[2].y),
+                       min3(x[3].x, x[3].y, x[4].x)),
+                  min3(x[4].y, x[5].x, x[5].y), min3(x[6].x, x[6].y, min(x[7].x, x[7].y)));
+  float mx = max3(max3(max3(x[0].x, x[0].y, x[1].x), max3(x[1].y, x[2].x, x[2].y),
+                       max3(x[3].x, x[3].y, x[4].x)),
+                  max3(x[4].y, x[5].x, x[5].y), max3(x[6].x, x[6].y, max(x[7].x, x[7].y)));
+  // the 4 lanes of a group are j = 4k .. 4k+3
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
+  mx = __fadd_rn(mx, 0.0f);
+  const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(L));
+  const __half sh = __float2half_rn(s);
+  const __half zh = __float2half_rn(mn);
+  const float sf = __half2float(sh);
+  const float zf = __half2float(zh);
+
+  uint32_t q[kEPL];   // code e in the low bits of q[e]; lane element e = pair e%8, half e/8
+  bool exact = true;
+  if (sf != 0.0f) {
+    const float r = __frcp_rn(sf);
+    const float nzr = __fmul_rn(-zf, r);
+    const float t_lo = __fmaf_rn(mn, r, nzr), t_hi = __fmaf_rn(mx, r, nzr);
+    exact = fabsf(nzr) > 1024.0f || t_lo < -0.49f || t_hi > L + 0.49f;
+    if (!exact) {
+      constexpr float thr = 0.5f - (BITS == 4 ? 0x1p-13f : 0x1p-12f);
+      const float2 r2 = make_float2(r, r), n2 = make_float2(nzr, nzr);
+      const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
+      const float2 mm2 = make_float2(-kRoundMagic, -kRoundMagic);
+      const float2 t2 = make_float2(-thr * thr, -thr * thr);
+      uint32_t all_neg = 0xffffffffu;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const float2 y = __ffma2_rn(x[p], r2, n2);
+        const float2 yk = __fadd2_rn(y, m2);        // integer in the low bits
+        const float2 k = __fadd2_rn(yk, mm2);       // that integer as a float
+        const float2 d = sub2(y, k);                // distance to it, |d| <= 0.5
+        const float2 e = __ffma2_rn(d, d, t2);      // < 0 iff |d| < thr
+        all_neg &= __float_as_uint(e.x) & __float_as_uint(e.y);
+        q[p] = __float_as_uint(yk.x);
+        q[p + 8] = __float_as_uint(yk.y);
+      }
+      exact = (all_neg >> 31) == 0;
+    }
+    if (exact) {
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        int r0 = __float2int_rn(__fdiv_rn(__fsub_rn(x[p].x, zf), sf));
+        int r1 = __float2int_rn(__fdiv_rn(__fsub_rn(x[p].y, zf), sf));
+        q[p] = static_cast<uint32_t>(min(max(r0, 0), L));
+        q[p + 8] = static_cast<uint32_t>(min(max(r1, 0), L));
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kEPL; ++e) q[e] = 0;
+  }
+  if (!valid) return;
+  if (BITS == 4) {
+    // byte b holds elements 2b (low nibble) and 2b+1 (high nibble)
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = (q[2 * i] & 15u) | ((q[2 * i + 1] & 15u) << 4);
+    const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+    *reinterpret_cast<uint2*>(code_dst + j * 8) = make_uint2(lo, hi);
+  } else {
+    uint4 w;
+    w.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+    w.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+    w.z = __byte_perm(__byte_perm(q[8], q[9], 0x0040), __byte_perm(q[10], q[11], 0x0040), 0x5410);
+    w.w = __byte_perm(__byte_perm(q[12], q[13], 0x0040), __byte_perm(q[14], q[15], 0x0040), 0x5410);
+    *reinterpret_cast<uint4*>(code_dst + j * 16) = w;
+  }
+  if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(sh, zh);
+}
+
+template <int D, typename InT>
+__global__ void __launch_bounds__(256, 3) quantize_kernel(PoolView pool, const InT* __restrict__ k,
+                                                       const InT* __restrict__ v,
+                                                       int64_t n_tokens, int64_t stride,
+                                                       const int32_t* __restrict__ block_ids,
+                                                       int64_t n_items) {
+  using S = Shape<D>;
+  const int lane = threadIdx.x & 31;
+  const int r = lane / S::LPV;
+  const int j = lane % S::LPV;
+  const int hkv = pool.n_kv_heads;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+
+  for (int64_t item = warp0; item < n_items; item += n_warps) {
+    const int64_t group_of_tokens = item / hkv;
+    const int h = static_cast<int>(item - group_of_tokens * hkv);
+    const int64_t t0 = group_of_tokens * S::VPW;
+    const int64_t t = t0 + r;
+    const bool valid = t < n_tokens;
+    const int32_t blk = __ldg(block_ids + t0 / kBlockTokens);
+    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+      if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const int slot = static_cast<int>(t % kBlockTokens);
+    const bool is8 = blk >= pool.n_q4;
+    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+    const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
+
+    // issue all four 16-byte loads (K and V) before any arithmetic
+    uint4 kw0 = make_uint4(0, 0, 0, 0), kw1 = kw0, vw0 = kw0, vw1 = kw0;
+    if (valid) {
+      const int64_t src = t * stride + static_cast<int64_t>(h) * D + j * kEPL;
+      kw0 = __ldg(reinterpret_cast<const uint4*>(k + src));
+      kw1 = __ldg(reinterpret_cast<const uint4*>(k + src) + 1);
+      vw0 = __ldg(reinterpret_cast<const uint4*>(v + src));
+      vw1 = __ldg(reinterpret_cast<const uint4*>(v + src) + 1);
+    }
+    float2 x[8];
+    // keys: rotate, then code
+    unpack16<InT>(kw0, kw1, x);
+    if (pool.k_rotated) rotate_pairs<D>(x, j);
+    if (is8)
+      encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
+    else
+      encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
+    // values: code unrotated
+    unpack16<InT>(vw0, vw1, x);
+    if (is8)
+      encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+    else
+      encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+    // a freshly written slot is live
+    if (valid && h == 0 && j == 0)
+      atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32,
+                ~(1u << (slot % 32)));
+  }
+}
+
+// Scalar butterflies for the decoder's optional un-rotation (channels 16j ..
+// 16j+15 of the lane in order); same stage order and operations as above.
 template <int D>
 __device__ __forceinline__ void fwht_vector(float (&x)[kEPL], int j) {
 #pragma unroll
@@ -69,131 +305,6 @@ __device__ __forceinline__ void rotate_vector(float (&x)[kEPL], int j) {
   const float c = rotation_constant(D);
 #pragma unroll
   for (int i = 0; i < kEPL; ++i) x[i] = __fmul_rn(x[i], c);
-}
-
-template <typename T>
-__device__ __forceinline__ void load16(const T* __restrict__ src, bool valid, float (&x)[kEPL]) {
-  static_assert(sizeof(T) == 2, "16-bit inputs");
-  uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
-  if (valid) {
-    w0 = __ldg(reinterpret_cast<const uint4*>(src));
-    w1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
-  }
-  const T* e0 = reinterpret_cast<const T*>(&w0);
-  const T* e1 = reinterpret_cast<const T*>(&w1);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    x[i] = to_float<T>(e0[i]);
-    x[8 + i] = to_float<T>(e1[i]);
-  }
-}
-
-// Encode the lane's 16 values (one quarter of a 64-value group) and store
-// codes and, from the group's first lane, its (scale, zero) pair.
-template <int BITS>
-__device__ __forceinline__ void encode_store(const float (&x)[kEPL], int j, bool valid,
-                                             uint8_t* __restrict__ code_dst,
-                                             __half2* __restrict__ param_dst) {
-  constexpr int L = (1 << BITS) - 1;
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < kEPL; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
-  // the 4 lanes of a group are j = 4k .. 4k+3
-  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
-  mx = __fadd_rn(mx, 0.0f);
-  const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(L));
-  const __half sh = __float2half_rn(s);
-  const __half zh = __float2half_rn(mn);
-  const float sf = __half2float(sh);
-  const float zf = __half2float(zh);
-
-  uint32_t q[kEPL];
-#pragma unroll
-  for (int i = 0; i < kEPL; ++i) {
-    int r = 0;
-    if (sf != 0.0f) {
-      r = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], zf), sf));
-      r = min(max(r, 0), L);
-    }
-    q[i] = static_cast<uint32_t>(r);
-  }
-  if (!valid) return;
-  if (BITS == 4) {
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      lo |= q[i] << (4 * i);
-      hi |= q[8 + i] << (4 * i);
-    }
-    *reinterpret_cast<uint2*>(code_dst + j * 8) = make_uint2(lo, hi);
-  } else {
-    uint4 w;
-    w.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
-    w.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
-    w.z = q[8] | (q[9] << 8) | (q[10] << 16) | (q[11] << 24);
-    w.w = q[12] | (q[13] << 8) | (q[14] << 16) | (q[15] << 24);
-    *reinterpret_cast<uint4*>(code_dst + j * 16) = w;
-  }
-  if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(sh, zh);
-}
-
-template <int D, typename InT>
-__global__ void __launch_bounds__(256) quantize_kernel(PoolView pool, const InT* __restrict__ k,
-                                                       const InT* __restrict__ v,
-                                                       int64_t n_tokens, int64_t stride,
-                                                       const int32_t* __restrict__ block_ids,
-                                                       int64_t n_items) {
-  using S = Shape<D>;
-  const int lane = threadIdx.x & 31;
-  const int r = lane / S::LPV;
-  const int j = lane % S::LPV;
-  const int hkv = pool.n_kv_heads;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-
-  for (int64_t item = warp0; item < n_items; item += n_warps) {
-    const int64_t group_of_tokens = item / hkv;
-    const int h = static_cast<int>(item - group_of_tokens * hkv);
-    const int64_t t0 = group_of_tokens * S::VPW;
-    const int64_t t = t0 + r;
-    const bool valid = t < n_tokens;
-    const int32_t blk = __ldg(block_ids + t0 / kBlockTokens);
-    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
-      if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
-      continue;
-    }
-    const int slot = static_cast<int>(t % kBlockTokens);
-    const bool is8 = blk >= pool.n_q4;
-    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
-    const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
-
-    float x[kEPL];
-    const int64_t src = t * stride + static_cast<int64_t>(h) * D + j * kEPL;
-    // keys: rotate, then code
-    load16<InT>(k + (valid ? src : 0), valid, x);
-    if (pool.k_rotated) rotate_vector<D>(x, j);
-    if (is8)
-      encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
-    else
-      encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
-    // values: code unrotated
-    load16<InT>(v + (valid ? src : 0), valid, x);
-    if (is8)
-      encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
-    else
-      encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
-    // a freshly written slot is live
-    if (valid && h == 0 && j == 0)
-      atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32,
-                ~(1u << (slot % 32)));
-  }
 }
 
 // ---------------------------------------------------------------------------

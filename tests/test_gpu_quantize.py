@@ -170,3 +170,41 @@ def test_large_block_ids_and_many_tokens():
     ids = list(range(63, -1, -1))
     pool, ref = _quantize_both(k, v, ids, 64)
     assert_pool_equal(pool, ref, blocks=[0, 1, 31, 62, 63])
+
+
+def test_near_tie_values_take_the_exact_path():
+    # V is stored unrotated, so its quotients can be placed on and next to
+    # half-integers exactly: z = -1, s = 1/16 (all fp16-exact), values
+    # z + (k + 1/2) s and their fp16 neighbours.
+    rng = np.random.default_rng(61)
+    n, hkv, d = 512, 2, 128
+    base = np.full((n, hkv, d), -1.0, np.float32)
+    k = rng.integers(0, 15, size=(n, hkv, d))
+    vals = (-1.0 + (k + 0.5) / 16.0).astype(np.float16)
+    nudge = rng.integers(-1, 2, size=vals.shape)
+    bits = vals.view(np.uint16).astype(np.int32) + nudge
+    vals = bits.astype(np.uint16).view(np.float16)
+    base[:] = vals.astype(np.float32)
+    base[:, :, 0::64] = -1.0                    # every group spans exactly [-1, -1 + 15/16]
+    base[:, :, 1::64] = -1.0 + 15 / 16
+    v = torch.from_numpy(base.astype(np.float16))
+    kk = torch.from_numpy(rng.standard_normal((n, hkv, d)).astype(np.float16))
+    for n_q8 in (0, 2):
+        pool, ref = _quantize_both(kk, v, [0, 1], 2 - n_q8, n_q8)
+        assert_pool_equal(pool, ref)
+
+
+@pytest.mark.parametrize("scale,offset", [(1e-3, 0.0), (1.0, 0.0), (300.0, 0.0), (1.0, 900.0),
+                                          (0.01, -40.0), (50.0, 3000.0)])
+def test_distribution_sweep(scale, offset):
+    # large offsets relative to the spread force the exact path (|z / s| > 2^10)
+    n, hkv, d = 2048, 4, 128
+    rng = np.random.default_rng(int(scale * 1000 + offset) % 2**31)
+    x = rng.standard_normal((n, hkv, d)) * scale + offset
+    k = torch.from_numpy(x.astype(np.float16))
+    v = torch.from_numpy((x[::-1] * 0.5).copy().astype(np.float16))
+    ids = list(range(8))
+    pool, ref = _quantize_both(k, v, ids, 6, 2)
+    assert_pool_equal(pool, ref)
+    pool, ref = _quantize_both(k.to(torch.bfloat16), v.to(torch.bfloat16), ids, 8, 0)
+    assert_pool_equal(pool, ref)
