@@ -168,22 +168,36 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return Q4KV_ERR_CUDA;
   }
-  const int64_t ctx = static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens;
-  const int64_t max_splits = (ctx + 63) / 64;
+  // kernel 1 (tensor-core pipeline) handles every shape accepted above; its
+  // splits are whole 256-token blocks
+  const int kernel = 1;
+  const int64_t unit = kBlockTokens;
+  const int64_t nb = max_blocks_per_seq;
+  const int64_t ctx = nb * kBlockTokens;
   int64_t s = n_splits;
   if (s == 0) {
+    // persistent CTAs (one per SM) take items (sequence, KV head, split) in
+    // waves; cost = waves * (blocks per item + per-item overhead)
     const int64_t pairs = static_cast<int64_t>(batch > 0 ? batch : 1) * n_kv_heads;
-    const int64_t target = static_cast<int64_t>(num_sms) * 16;   // CTAs worth launching
-    s = (target + pairs - 1) / pairs;
-    const int64_t min_tokens = 256;                             // keep partials a small share
-    const int64_t cap = (ctx + min_tokens - 1) / min_tokens;
-    if (s > cap) s = cap;
+    double best = 1e300;
+    s = 1;
+    for (int64_t cand = 1; cand <= nb; ++cand) {
+      const int64_t bps = (nb + cand - 1) / cand;
+      if ((nb + bps - 1) / bps != cand) continue;         // each distinct split only once
+      const int64_t items = pairs * cand;
+      const int64_t waves = (items + num_sms - 1) / num_sms;
+      const double cost = static_cast<double>(waves) * (static_cast<double>(bps) + 0.75);
+      if (cost < best - 1e-9) {
+        best = cost;
+        s = cand;
+      }
+    }
   }
   if (s < 1) s = 1;
-  if (s > max_splits) s = max_splits;
+  if (s > nb) s = nb;
   if (s > 65535) s = 65535;
   int64_t tps = (ctx + s - 1) / s;
-  tps = (tps + 63) / 64 * 64;
+  tps = (tps + unit - 1) / unit * unit;
   s = (ctx + tps - 1) / tps;
   memset(plan, 0, sizeof(*plan));
   plan->batch = batch;
@@ -193,7 +207,7 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
   plan->max_blocks_per_seq = max_blocks_per_seq;
   plan->n_splits = static_cast<int32_t>(s);
   plan->tokens_per_split = static_cast<int32_t>(tps);
-  plan->kernel = 0;
+  plan->kernel = kernel;
   if (s > 1) {
     const size_t rows = static_cast<size_t>(batch) * n_q_heads * s;
     plan->workspace_bytes = round_up(rows * head_dim * sizeof(float), 256) + round_up(rows * 2 * sizeof(float), 256);

@@ -305,21 +305,45 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+int device_sm_count() {
+  static int cached[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream) {
   const q4kv_decode_plan& p = a.plan;
-  const dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
-  if (p.head_dim == 128)
-    decode_simple_kernel<128><<<grid, kThreads, 0, stream>>>(a);
-  else
-    decode_simple_kernel<256><<<grid, kThreads, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || p.n_splits == 1) return e;
   const unsigned rows = static_cast<unsigned>(p.batch) * p.n_q_heads;
   if (p.head_dim == 128)
     merge_kernel<128><<<rows, 128, 0, stream>>>(a);
   else
     merge_kernel<256><<<rows, 128, 0, stream>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  const q4kv_decode_plan& p = a.plan;
+  cudaError_t e;
+  if (p.kernel == 1) {
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    e = launch_decode_tc(a, sms, stream);
+  } else {
+    const dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
+    if (p.head_dim == 128)
+      decode_simple_kernel<128><<<grid, kThreads, 0, stream>>>(a);
+    else
+      decode_simple_kernel<256><<<grid, kThreads, 0, stream>>>(a);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess || p.n_splits == 1) return e;
+  return launch_merge(a, stream);
 }
 
 }  // namespace q4kv

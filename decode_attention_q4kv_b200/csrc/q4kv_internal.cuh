@@ -102,6 +102,11 @@ struct DecodeArgs {
   float* ws_o;   // [B][Hq][S][D]
   float* ws_ml;  // [B][Hq][S][2] (running max, running sum)
 };
+// plan.kernel selects the decode kernel: 1 = tensor-core pipeline
+// (decode_tc.cu), 0 = CUDA-core kernel (decode.cu); both share the merge.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
+int device_sm_count();
 
 }  // namespace q4kv

@@ -71,7 +71,7 @@ def test_plan_covers_context(B, hq, hkv, d, mb):
     st, p = _plan(B, hq, hkv, d, mb, 0, 148)
     assert st == 0
     ctx = mb * 256
-    assert p.tokens_per_split % 64 == 0 and p.tokens_per_split >= 64
+    assert p.tokens_per_split % 256 == 0 and p.kernel == 1
     assert p.n_splits * p.tokens_per_split >= ctx > (p.n_splits - 1) * p.tokens_per_split
     if p.n_splits > 1:
         assert p.workspace_bytes >= B * hq * p.n_splits * (d + 2) * 4
@@ -91,7 +91,7 @@ def test_plan_rejects_bad_shapes():
     assert _plan(1, 32, 8, 128, 0, 0, 148)[0] == _lib.ERR_INVALID_ARG      # empty table
     assert _plan(-1, 32, 8, 128, 4, 0, 148)[0] == _lib.ERR_INVALID_ARG
     st, p = _plan(1, 32, 8, 128, 4, 100000, 148)                            # clamped to the context
-    assert st == 0 and p.n_splits == 16 and p.tokens_per_split == 64
+    assert st == 0 and p.n_splits == 4 and p.tokens_per_split == 256 and p.kernel == 1
 
 
 def test_quantize_rejects_bad_arguments_without_launching():

@@ -54,10 +54,11 @@ class Case:
         self.pool.invalidate(slots.to(cuda()))
         self.ref.invalidate_slots(slots.tolist())
 
-    def run(self, n_splits=0, out_dtype=torch.float32, scale=0.0):
+    def run(self, n_splits=0, out_dtype=torch.float32, scale=0.0, kernel=1):
         dev = cuda()
         plan = q4.DecodePlan(len(self.lens), self.q.shape[1], self.pool.n_kv_heads, self.q.shape[2],
                              self.mb, n_splits=n_splits)
+        plan.c.kernel = kernel      # 1: tensor-core pipeline (default), 0: CUDA-core kernel
         out = q4.decode_attention(self.pool, self.q.to(dev), self.tables.to(dev), self.lens_t.to(dev),
                                   softmax_scale=scale, out_dtype=out_dtype, plan=plan)
         torch.cuda.synchronize()
@@ -84,10 +85,11 @@ def test_tiny_workload():
     assert pool.read_device_error() == 0
 
 
+@pytest.mark.parametrize("kernel", [1, 0])
 @pytest.mark.parametrize("n_splits", [0, 1, 2, 7, 64])
-def test_ragged_lengths_and_splits(n_splits):
+def test_ragged_lengths_and_splits(n_splits, kernel):
     c = Case([1000, 1, 257, 0, 513, 256], hq=32, hkv=8, d=128, seed=1)
-    out, plan = c.run(n_splits)
+    out, plan = c.run(n_splits, kernel=kernel)
     assert_close(out, c.oracle(), what=f"splits={plan.n_splits}")
     assert torch.all(out[3] == 0)
 
@@ -95,18 +97,21 @@ def test_ragged_lengths_and_splits(n_splits):
 @pytest.mark.parametrize("hq,hkv,d,dtype", [(16, 8, 256, "bf16"), (40, 8, 128, "fp16"),
                                             (8, 8, 128, "fp16"), (8, 1, 128, "bf16"),
                                             (4, 1, 256, "fp16"), (12, 4, 128, "bf16")])
-def test_gqa_shapes(hq, hkv, d, dtype):
+@pytest.mark.parametrize("kernel", [1, 0])
+def test_gqa_shapes(hq, hkv, d, dtype, kernel):
     c = Case([700, 300], hq=hq, hkv=hkv, d=d, dtype=dtype, seed=2)
-    out, _ = c.run()
+    out, _ = c.run(kernel=kernel)
     assert_close(out, c.oracle(), what=f"{hq}/{hkv}/{d}")
 
 
-def test_mixed_q8_blocks():
-    c = Case([900, 600], hq=32, hkv=8, d=128, seed=3, n_pool=8, q8_blocks=(4, 5, 6))
+@pytest.mark.parametrize("d,hq", [(128, 32), (256, 16)])
+def test_mixed_q8_blocks(d, hq):
+    c = Case([900, 600], hq=hq, hkv=8, d=d, seed=3, n_pool=8, q8_blocks=(4, 5, 6))
     # make sure some sequence blocks are 8-bit: the table uses ids drawn from the whole pool
     assert any(int(x) >= c.n_q4 for x in c.tables.view(-1))
-    out, _ = c.run()
-    assert_close(out, c.oracle(), what="mixed")
+    for s in (0, 3):
+        out, _ = c.run(s)
+        assert_close(out, c.oracle(), what="mixed")
 
 
 def test_eviction_mask_and_scribble_invariance():
