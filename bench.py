@@ -143,13 +143,18 @@ class Job:
         from decode_attention_q4kv_b200 import workloads as W
 
         self.w, self.dev, self.torch, self.q4 = w, device, torch, q4
-        self.n_layers = layers or w.layers
+        if isinstance(layers, (list, tuple)):
+            layer_ids = list(layers)
+        else:
+            layer_ids = list(range(layers or w.layers))
+        self.layer_ids = layer_ids
+        self.n_layers = len(layer_ids)
         n_tok = w.prefill_tokens or w.n_tokens
         n_pool = max(w.n_blocks, n_tok // 256) if w.permuted_pool else w.n_blocks
         self.n_q8 = w.n_q8_blocks
         self.n_q4 = n_pool - self.n_q8
         self.layers = []
-        for l in range(self.n_layers):
+        for l in layer_ids:
             lid = l + 1000 * rank
             k, v = W.kv_tokens(w, lid, n_tok, device)
             q = W.query(w, lid, device)
@@ -192,6 +197,9 @@ class Job:
         if w.q8_fraction:
             am = q4.block_absmean(L["k"])
             ids = q4.mixed_block_ids(am, self.n_q8, 0, self.n_q4)
+            L["ids"] = ids
+            # sequence b's i-th chunk lives in block ids[b * nb + i]
+            L["tables"] = ids.view(w.batch, w.blocks_per_seq)
         elif self.prefill_ids is not None:
             ids = self.prefill_ids
         else:
@@ -200,9 +208,21 @@ class Job:
         if self.evict is not None:
             L["pool"].invalidate(self.evict)
 
+    @property
+    def ids_per_layer(self):
+        return [L.get("ids") for L in self.layers]
+
+    @property
+    def last_ids(self):
+        return getattr(self, "_last_ids", None if not self.w.q8_fraction else self.layers[0].get("ids"))
+
+    @last_ids.setter
+    def last_ids(self, v):
+        self._last_ids = v
+
     def decode_layer(self, L):
-        self.q4.decode_attention(L["pool"], L["q"], self.tables, self.lens, plan=self.plan,
-                                 workspace=self.ws, out=L["out"])
+        self.q4.decode_attention(L["pool"], L["q"], L.get("tables", self.tables), self.lens,
+                                 plan=self.plan, workspace=self.ws, out=L["out"])
 
     def step(self, events=None):
         for L in self.layers:

@@ -126,6 +126,14 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// keys: u8 codes x s8 query digits, exact int32 accumulation
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ uint32_t movtrans(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -172,37 +180,41 @@ struct Geo {
   static_assert(TS * PB <= kParamBytes, "stage params");
 };
 
-// Key A operand of k-step s for the thread's two rows (from their key bytes).
-// Thread t owns channels 128c + 32t + [0, 32) of each row (c < D/128); k-step
-// s uses chunk c = s/8, 8-channel word w = (s%8)/2, pairs p0 = 2 (s%2) and
-// p0 + 1, where pair p of a word = channels (p, p + 4) of it.
-template <int D, bool Q8>
-__device__ __forceinline__ void key_a(const uint32_t* rg, const uint32_t* rg8, int s, uint32_t (&a)[4]) {
-  const int c = s / 8, w = (s % 8) / 2, p0 = 2 * (s % 2);
+// Key A operand (u8) of 32-channel step kk for the thread's two rows.  Thread
+// t owns channels 128c + 32t + [0, 32) of each row (c < D/128); step kk uses
+// chunk c = kk/4 and its 8-channel word w = kk%4: register 0 (k = 4t .. 4t+3)
+// holds channels 8w + {0, 2, 4, 6}, register 2 (k = 16 + 4t ..) 8w + {1, 3, 5, 7}.
+template <bool Q8>
+__device__ __forceinline__ void key_a8(const uint32_t* rg, const uint32_t* rg8, int kk, uint32_t (&a)[4]) {
   if (!Q8) {
-    // 16 bytes per chunk = 4 words of 8 nibbles; word index c*4 + w
-    const uint32_t x0 = rg[c * 4 + w], x1 = rg8[c * 4 + w];
-    if (p0 == 0) {   // pairs 0 (lo nibbles of bytes 0, 2) and 1 (hi nibbles of bytes 0, 2)
-      a[0] = lo_nib(x0); a[1] = lo_nib(x1); a[2] = hi_nib(x0); a[3] = hi_nib(x1);
-    } else {         // pairs 2, 3: the same for bytes 1, 3
-      a[0] = lo_nib(x0 >> 8); a[1] = lo_nib(x1 >> 8); a[2] = hi_nib(x0 >> 8); a[3] = hi_nib(x1 >> 8);
-    }
+    // a 4-bit word holds elements 0..7 at nibbles 0..7: the low nibbles are 0, 2, 4, 6
+    const uint32_t x0 = rg[kk], x1 = rg8[kk];
+    a[0] = x0 & 0x0F0F0F0Fu;
+    a[1] = x1 & 0x0F0F0F0Fu;
+    a[2] = (x0 >> 4) & 0x0F0F0F0Fu;
+    a[3] = (x1 >> 4) & 0x0F0F0F0Fu;
   } else {
-    // 32 bytes per chunk = 8 words of 4 codes; channels 8w + e are in words 2w (e < 4), 2w+1
-    const uint32_t l0 = rg[c * 8 + 2 * w], h0 = rg[c * 8 + 2 * w + 1];
-    const uint32_t l1 = rg8[c * 8 + 2 * w], h1 = rg8[c * 8 + 2 * w + 1];
-    const uint32_t s0 = p0 | (p0 << 8) + 0x400u;          // [lo.p0, -, hi.p0, -]
-    const uint32_t s1 = (p0 + 1) | ((p0 + 1) << 8) + 0x400u;
-    a[0] = byte_pair(__byte_perm(l0, h0, s0));
-    a[1] = byte_pair(__byte_perm(l1, h1, s0));
-    a[2] = byte_pair(__byte_perm(l0, h0, s1));
-    a[3] = byte_pair(__byte_perm(l1, h1, s1));
+    // 8-bit: channels 8w .. 8w+3 in word 2w, 8w+4 .. 8w+7 in word 2w+1
+    a[0] = __byte_perm(rg[2 * kk], rg[2 * kk + 1], 0x6420);
+    a[1] = __byte_perm(rg8[2 * kk], rg8[2 * kk + 1], 0x6420);
+    a[2] = __byte_perm(rg[2 * kk], rg[2 * kk + 1], 0x7531);
+    a[3] = __byte_perm(rg8[2 * kk], rg8[2 * kk + 1], 0x7531);
   }
 }
 
-// Value A operands for one 16-token tile: tokens T = 2t, 2t+1, 2t+8, 2t+9 of
-// the tile, thread g's channels cb + [0, D/8).  Tile mv (channels) uses rows
-// g -> cb + 2 mv and g + 8 -> cb + 2 mv + 1.
+// Token order inside a 16-token tile: accumulator row r holds token pi(r),
+// pi swapping 2 <-> 3 and 6 <-> 7 in each half.  With it the four value rows a
+// thread reads at one time fall on both 64-byte halves of the 128-byte bank
+// window, halving shared-memory bank conflicts; any permutation is correct
+// because both contractions sum over tokens.
+__device__ __forceinline__ int tok_perm(int r) { return r ^ ((r >> 1) & 1); }
+
+// Value A operands for one 16-token tile: tokens T = pi(2t), pi(2t+1),
+// pi(2t+8), pi(2t+9) of the tile, thread g's channels cb + [0, D/8).  Tile mv
+// (channels) uses rows g -> cb + 2 mv and g + 8 -> cb + 2 mv + 1.  The codes
+// enter the MMA as exact small integers: an offset form (1024 + code) would
+// save one instruction per register, but the accumulator would then carry
+// ~1024 x the weight sum and lose accuracy over long contexts.
 template <int D, bool Q8>
 __device__ __forceinline__ void value_a(const uint32_t* v0, const uint32_t* v1, const uint32_t* v8,
                                         const uint32_t* v9, int mv, uint32_t (&a)[4]) {
@@ -256,18 +268,26 @@ __device__ __forceinline__ void reset(WarpState<D, NT>& st) {
   }
 }
 
-// One 16-token tile of a stage: keys, softmax update, values.
-template <int D, int NT, bool Q8>
-__device__ __forceinline__ void tile(WarpState<D, NT>& st, const uint8_t* stage, int row0, int nvalid,
-                                     const uint32_t (&bq)[D / 16][NT][4], const float (&qs)[NT][2],
-                                     float sc2, int lane) {
+// NTILE 16-token tiles of one stage: keys for every tile, one online-softmax
+// update over all of them, then values.  The running max moves only when the
+// tile max exceeds it by more than kLazy (log2 units), so the accumulators are
+// rescaled rarely; weights stay <= 2^kLazy.
+constexpr float kLazy = 2.0f;
+
+template <int D, int NT, bool Q8, int NTILE>
+__device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage, const int (&row0)[NTILE],
+                                      int nvalid, const uint32_t (&bq)[D / 32][NT][2][2],
+                                      const float (&qs)[NT][2], const float (&ks)[NT], int lane) {
   using G = Geo<D, Q8>;
   const int g = lane >> 2, t = lane & 3;
-  // ---- keys: two rows per thread (tile rows g and g + 8) ----
-  uint32_t rg[G::KB / 4], rg8[G::KB / 4];
-  {
-    const uint8_t* kc = stage + (row0 + g) * G::RB;
-    const uint8_t* kc8 = stage + (row0 + g + 8) * G::RB;
+  const int pg = tok_perm(g), pg8 = tok_perm(g + 8);
+  // ---- keys ----
+  float sk[NTILE][NT][4];
+#pragma unroll
+  for (int i = 0; i < NTILE; ++i) {
+    uint32_t rg[G::KB / 4], rg8[G::KB / 4];
+    const uint8_t* kc = stage + (row0[i] + pg) * G::RB;
+    const uint8_t* kc8 = stage + (row0[i] + pg8) * G::RB;
 #pragma unroll
     for (int c = 0; c < D / 128; ++c) {
 #pragma unroll
@@ -279,109 +299,135 @@ __device__ __forceinline__ void tile(WarpState<D, NT>& st, const uint8_t* stage,
         rg8[wi] = u8.x; rg8[wi + 1] = u8.y; rg8[wi + 2] = u8.z; rg8[wi + 3] = u8.w;
       }
     }
-  }
-  float sacc[NT][4];
+    int hi[NT][4], lo[NT][4];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.0f;
+    for (int j = 0; j < NT; ++j)
 #pragma unroll
-  for (int s = 0; s < D / 16; ++s) {
-    uint32_t a[4];
-    key_a<D, Q8>(rg, rg8, s, a);
+      for (int e = 0; e < 4; ++e) hi[j][e] = lo[j][e] = 0;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      mma16816(sacc[j], a, bq[s][j][0], bq[s][j][1]);   // q hi
-      mma16816(sacc[j], a, bq[s][j][2], bq[s][j][3]);   // q lo
+    for (int kk = 0; kk < D / 32; ++kk) {
+      uint32_t a[4];
+      key_a8<Q8>(rg, rg8, kk, a);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        mma_u8s8(hi[j], a, bq[kk][j][1][0], bq[kk][j][1][1]);
+        mma_u8s8(lo[j], a, bq[kk][j][0][0], bq[kk][j][0][1]);
+      }
     }
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sk[i][j][e] = static_cast<float>(hi[j][e] * 256 + lo[j][e]);
   }
-  // ---- per-token parameters for the thread's two columns' groups ----
-  // D = 128: columns (h, 0), (h, 1); D = 256: (h, 2 (t%2)), (h, 2 (t%2) + 1).
+  // ---- per-token parameters and logits (log2 units) ----
+  // D = 128: the thread's columns are (h, 0), (h, 1); D = 256: (h, 2 (t%2)), (h, 2 (t%2) + 1).
   const int gbase = (G::NG == 2) ? 0 : 2 * (t & 1);
   const uint8_t* kp = stage + kOffKP;
   const uint8_t* vp = stage + kOffVP;
   const uint32_t* mask = reinterpret_cast<const uint32_t*>(stage + kOffMask);
-  const StageMeta& meta = *reinterpret_cast<const StageMeta*>(stage + kOffMeta);
-  float logit[NT][2];
-  float ws[2][2], wz[2][2];   // [row][e]: value scale, zero
-  bool live[2];
+  const int slot0 = reinterpret_cast<const StageMeta*>(stage + kOffMeta)->slot0;
+  float logit[NTILE][NT][2];
+  float ws[NTILE][2][2], wz[NTILE][2][2];   // [tile][row][e]: value scale, zero (0 unless live)
+  bool live[NTILE][2];
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = row0 + g + 8 * r;
-    const bool valid = row < nvalid;
-    const int slot = meta.slot0 + row;
-    const bool masked = valid && ((mask[slot >> 5] >> (slot & 31)) & 1u);
-    live[r] = valid && !masked;
-    const uint2 kpw = lds<uint2>(kp + row * G::PB + gbase * 4);
-    const uint2 vpw = lds<uint2>(vp + row * G::PB + gbase * 4);
-    const float2 k0 = __half22float2(u2h(kpw.x)), k1 = __half22float2(u2h(kpw.y));
-    const float2 v0 = __half22float2(u2h(vpw.x)), v1 = __half22float2(u2h(vpw.y));
-    // rows outside the range or remapped may hold any bytes (even NaN
-    // parameters): select, never multiply, them away
-    ws[r][0] = live[r] ? v0.x : 0.0f;
-    wz[r][0] = live[r] ? v0.y : 0.0f;
-    ws[r][1] = live[r] ? v1.x : 0.0f;
-    wz[r][1] = live[r] ? v1.y : 0.0f;
+  for (int i = 0; i < NTILE; ++i) {
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      float part = __fmaf_rn(k0.x, sacc[j][2 * r], k1.x * sacc[j][2 * r + 1]) * sc2 +
-                   (k0.y * qs[j][0] + k1.y * qs[j][1]);
-      if (G::NG == 4) part += __shfl_xor_sync(0xffffffffu, part, 1);
-      logit[j][r] = !valid ? -INFINITY : (masked ? Q4KV_SENTINEL_LOGIT * kLog2e : part);
+    for (int r = 0; r < 2; ++r) {
+      const int row = row0[i] + (r ? pg8 : pg);
+      const bool valid = row < nvalid;
+      const int slot = slot0 + row;
+      const bool masked = valid && ((mask[slot >> 5] >> (slot & 31)) & 1u);
+      const bool lv = valid && !masked;
+      live[i][r] = lv;
+      const uint2 kpw = lds<uint2>(kp + row * G::PB + gbase * 4);
+      const uint2 vpw = lds<uint2>(vp + row * G::PB + gbase * 4);
+      const float2 k0 = __half22float2(u2h(kpw.x)), k1 = __half22float2(u2h(kpw.y));
+      const float2 v0 = __half22float2(u2h(vpw.x)), v1 = __half22float2(u2h(vpw.y));
+      // rows outside the range or remapped may hold any bytes (even NaN
+      // parameters): select, never multiply, them away
+      ws[i][r][0] = lv ? v0.x : 0.0f;
+      wz[i][r][0] = lv ? v0.y : 0.0f;
+      ws[i][r][1] = lv ? v1.x : 0.0f;
+      wz[i][r][1] = lv ? v1.y : 0.0f;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        float part = __fmaf_rn(k0.x, sk[i][j][2 * r], k1.x * sk[i][j][2 * r + 1]) * ks[j] +
+                     __fmaf_rn(k0.y, qs[j][0], k1.y * qs[j][1]);
+        if (G::NG == 4) part += __shfl_xor_sync(0xffffffffu, part, 1);
+        logit[i][j][r] = !valid ? -INFINITY : (masked ? Q4KV_SENTINEL_LOGIT * kLog2e : part);
+      }
     }
   }
-  // ---- online softmax over the tile (16 tokens), per column head ----
-  uint32_t wb[NT][2];   // W pairs for rows g, g + 8 (accumulator layout)
+  // ---- online softmax over the NTILE tiles ----
+  uint32_t wb[NTILE][NT][2];
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
-    float mx = fmaxf(logit[j][0], logit[j][1]);
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NTILE; ++i) mx = fmaxf(mx, fmaxf(logit[i][j][0], logit[i][j][1]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    const float m_new = fmaxf(st.m[j], mx);
-    float alpha = 1.0f, p0 = 0.0f, p1 = 0.0f;
-    if (m_new != -INFINITY) {
-      alpha = ex2(st.m[j] - m_new);   // 0 when the old max is -inf
-      p0 = ex2(logit[j][0] - m_new);
-      p1 = ex2(logit[j][1] - m_new);
+    if (mx > st.m[j] + kLazy) {          // also taken on the first live tile (m = -inf)
+      const float alpha = ex2(st.m[j] - mx);
+      st.m[j] = mx;
+      st.l[j] *= alpha;
+      st.z[j][0] *= alpha;
+      st.z[j][1] *= alpha;
+#pragma unroll
+      for (int mv = 0; mv < D / 16; ++mv)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.o[mv][j][e] *= alpha;
     }
-    st.m[j] = m_new;
-    st.l[j] = __fmaf_rn(st.l[j], alpha, p0 + p1);
-    const float q0 = live[0] ? p0 : 0.0f, q1 = live[1] ? p1 : 0.0f;
-    st.z[j][0] = __fmaf_rn(st.z[j][0], alpha, __fmaf_rn(q0, wz[0][0], q1 * wz[1][0]));
-    st.z[j][1] = __fmaf_rn(st.z[j][1], alpha, __fmaf_rn(q0, wz[0][1], q1 * wz[1][1]));
+    const float m = st.m[j];
+    float lsum = 0.0f, z0 = 0.0f, z1 = 0.0f;
 #pragma unroll
-    for (int mv = 0; mv < D / 16; ++mv)
+    for (int i = 0; i < NTILE; ++i) {
+      float p[2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st.o[mv][j][e] *= alpha;
-    wb[j][0] = h2u(__floats2half2_rn(q0 * ws[0][0], q0 * ws[0][1]));
-    wb[j][1] = h2u(__floats2half2_rn(q1 * ws[1][0], q1 * ws[1][1]));
+      for (int r = 0; r < 2; ++r) {
+        p[r] = logit[i][j][r] == -INFINITY ? 0.0f : ex2(logit[i][j][r] - m);
+        lsum += p[r];
+        const float q = live[i][r] ? p[r] : 0.0f;
+        z0 = __fmaf_rn(q, wz[i][r][0], z0);
+        z1 = __fmaf_rn(q, wz[i][r][1], z1);
+        wb[i][j][r] = h2u(__floats2half2_rn(q * ws[i][r][0], q * ws[i][r][1]));
+      }
+    }
+    st.l[j] += lsum;
+    st.z[j][0] += z0;
+    st.z[j][1] += z1;
   }
   // ---- values ----
-  uint32_t bw[NT][2];
-#pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    bw[j][0] = movtrans(wb[j][0]);   // tokens 2t, 2t+1 of rows 0-7
-    bw[j][1] = movtrans(wb[j][1]);   // tokens 8 + 2t, 9 + 2t
-  }
   constexpr int VW = G::VB / 4;   // words of value codes per token row
-  uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
-  {
+#pragma unroll
+  for (int i = 0; i < NTILE; ++i) {
+    uint32_t bw[NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      bw[j][0] = movtrans(wb[i][j][0]);   // tokens pi(2t), pi(2t+1)
+      bw[j][1] = movtrans(wb[i][j][1]);   // tokens pi(8+2t), pi(9+2t)
+    }
+    uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
     const uint8_t* vc = stage + kOffV + g * G::VB;
+    const int r0 = row0[i] + tok_perm(2 * t), r1 = row0[i] + tok_perm(2 * t + 1);
+    const int r8 = row0[i] + tok_perm(2 * t + 8), r9 = row0[i] + tok_perm(2 * t + 9);
 #pragma unroll
     for (int q = 0; q < VW; q += 2) {
-      const uint2 a0 = lds<uint2>(vc + (row0 + 2 * t) * G::RB + 4 * q);
-      const uint2 a1 = lds<uint2>(vc + (row0 + 2 * t + 1) * G::RB + 4 * q);
-      const uint2 a8 = lds<uint2>(vc + (row0 + 2 * t + 8) * G::RB + 4 * q);
-      const uint2 a9 = lds<uint2>(vc + (row0 + 2 * t + 9) * G::RB + 4 * q);
+      const uint2 a0 = lds<uint2>(vc + r0 * G::RB + 4 * q);
+      const uint2 a1 = lds<uint2>(vc + r1 * G::RB + 4 * q);
+      const uint2 a8 = lds<uint2>(vc + r8 * G::RB + 4 * q);
+      const uint2 a9 = lds<uint2>(vc + r9 * G::RB + 4 * q);
       v0[q] = a0.x; v0[q + 1] = a0.y; v1[q] = a1.x; v1[q + 1] = a1.y;
       v8[q] = a8.x; v8[q + 1] = a8.y; v9[q] = a9.x; v9[q + 1] = a9.y;
     }
-  }
 #pragma unroll
-  for (int mv = 0; mv < D / 16; ++mv) {
-    uint32_t a[4];
-    value_a<D, Q8>(v0, v1, v8, v9, mv, a);
+    for (int mv = 0; mv < D / 16; ++mv) {
+      uint32_t a[4];
+      value_a<D, Q8>(v0, v1, v8, v9, mv, a);
 #pragma unroll
-    for (int j = 0; j < NT; ++j) mma16816(st.o[mv][j], a, bw[j][0], bw[j][1]);
+      for (int j = 0; j < NT; ++j) mma16816(st.o[mv][j], a, bw[j][0], bw[j][1]);
+    }
   }
 }
 
@@ -392,8 +438,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kNS * kStageBytes);
   uint64_t* empty = full + kNS;
   float* qrot = reinterpret_cast<float*>(empty + kNS);                 // [G][D]
-  float* qsum = qrot + 8 * D;                                          // [8][4]
-  float* mrg_ml = qsum + 32;                                           // [kCW][8][2]
+  float* qsum = qrot + 8 * D;                                          // [8][4] sums, [32 + h] scales
+  float* mrg_ml = qsum + 64;                                           // [kCW][8][2]
   float* mrg_o = mrg_ml + kCW * 16;                                    // [kCW][G][D]
   __shared__ int s_flags[2];                                            // poison, timeout
 
@@ -494,8 +540,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
   constexpr int NG = D / kGroup;
   const float sc2 = a.scale * kLog2e;
   WarpState<D, NT> st;
-  uint32_t bq[D / 16][NT][4];
-  float qs[NT][2];
+  uint32_t bq[D / 32][NT][2][2];   // [step][n-tile][digit][register]
+  float qs[NT][2], ks[NT];
   uint32_t it = 0;
   bool dead = false;
 
@@ -503,7 +549,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
     const int split = item % S;
     const int kvh = (item / S) % hkv;
     const int b = item / (S * hkv);
-    // ---- rotated query of the item's G heads -> B fragments ----
+    // ---- rotated query of the item's G heads -> 16-bit fixed point -> B fragments ----
     for (int i = threadIdx.x; i < G * D; i += kCW * 32) {
       const int64_t qi = (static_cast<int64_t>(b) * hq + kvh * G) * D + i;
       qrot[i] = a.q_dtype == Q4KV_F16 ? __half2float(static_cast<const __half*>(a.q)[qi])
@@ -525,7 +571,20 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
       for (int i = threadIdx.x; i < G * D; i += kCW * 32) qrot[i] *= c;
       consumer_sync();
     }
-    if (threadIdx.x < G * NG) {   // group sums of the rotated query
+    // warp h < G: scale 2^E with max |q_rot[h]| * 2^E <= 32000, then q_int = rne(q_rot * 2^E)
+    if (warp < G) {
+      float mx = 0.0f;
+      for (int c = lane; c < D; c += 32) mx = fmaxf(mx, fabsf(qrot[warp * D + c]));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      int e = 0;
+      if (mx > 0.0f) e = static_cast<int>(floorf(log2f(32000.0f / mx)));
+      e = max(-100, min(100, e));
+      for (int c = lane; c < D; c += 32) qrot[warp * D + c] = rintf(ldexpf(qrot[warp * D + c], e));
+      if (lane == 0) qsum[32 + warp] = ldexpf(1.0f, -e);       // 2^-E of head `warp`
+    }
+    consumer_sync();
+    if (threadIdx.x < G * NG) {   // exact group sums of the integer query
       const int h = threadIdx.x / NG, gr = threadIdx.x % NG;
       float acc = 0.0f;
       for (int c = 0; c < kGroup; ++c) acc += qrot[h * D + gr * kGroup + c];
@@ -537,26 +596,34 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
       const int col = 8 * j + g;                // this thread's B column
       const int h = col / NG, gr = col % NG;
 #pragma unroll
-      for (int s = 0; s < D / 16; ++s) {
-        const int c = s / 8, w = (s % 8) / 2, p0 = 2 * (s % 2);
-        const int base = 128 * c + 32 * t + 8 * w;
-        float v[4];
-        const int chs[4] = {base + p0, base + p0 + 4, base + p0 + 1, base + p0 + 5};
+      for (int kk = 0; kk < D / 32; ++kk) {
+        const int base = 128 * (kk / 4) + 32 * t + 8 * (kk % 4);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          v[e] = (h < G && chs[e] / kGroup == gr) ? qrot[h * D + chs[e]] : 0.0f;
-        const __half2 h01 = __floats2half2_rn(v[0], v[1]), h23 = __floats2half2_rn(v[2], v[3]);
-        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-        bq[s][j][0] = h2u(h01);
-        bq[s][j][1] = h2u(h23);
-        bq[s][j][2] = h2u(__floats2half2_rn(v[0] - f01.x, v[1] - f01.y));
-        bq[s][j][3] = h2u(__floats2half2_rn(v[2] - f23.x, v[3] - f23.y));
+        for (int r = 0; r < 2; ++r) {           // register r: channels base + r + {0, 2, 4, 6}
+          uint32_t d0 = 0, d1 = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int ch = base + r + 2 * e;
+            const int qv = (h < G && ch / kGroup == gr) ? static_cast<int>(qrot[h * D + ch]) : 0;
+            const int q0 = ((qv + 128) & 255) - 128;     // balanced low digit
+            const int q1 = (qv - q0) >> 8;               // high digit, |q1| <= 125
+            d0 |= static_cast<uint32_t>(q0 & 255) << (8 * e);
+            d1 |= static_cast<uint32_t>(q1 & 255) << (8 * e);
+          }
+          bq[kk][j][0][r] = d0;
+          bq[kk][j][1][r] = d1;
+        }
       }
+      {
+        const int c2 = 8 * j + 2 * t;             // the thread's accumulator columns c2, c2 + 1
+        const int h2 = c2 / NG;
+        const float sc = h2 < G ? sc2 * qsum[32 + h2] : 0.0f;
+        ks[j] = sc;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {   // the thread's accumulator columns 8j + 2t + e
-        const int c2 = 8 * j + 2 * t + e;
-        const int h2 = c2 / NG, g2 = c2 % NG;
-        qs[j][e] = h2 < G ? qsum[h2 * 4 + g2] * sc2 : 0.0f;
+        for (int e = 0; e < 2; ++e) {
+          const int g2 = (c2 + e) % NG;
+          qs[j][e] = h2 < G ? qsum[h2 * 4 + g2] * sc : 0.0f;
+        }
       }
     }
     reset(st);
@@ -571,13 +638,20 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
       const bool last = dead ? true : meta.last;
       timeout |= dead || meta.timeout;
       poison |= meta.poison;
-      if (!dead && !meta.timeout && meta.blk >= 0) {
+      if (!dead && !meta.timeout && meta.blk >= 0 && warp * 16 < meta.ntok) {
+        // warp w takes the stage's tiles w, w + 8, ... (rows past ntok are masked)
         if (!meta.is8) {
-          for (int mt = warp; mt < Geo<D, false>::MTILES; mt += kCW)
-            if (mt * 16 < meta.ntok) tile<D, NT, false>(st, stg, mt * 16, meta.ntok, bq, qs, sc2, lane);
-        } else {
-          for (int mt = warp; mt < Geo<D, true>::MTILES; mt += kCW)
-            if (mt * 16 < meta.ntok) tile<D, NT, true>(st, stg, mt * 16, meta.ntok, bq, qs, sc2, lane);
+          constexpr int NTL = Geo<D, false>::MTILES / kCW;
+          int r0[NTL];
+#pragma unroll
+          for (int i = 0; i < NTL; ++i) r0[i] = (warp + i * kCW) * 16;
+          tiles<D, NT, false, NTL>(st, stg, r0, meta.ntok, bq, qs, ks, lane);
+        } else if (warp < Geo<D, true>::MTILES) {
+          constexpr int NTL = Geo<D, true>::MTILES >= kCW ? Geo<D, true>::MTILES / kCW : 1;
+          int r0[NTL];
+#pragma unroll
+          for (int i = 0; i < NTL; ++i) r0[i] = (warp + i * kCW) * 16;
+          tiles<D, NT, true, NTL>(st, stg, r0, meta.ntok, bq, qs, ks, lane);
         }
       }
       __syncwarp();
@@ -654,7 +728,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
 
 size_t decode_tc_smem_bytes(int head_dim) {
   return static_cast<size_t>(kNS) * kStageBytes + 2 * kNS * sizeof(uint64_t) +
-         (8 * head_dim + 32 + kCW * 16) * sizeof(float) + static_cast<size_t>(kCW) * 1024 * sizeof(float);
+         (8 * head_dim + 64 + kCW * 16) * sizeof(float) + static_cast<size_t>(kCW) * 1024 * sizeof(float);
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stream) {

@@ -212,63 +212,86 @@ __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool v
   if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(sh, zh);
 }
 
+// One warp item = (group of VPW consecutive tokens, KV head).  Items are
+// walked with a grid stride; the next item's K/V rows are loaded before the
+// current one is encoded, so every warp keeps two items of loads in flight.
+template <typename InT>
+struct ItemLoad {
+  uint4 k0, k1, v0, v1;
+  int32_t blk;
+};
+
 template <int D, typename InT>
-__global__ void __launch_bounds__(256, 3) quantize_kernel(PoolView pool, const InT* __restrict__ k,
-                                                       const InT* __restrict__ v,
-                                                       int64_t n_tokens, int64_t stride,
-                                                       const int32_t* __restrict__ block_ids,
-                                                       int64_t n_items) {
+__device__ __forceinline__ void load_item(uint32_t item, uint32_t hkv, int r, int j, uint32_t n_tokens,
+                                          int64_t stride, const InT* __restrict__ k,
+                                          const InT* __restrict__ v,
+                                          const int32_t* __restrict__ block_ids, ItemLoad<InT>& L) {
+  using S = Shape<D>;
+  const uint32_t grp = item / hkv, h = item - grp * hkv;
+  const uint32_t t0 = grp * S::VPW, t = t0 + r;
+  L.blk = __ldg(block_ids + t0 / kBlockTokens);
+  L.k0 = L.k1 = L.v0 = L.v1 = make_uint4(0, 0, 0, 0);
+  if (t < n_tokens) {
+    const int64_t src = static_cast<int64_t>(t) * stride + h * D + j * kEPL;
+    L.k0 = __ldg(reinterpret_cast<const uint4*>(k + src));
+    L.k1 = __ldg(reinterpret_cast<const uint4*>(k + src) + 1);
+    L.v0 = __ldg(reinterpret_cast<const uint4*>(v + src));
+    L.v1 = __ldg(reinterpret_cast<const uint4*>(v + src) + 1);
+  }
+}
+
+template <int D, typename InT>
+__global__ void __launch_bounds__(256, 2) quantize_kernel(PoolView pool, const InT* __restrict__ k,
+                                                          const InT* __restrict__ v,
+                                                          uint32_t n_tokens, int64_t stride,
+                                                          const int32_t* __restrict__ block_ids,
+                                                          uint32_t n_items) {
   using S = Shape<D>;
   const int lane = threadIdx.x & 31;
   const int r = lane / S::LPV;
   const int j = lane % S::LPV;
-  const int hkv = pool.n_kv_heads;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const uint32_t hkv = pool.n_kv_heads;
+  const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
+  uint32_t item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (item >= n_items) return;
 
-  for (int64_t item = warp0; item < n_items; item += n_warps) {
-    const int64_t group_of_tokens = item / hkv;
-    const int h = static_cast<int>(item - group_of_tokens * hkv);
-    const int64_t t0 = group_of_tokens * S::VPW;
-    const int64_t t = t0 + r;
+  ItemLoad<InT> cur, nxt;
+  load_item<D, InT>(item, hkv, r, j, n_tokens, stride, k, v, block_ids, cur);
+  for (; item < n_items; item += n_warps) {
+    const uint32_t next = item + n_warps;
+    if (next < n_items) load_item<D, InT>(next, hkv, r, j, n_tokens, stride, k, v, block_ids, nxt);
+
+    const uint32_t grp = item / hkv, h = item - grp * hkv;
+    const uint32_t t0 = grp * S::VPW, t = t0 + r;
     const bool valid = t < n_tokens;
-    const int32_t blk = __ldg(block_ids + t0 / kBlockTokens);
+    const int32_t blk = cur.blk;
     if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
       if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
-      continue;
+    } else {
+      const int slot = static_cast<int>(t % kBlockTokens);
+      const bool is8 = blk >= pool.n_q4;
+      const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+      const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
+      float2 x[8];
+      // keys: rotate, then code
+      unpack16<InT>(cur.k0, cur.k1, x);
+      if (pool.k_rotated) rotate_pairs<D>(x, j);
+      if (is8)
+        encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
+      else
+        encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
+      // values: code unrotated
+      unpack16<InT>(cur.v0, cur.v1, x);
+      if (is8)
+        encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+      else
+        encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+      // a freshly written slot is live
+      if (valid && h == 0 && j == 0)
+        atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32,
+                  ~(1u << (slot % 32)));
     }
-    const int slot = static_cast<int>(t % kBlockTokens);
-    const bool is8 = blk >= pool.n_q4;
-    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
-    const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
-
-    // issue all four 16-byte loads (K and V) before any arithmetic
-    uint4 kw0 = make_uint4(0, 0, 0, 0), kw1 = kw0, vw0 = kw0, vw1 = kw0;
-    if (valid) {
-      const int64_t src = t * stride + static_cast<int64_t>(h) * D + j * kEPL;
-      kw0 = __ldg(reinterpret_cast<const uint4*>(k + src));
-      kw1 = __ldg(reinterpret_cast<const uint4*>(k + src) + 1);
-      vw0 = __ldg(reinterpret_cast<const uint4*>(v + src));
-      vw1 = __ldg(reinterpret_cast<const uint4*>(v + src) + 1);
-    }
-    float2 x[8];
-    // keys: rotate, then code
-    unpack16<InT>(kw0, kw1, x);
-    if (pool.k_rotated) rotate_pairs<D>(x, j);
-    if (is8)
-      encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
-    else
-      encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
-    // values: code unrotated
-    unpack16<InT>(vw0, vw1, x);
-    if (is8)
-      encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
-    else
-      encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
-    // a freshly written slot is live
-    if (valid && h == 0 && j == 0)
-      atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32,
-                ~(1u << (slot % 32)));
+    cur = nxt;
   }
 }
 
@@ -437,11 +460,18 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
   const int d = pool.head_dim;
   const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;
   const int64_t n_items = ((n_tokens + vpw - 1) / vpw) * pool.n_kv_heads;
-  const dim3 grid(grid_for(n_items)), block(256);
+  if (n_items >= (int64_t{1} << 32) || n_tokens >= (int64_t{1} << 32)) return cudaErrorInvalidValue;
+  // two CTAs of 8 warps per SM, each warp with two items of loads in flight
+  const int sms = device_sm_count();
+  int64_t g = (n_items + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 2;
+  if (g > cap) g = cap;
+  const dim3 grid(static_cast<unsigned>(g < 1 ? 1 : g)), block(256);
+  const uint32_t nt = static_cast<uint32_t>(n_tokens), ni = static_cast<uint32_t>(n_items);
 #define Q4KV_LAUNCH_Q(DD, T)                                                          \
   quantize_kernel<DD, T><<<grid, block, 0, stream>>>(pool, static_cast<const T*>(k),  \
-                                                     static_cast<const T*>(v), n_tokens, \
-                                                     token_stride, block_ids, n_items)
+                                                     static_cast<const T*>(v), nt,    \
+                                                     token_stride, block_ids, ni)
   if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(128, __half);
   else if (d == 128) Q4KV_LAUNCH_Q(128, __nv_bfloat16);
   else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(256, __half);

@@ -203,3 +203,21 @@ def test_bad_table_entry_and_length():
     assert bits & 1 and bits & 2
     assert torch.all(out[1] == 0) and torch.all(out[2] == 0)
     assert torch.equal(out[0], good[0])
+
+
+@pytest.mark.parametrize("kernel", [1, 0])
+def test_long_sequences_with_mixed_widths_and_eviction(kernel):
+    # long contexts accumulate many tiles: checks the offset-form value
+    # accumulation and the lazy rescale over 32K tokens
+    c = Case([32768, 20000], hq=8, hkv=2, d=128, seed=13, n_pool=300, q8_blocks=range(60))
+    g = torch.Generator().manual_seed(14)
+    slots = []
+    for b, n in enumerate(c.lens):
+        pos = torch.randperm(n, generator=g)[: n // 3]
+        blk = c.tables[b].to(torch.int64)[pos // 256]
+        slots.append(blk * 256 + pos % 256)
+    c.invalidate(torch.cat(slots))
+    want = c.oracle()
+    for s in (0, 1):
+        out, _ = c.run(s, kernel=kernel)
+        assert_close(out, want, what=f"long, splits {s}")
