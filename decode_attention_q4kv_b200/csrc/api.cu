@@ -241,6 +241,11 @@ q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan*
       !aligned(q, 16) || !aligned(block_tables, 16) || !aligned(seq_lens, 4) || !aligned(out, 16))
     return Q4KV_ERR_INVALID_ARG;
   if (pool->n_q4_blocks + pool->n_q8_blocks == 0) return Q4KV_ERR_INVALID_ARG;
+  // TMA row coordinates are int32: (blocks of one width) x heads x 256 < 2^31
+  const int64_t code_rows =
+      static_cast<int64_t>(pool->n_q4_blocks > pool->n_q8_blocks ? pool->n_q4_blocks : pool->n_q8_blocks) *
+      pool->n_kv_heads * kBlockTokens;
+  if (code_rows >= (int64_t{1} << 31)) return Q4KV_ERR_UNSUPPORTED;
   if (plan->workspace_bytes > 0 &&
       (workspace == nullptr || workspace_bytes < plan->workspace_bytes || !aligned(workspace, 256)))
     return Q4KV_ERR_WORKSPACE;

@@ -30,10 +30,12 @@
 //           weights come out of the key MMA in the accumulator layout; one
 //           movmatrix.trans per 8x8 turns them into the B operand.
 //
-// Data movement: a producer warp streams each (block, KV head) run of codes,
-// scales/zeros and the block's remap mask with 1-D TMA bulk copies
-// (cp.async.bulk, no multicast) into a 4-deep ring of shared-memory stages
-// guarded by mbarriers; 8 consumer warps each take 16-token tiles of a stage.
+// Data movement: a producer warp streams each (block, KV head) run of codes
+// with 2-D TMA tensor copies (cp.async.bulk.tensor, no multicast) that swizzle
+// 16-byte chunks across banks (64B pattern for 64-byte rows, 128B for 128-byte
+// rows), and the run's scales/zeros and the block's remap mask with 1-D bulk
+// copies, into a 4-deep ring of shared-memory stages guarded by mbarriers; 8
+// consumer warps each take 16-token tiles of a stage.
 // Every mbarrier wait is bounded: on time-out the kernel raises
 // Q4KV_DEVERR_TIMEOUT, poisons the affected rows and returns.
 //
@@ -41,7 +43,11 @@
 // (sequence, KV head, split) with a static stride; the producer runs ahead
 // across item boundaries.  Each item ends with a cross-warp log-sum-exp merge
 // in shared memory and writes either the final row (one split) or a partial.
+#include <cuda.h>   // CUtensorMap and its enums; the encoder is reached through the runtime
 #include <math.h>
+#include <string.h>
+
+#include <mutex>
 
 #include "q4kv_internal.cuh"
 
@@ -58,7 +64,8 @@ constexpr int kOffKP = 2 * kCodeBytes;
 constexpr int kOffVP = kOffKP + kParamBytes;
 constexpr int kOffMask = kOffVP + kParamBytes;
 constexpr int kOffMeta = kOffMask + 32;
-constexpr int kStageBytes = kOffMeta + 32;  // 36928, a multiple of 16
+constexpr int kStageBytes = 37 * 1024;      // 1024-byte aligned stages (128B swizzle atoms)
+static_assert(kOffMeta + 32 <= kStageBytes, "stage layout");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned kSpinLimit = 1u << 26;   // bounded mbarrier waits
 
@@ -114,6 +121,13 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_rows(void* dst, const CUtensorMap* map, int row, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void consumer_sync() {
@@ -177,7 +191,21 @@ struct Geo {
   static constexpr int MTILES = TS / 16;                // 16-token tiles per stage
   static constexpr int KB = Q8 ? D / 4 : D / 8;         // key bytes a thread owns per row
   static constexpr int VB = Q8 ? D / 8 : D / 16;        // value bytes a thread owns per row
+  static constexpr int SW = RB == 64 ? 64 : (RB == 128 ? 128 : 0);   // TMA swizzle span
   static_assert(TS * PB <= kParamBytes, "stage params");
+};
+
+// Byte offset of (row, byte) of a code tile in shared memory after the TMA
+// swizzle: the 16-byte chunk index is XOR-ed with address bits 7.. (row bits).
+template <int RB, int SW>
+__device__ __forceinline__ int swz(int row, int byte) {
+  if (SW == 128) return row * RB + ((((byte >> 4) ^ row) & 7) << 4) + (byte & 15);
+  if (SW == 64) return row * RB + ((((byte >> 4) ^ (row >> 1)) & 3) << 4) + (byte & 15);
+  return row * RB + byte;
+}
+
+struct TileMaps {       // one map per code array; unused ones stay zero
+  CUtensorMap k4, v4, k8, v8;
 };
 
 // Key A operand (u8) of 32-channel step kk for the thread's two rows.  Thread
@@ -268,6 +296,41 @@ __device__ __forceinline__ void reset(WarpState<D, NT>& st) {
   }
 }
 
+// Per-thread byte offsets inside a stage for the warp's first tile.  Tiles
+// start at multiples of 16 rows, so the token permutation and the TMA
+// swizzle depend only on the row's low four bits -- a per-thread constant --
+// and tile i of the warp sits a compile-time 128 * i rows further on.
+// Computing these once keeps address arithmetic out of the tile loop.
+template <int D, bool Q8>
+struct TileOffsets {
+  using G = Geo<D, Q8>;
+  static constexpr int NC = D / 128;                        // 128-channel chunks
+  static constexpr int NQ = G::KB / NC / 16;                // 16-byte key loads per chunk
+  int k[2][NC * NQ];   // key rows pi(g), pi(g + 8)
+  int v[4];            // value rows pi(2t), pi(2t+1), pi(2t+8), pi(2t+9) (thread g's bytes)
+  int p[2];            // parameter rows pi(g), pi(g + 8) (the thread's two groups)
+  int row[2];          // pi(g), pi(g + 8) relative to the warp's first tile
+
+  __device__ __forceinline__ void init(int warp, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int r0 = warp * 16;
+    const int rr[2] = {tok_perm(g), tok_perm(g + 8)};
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      row[x] = r0 + rr[x];
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+          k[x][c * NQ + q] = swz<G::RB, G::SW>(row[x], c * (G::RB / NC) + t * (G::KB / NC) + q * 16);
+      p[x] = row[x] * G::PB + ((G::NG == 2) ? 0 : 2 * (t & 1)) * 4;
+    }
+    const int vr[4] = {tok_perm(2 * t), tok_perm(2 * t + 1), tok_perm(2 * t + 8), tok_perm(2 * t + 9)};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) v[x] = swz<G::RB, G::SW>(r0 + vr[x], g * G::VB);
+  }
+};
+
 // NTILE 16-token tiles of one stage: keys for every tile, one online-softmax
 // update over all of them, then values.  The running max moves only when the
 // tile max exceeds it by more than kLazy (log2 units), so the accumulators are
@@ -275,29 +338,25 @@ __device__ __forceinline__ void reset(WarpState<D, NT>& st) {
 constexpr float kLazy = 2.0f;
 
 template <int D, int NT, bool Q8, int NTILE>
-__device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage, const int (&row0)[NTILE],
-                                      int nvalid, const uint32_t (&bq)[D / 32][NT][2][2],
+__device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage,
+                                      const TileOffsets<D, Q8>& o, int nvalid,
+                                      const uint32_t (&bq)[D / 32][NT][2][2],
                                       const float (&qs)[NT][2], const float (&ks)[NT], int lane) {
   using G = Geo<D, Q8>;
-  const int g = lane >> 2, t = lane & 3;
-  const int pg = tok_perm(g), pg8 = tok_perm(g + 8);
+  using O = TileOffsets<D, Q8>;
+  constexpr int kTileRows = kCW * 16;   // rows between a warp's tiles
+  const int t = lane & 3;
   // ---- keys ----
   float sk[NTILE][NT][4];
 #pragma unroll
   for (int i = 0; i < NTILE; ++i) {
     uint32_t rg[G::KB / 4], rg8[G::KB / 4];
-    const uint8_t* kc = stage + (row0[i] + pg) * G::RB;
-    const uint8_t* kc8 = stage + (row0[i] + pg8) * G::RB;
+    const uint8_t* base = stage + i * kTileRows * G::RB;
 #pragma unroll
-    for (int c = 0; c < D / 128; ++c) {
-#pragma unroll
-      for (int q = 0; q < G::KB / (D / 128) / 16; ++q) {
-        const int off = c * (G::RB / (D / 128)) + t * (G::KB / (D / 128)) + q * 16;
-        const uint4 u = lds<uint4>(kc + off), u8 = lds<uint4>(kc8 + off);
-        const int wi = c * (G::KB / (D / 128) / 4) + q * 4;
-        rg[wi] = u.x; rg[wi + 1] = u.y; rg[wi + 2] = u.z; rg[wi + 3] = u.w;
-        rg8[wi] = u8.x; rg8[wi + 1] = u8.y; rg8[wi + 2] = u8.z; rg8[wi + 3] = u8.w;
-      }
+    for (int n = 0; n < O::NC * O::NQ; ++n) {
+      const uint4 u = lds<uint4>(base + o.k[0][n]), u8 = lds<uint4>(base + o.k[1][n]);
+      rg[4 * n] = u.x; rg[4 * n + 1] = u.y; rg[4 * n + 2] = u.z; rg[4 * n + 3] = u.w;
+      rg8[4 * n] = u8.x; rg8[4 * n + 1] = u8.y; rg8[4 * n + 2] = u8.z; rg8[4 * n + 3] = u8.w;
     }
     int hi[NT][4], lo[NT][4];
 #pragma unroll
@@ -321,9 +380,6 @@ __device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage
   }
   // ---- per-token parameters and logits (log2 units) ----
   // D = 128: the thread's columns are (h, 0), (h, 1); D = 256: (h, 2 (t%2)), (h, 2 (t%2) + 1).
-  const int gbase = (G::NG == 2) ? 0 : 2 * (t & 1);
-  const uint8_t* kp = stage + kOffKP;
-  const uint8_t* vp = stage + kOffVP;
   const uint32_t* mask = reinterpret_cast<const uint32_t*>(stage + kOffMask);
   const int slot0 = reinterpret_cast<const StageMeta*>(stage + kOffMeta)->slot0;
   float logit[NTILE][NT][2];
@@ -331,16 +387,18 @@ __device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage
   bool live[NTILE][2];
 #pragma unroll
   for (int i = 0; i < NTILE; ++i) {
+    // the tile's 16 mask bits: slots slot0 + first row .. + 15 (16-aligned)
+    const int s16 = slot0 + o.row[0] - tok_perm((lane >> 2)) + i * kTileRows;   // first slot of the tile
+    const uint32_t mbits = mask[s16 >> 5] >> (s16 & 16);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int row = row0[i] + (r ? pg8 : pg);
+      const int row = o.row[r] + i * kTileRows;
       const bool valid = row < nvalid;
-      const int slot = slot0 + row;
-      const bool masked = valid && ((mask[slot >> 5] >> (slot & 31)) & 1u);
+      const bool masked = valid && ((mbits >> (row & 15)) & 1u);
       const bool lv = valid && !masked;
       live[i][r] = lv;
-      const uint2 kpw = lds<uint2>(kp + row * G::PB + gbase * 4);
-      const uint2 vpw = lds<uint2>(vp + row * G::PB + gbase * 4);
+      const uint2 kpw = lds<uint2>(stage + kOffKP + o.p[r] + i * kTileRows * G::PB);
+      const uint2 vpw = lds<uint2>(stage + kOffVP + o.p[r] + i * kTileRows * G::PB);
       const float2 k0 = __half22float2(u2h(kpw.x)), k1 = __half22float2(u2h(kpw.y));
       const float2 v0 = __half22float2(u2h(vpw.x)), v1 = __half22float2(u2h(vpw.y));
       // rows outside the range or remapped may hold any bytes (even NaN
@@ -409,17 +467,22 @@ __device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage
       bw[j][1] = movtrans(wb[i][j][1]);   // tokens pi(8+2t), pi(9+2t)
     }
     uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
-    const uint8_t* vc = stage + kOffV + g * G::VB;
-    const int r0 = row0[i] + tok_perm(2 * t), r1 = row0[i] + tok_perm(2 * t + 1);
-    const int r8 = row0[i] + tok_perm(2 * t + 8), r9 = row0[i] + tok_perm(2 * t + 9);
+    const uint8_t* vc = stage + kOffV + i * kTileRows * G::RB;
+    if (VW == 2) {
+      const uint2 a0 = lds<uint2>(vc + o.v[0]), a1 = lds<uint2>(vc + o.v[1]);
+      const uint2 a8 = lds<uint2>(vc + o.v[2]), a9 = lds<uint2>(vc + o.v[3]);
+      v0[0] = a0.x; v0[1] = a0.y; v1[0] = a1.x; v1[1] = a1.y;
+      v8[0] = a8.x; v8[1] = a8.y; v9[0] = a9.x; v9[1] = a9.y;
+    } else {
 #pragma unroll
-    for (int q = 0; q < VW; q += 2) {
-      const uint2 a0 = lds<uint2>(vc + r0 * G::RB + 4 * q);
-      const uint2 a1 = lds<uint2>(vc + r1 * G::RB + 4 * q);
-      const uint2 a8 = lds<uint2>(vc + r8 * G::RB + 4 * q);
-      const uint2 a9 = lds<uint2>(vc + r9 * G::RB + 4 * q);
-      v0[q] = a0.x; v0[q + 1] = a0.y; v1[q] = a1.x; v1[q + 1] = a1.y;
-      v8[q] = a8.x; v8[q + 1] = a8.y; v9[q] = a9.x; v9[q + 1] = a9.y;
+      for (int q = 0; q < VW; q += 4) {   // 16-byte pieces of the thread's bytes (never swizzle-split)
+        const uint4 a0 = lds<uint4>(vc + o.v[0] + 4 * q), a1 = lds<uint4>(vc + o.v[1] + 4 * q);
+        const uint4 a8 = lds<uint4>(vc + o.v[2] + 4 * q), a9 = lds<uint4>(vc + o.v[3] + 4 * q);
+        v0[q] = a0.x; v0[q + 1] = a0.y; v0[q + 2] = a0.z; v0[q + 3] = a0.w;
+        v1[q] = a1.x; v1[q + 1] = a1.y; v1[q + 2] = a1.z; v1[q + 3] = a1.w;
+        v8[q] = a8.x; v8[q + 1] = a8.y; v8[q + 2] = a8.z; v8[q + 3] = a8.w;
+        v9[q] = a9.x; v9[q + 1] = a9.y; v9[q + 2] = a9.z; v9[q + 3] = a9.w;
+      }
     }
 #pragma unroll
     for (int mv = 0; mv < D / 16; ++mv) {
@@ -432,8 +495,12 @@ __device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage
 }
 
 template <int D, int NT>
-__global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeArgs a, int n_items) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    decode_tc_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ TileMaps maps,
+                     int n_items) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // swizzled TMA tiles need 1024-byte aligned destinations
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kNS * kStageBytes);
   uint64_t* empty = full + kNS;
@@ -512,10 +579,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
           const uint8_t* vc = (is8 ? P.v_codes8 : P.v_codes4) + row * rb;
           const uint8_t* kpp = reinterpret_cast<const uint8_t*>(is8 ? P.k_params8 : P.k_params4) + row * pb;
           const uint8_t* vpp = reinterpret_cast<const uint8_t*>(is8 ? P.v_params8 : P.v_params4) + row * pb;
-          const uint32_t cb = rows * rb, prb = rows * pb;
+          // codes: one TS-row box per tensor (the box never leaves the block)
+          const int ts = is8 ? Geo<D, true>::TS : Geo<D, false>::TS;
+          const uint32_t cb = static_cast<uint32_t>(ts) * rb, prb = rows * pb;
           mbar_arrive_tx(&full[s], 2 * cb + 2 * prb + 32);
-          bulk_g2s(stg, kc, cb, &full[s]);
-          bulk_g2s(stg + kOffV, vc, cb, &full[s]);
+          tma_rows(stg, is8 ? &maps.k8 : &maps.k4, static_cast<int>(row), &full[s]);
+          tma_rows(stg + kOffV, is8 ? &maps.v8 : &maps.v4, static_cast<int>(row), &full[s]);
+          (void)kc;
+          (void)vc;
           bulk_g2s(stg + kOffKP, kpp, prb, &full[s]);
           bulk_g2s(stg + kOffVP, vpp, prb, &full[s]);
           bulk_g2s(stg + kOffMask, P.mask + static_cast<int64_t>(meta.blk) * kMaskWords, 32, &full[s]);
@@ -544,6 +615,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
   float qs[NT][2], ks[NT];
   uint32_t it = 0;
   bool dead = false;
+  TileOffsets<D, false> off4;
+  off4.init(warp, lane);
 
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int split = item % S;
@@ -642,16 +715,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
         // warp w takes the stage's tiles w, w + 8, ... (rows past ntok are masked)
         if (!meta.is8) {
           constexpr int NTL = Geo<D, false>::MTILES / kCW;
-          int r0[NTL];
-#pragma unroll
-          for (int i = 0; i < NTL; ++i) r0[i] = (warp + i * kCW) * 16;
-          tiles<D, NT, false, NTL>(st, stg, r0, meta.ntok, bq, qs, ks, lane);
+          tiles<D, NT, false, NTL>(st, stg, off4, meta.ntok, bq, qs, ks, lane);
         } else if (warp < Geo<D, true>::MTILES) {
           constexpr int NTL = Geo<D, true>::MTILES >= kCW ? Geo<D, true>::MTILES / kCW : 1;
-          int r0[NTL];
-#pragma unroll
-          for (int i = 0; i < NTL; ++i) r0[i] = (warp + i * kCW) * 16;
-          tiles<D, NT, true, NTL>(st, stg, r0, meta.ntok, bq, qs, ks, lane);
+          TileOffsets<D, true> off8;   // 8-bit blocks are rare: offsets made on demand
+          off8.init(warp, lane);
+          tiles<D, NT, true, NTL>(st, stg, off8, meta.ntok, bq, qs, ks, lane);
         }
       }
       __syncwarp();
@@ -727,9 +796,45 @@ __global__ void __launch_bounds__(kThreadsTC, 1) decode_tc_kernel(const DecodeAr
 }  // namespace
 
 size_t decode_tc_smem_bytes(int head_dim) {
-  return static_cast<size_t>(kNS) * kStageBytes + 2 * kNS * sizeof(uint64_t) +
+  return 1024 + static_cast<size_t>(kNS) * kStageBytes + 2 * kNS * sizeof(uint64_t) +
          (8 * head_dim + 64 + kCW * 16) * sizeof(float) + static_cast<size_t>(kCW) * 1024 * sizeof(float);
 }
+
+namespace {
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn tensor_map_encoder() {
+  static std::once_flag once;
+  static EncodeFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+// Rows of `row_bytes` codes, `box_rows` rows per copy.
+bool encode_rows(EncodeFn enc, CUtensorMap* m, void* base, uint64_t rows, uint32_t row_bytes,
+                 uint32_t box_rows) {
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {row_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = row_bytes == 64    ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                                   : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stream) {
   const q4kv_decode_plan& p = a.plan;
@@ -738,12 +843,30 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
   const int g = p.n_q_heads / p.n_kv_heads;
   const int nt = (g * (p.head_dim / kGroup) + 7) / 8;
   const size_t smem = decode_tc_smem_bytes(p.head_dim);
+
+  EncodeFn enc = tensor_map_encoder();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  TileMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const int d = p.head_dim;
+  const uint64_t per_block = static_cast<uint64_t>(a.pool.n_kv_heads) * kBlockTokens;
+  const uint32_t ts4 = static_cast<uint32_t>(kCodeBytes / (d / 2)), ts8 = static_cast<uint32_t>(kCodeBytes / d);
+  if (a.pool.n_q4 > 0 &&
+      (!encode_rows(enc, &maps.k4, a.pool.k_codes4, a.pool.n_q4 * per_block, d / 2, ts4) ||
+       !encode_rows(enc, &maps.v4, a.pool.v_codes4, a.pool.n_q4 * per_block, d / 2, ts4)))
+    return cudaErrorInvalidValue;
+  if (a.pool.n_q8 > 0 &&
+      (!encode_rows(enc, &maps.k8, a.pool.k_codes8, a.pool.n_q8 * per_block, d, ts8) ||
+       !encode_rows(enc, &maps.v8, a.pool.v_codes8, a.pool.n_q8 * per_block, d, ts8)))
+    return cudaErrorInvalidValue;
+
   cudaError_t e = cudaSuccess;
 #define Q4KV_TC(DD, NN)                                                                           \
   do {                                                                                            \
     e = cudaFuncSetAttribute(decode_tc_kernel<DD, NN>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(smem));                                             \
-    if (e == cudaSuccess) decode_tc_kernel<DD, NN><<<grid, kThreadsTC, smem, stream>>>(a, n_items); \
+    if (e == cudaSuccess)                                                                         \
+      decode_tc_kernel<DD, NN><<<grid, kThreadsTC, smem, stream>>>(a, maps, n_items);             \
   } while (0)
   if (p.head_dim == 128 && nt == 1) Q4KV_TC(128, 1);
   else if (p.head_dim == 128) Q4KV_TC(128, 2);
