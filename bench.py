@@ -155,7 +155,7 @@ class Job:
         self.n_q4 = n_pool - self.n_q8
         self.layers = []
         for l in layer_ids:
-            lid = l + 1000 * rank
+            lid = rank_layer_id(l, rank)
             k, v = W.kv_tokens(w, lid, n_tok, device)
             q = W.query(w, lid, device)
             pool = q4.Q4KVPool(w.n_kv_heads, w.head_dim, self.n_q4, self.n_q8, device=device)
@@ -241,6 +241,31 @@ class Job:
         return self.n_layers * (self.quant_bytes + self.decode_bytes)
 
 
+# ---------------------------------------------------------------------------
+# multi-rank plumbing (weak scaling: every rank runs its own replica)
+# ---------------------------------------------------------------------------
+
+def rank_layer_id(layer: int, rank: int) -> int:
+    """Input stream of `layer` on `rank`: ranks draw disjoint data."""
+    return layer + 1000 * rank
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of `value` over all ranks of the default process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, bytes_per_step: float, steps: int, elapsed_s: float) -> float:
+    """Whole-job GB/s: every rank moved bytes_per_step per step; time = slowest rank."""
+    return world * bytes_per_step * steps / elapsed_s / 1e9
+
+
 def sources_digest():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decode_attention_q4kv_b200", "csrc")
@@ -313,11 +338,7 @@ def run_gpu(args):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    elapsed = start.elapsed_time(stop) / 1e3
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = reduce_max(start.elapsed_time(stop) / 1e3, dev)
     q_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
     d_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
 
@@ -357,7 +378,7 @@ def run_gpu(args):
                         traffic=traffic_for(f"decode:{w.name}"),
                         kernel="decode", algorithmic_bytes_per_launch=job.decode_bytes,
                         us_per_launch=round(d_cold_ms * 1e3, 2), peak_source=f"{peak_src} hbm_gbs (burst copy)")
-        value = world * job.bytes_per_step * args.steps / elapsed / 1e9
+        value = job_throughput(world, job.bytes_per_step, args.steps, elapsed)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -425,16 +446,11 @@ def run_e2e(job, args, dev, world):
         one_step()
     b.record()
     torch.cuda.synchronize()
-    el = a.elapsed_time(b) / 1e3
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([el], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        el = float(t.item())
+    el = reduce_max(a.elapsed_time(b) / 1e3, dev)
     L0 = job.layers[0]
     h2d = job.n_layers * sum(L0[x].numel() * L0[x].element_size() for x in ("k", "v", "q"))
     d2h = job.n_layers * L0["out"].numel() * L0["out"].element_size()
-    return {"value": round(world * job.bytes_per_step * steps / el / 1e9, 2), "unit": "GB/s",
+    return {"value": round(job_throughput(world, job.bytes_per_step, steps, el), 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "inputs copied from pinned host memory and the fp16 output read back, per layer, inside the timed region"}
 
