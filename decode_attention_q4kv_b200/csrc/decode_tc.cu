@@ -622,46 +622,75 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const int split = item % S;
     const int kvh = (item / S) % hkv;
     const int b = item / (S * hkv);
-    // ---- rotated query of the item's G heads -> 16-bit fixed point -> B fragments ----
-    for (int i = threadIdx.x; i < G * D; i += kCW * 32) {
-      const int64_t qi = (static_cast<int64_t>(b) * hq + kvh * G) * D + i;
-      qrot[i] = a.q_dtype == Q4KV_F16 ? __half2float(static_cast<const __half*>(a.q)[qi])
-                                      : __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qi]);
-    }
-    consumer_sync();
-    if (P.k_rotated) {
-      for (int hs = 1; hs < D; hs <<= 1) {
-        for (int i = threadIdx.x; i < G * (D / 2); i += kCW * 32) {
-          const int h = i / (D / 2), p = i % (D / 2);
-          const int lo = h * D + (p / hs) * 2 * hs + (p % hs), hi = lo + hs;
-          const float x = qrot[lo], y = qrot[hi];
-          qrot[lo] = x + y;
-          qrot[hi] = x - y;
-        }
-        consumer_sync();
-      }
-      const float c = rotation_constant(D);
-      for (int i = threadIdx.x; i < G * D; i += kCW * 32) qrot[i] *= c;
-      consumer_sync();
-    }
-    // warp h < G: scale 2^E with max |q_rot[h]| * 2^E <= 32000, then q_int = rne(q_rot * 2^E)
+    // ---- warp h < G: rotate query head h in registers, scale it to 16-bit
+    // fixed point (max |q_rot| * 2^E <= 32000) and sum it per group ----
     if (warp < G) {
+      constexpr int E = D / 32;                   // lane holds channels E*lane .. E*lane + E-1
+      float x[E];
+      const int64_t qi = ((static_cast<int64_t>(b) * hq + kvh * G + warp) * D + E * lane);
+      if (E == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(a.q) + 2 * qi);
+        const uint32_t ww[2] = {w.x, w.y};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t h16 = (ww[e / 2] >> (16 * (e % 2))) & 0xFFFFu;
+          x[e] = a.q_dtype == Q4KV_F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(h16)))
+                                       : __uint_as_float(h16 << 16);
+        }
+      } else {
+        const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.q) + 2 * qi);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint32_t h16 = (ww[e / 2] >> (16 * (e % 2))) & 0xFFFFu;
+          x[e] = a.q_dtype == Q4KV_F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(h16)))
+                                       : __uint_as_float(h16 << 16);
+        }
+      }
+      if (P.k_rotated) {   // c * H q: butterflies inside the lane, then across lanes (fp32)
+#pragma unroll
+        for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if ((e & h) == 0) {
+              const float u = x[e], v = x[e + h];
+              x[e] = u + v;
+              x[e + h] = u - v;
+            }
+#pragma unroll
+        for (int h = E; h < D; h <<= 1) {
+          const int lb = h / E;
+          const bool upper = (lane & lb) != 0;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[e], lb);
+            x[e] = upper ? o - x[e] : x[e] + o;
+          }
+        }
+        const float c = rotation_constant(D);
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] *= c;
+      }
       float mx = 0.0f;
-      for (int c = lane; c < D; c += 32) mx = fmaxf(mx, fabsf(qrot[warp * D + c]));
+#pragma unroll
+      for (int e = 0; e < E; ++e) mx = fmaxf(mx, fabsf(x[e]));
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      int e = 0;
-      if (mx > 0.0f) e = static_cast<int>(floorf(log2f(32000.0f / mx)));
-      e = max(-100, min(100, e));
-      for (int c = lane; c < D; c += 32) qrot[warp * D + c] = rintf(ldexpf(qrot[warp * D + c], e));
-      if (lane == 0) qsum[32 + warp] = ldexpf(1.0f, -e);       // 2^-E of head `warp`
-    }
-    consumer_sync();
-    if (threadIdx.x < G * NG) {   // exact group sums of the integer query
-      const int h = threadIdx.x / NG, gr = threadIdx.x % NG;
-      float acc = 0.0f;
-      for (int c = 0; c < kGroup; ++c) acc += qrot[h * D + gr * kGroup + c];
-      qsum[h * 4 + gr] = acc;
+      int ex = 0;
+      if (mx > 0.0f) ex = static_cast<int>(floorf(log2f(32000.0f / mx)));
+      ex = max(-100, min(100, ex));
+      float part = 0.0f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float qv = rintf(ldexpf(x[e], ex));
+        qrot[warp * D + E * lane + e] = qv;
+        part += qv;
+      }
+      // exact group sums: the 64 / E lanes of a group are consecutive
+#pragma unroll
+      for (int off = 1; off < kGroup / E; off <<= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (lane % (kGroup / E) == 0) qsum[warp * 4 + lane / (kGroup / E)] = part;
+      if (lane == 0) qsum[32 + warp] = ldexpf(1.0f, -ex);        // 2^-E of head `warp`
     }
     consumer_sync();
 #pragma unroll
