@@ -275,32 +275,80 @@ __global__ void __launch_bounds__(kThreads) decode_simple_kernel(const DecodeArg
 // Log-sum-exp merge of the splits of one (sequence, query head) row:
 //   M = max m_i, L = sum l_i e^(m_i - M), out = sum o_i e^(m_i - M) / L.
 // A poisoned split (l < 0) or an empty row (M = -inf) gives 0.
+// Log-sum-exp merge of the S partials of one query row:
+//   M = max m_i,  w_i = e^(m_i - M),  out = sum w_i o_i / sum w_i l_i.
+// A poisoned split (l < 0) or a row with no token gives 0.  Thread i owns
+// channels 4i .. 4i+3; the weights are computed once per split and shared
+// through shared memory, so the channel loop is one float4 load and four
+// FMAs per split.
+template <int T>
+__device__ __forceinline__ float block_reduce(float x, bool is_max, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float y = __shfl_xor_sync(0xffffffffu, x, off);
+    x = is_max ? fmaxf(x, y) : x + y;
+  }
+  if (T > 32) {
+    __syncthreads();   // red may still be read by the previous reduction
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = x;
+    __syncthreads();
+    x = red[0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) x = is_max ? fmaxf(x, red[w]) : x + red[w];
+  }
+  return x;
+}
+
 template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(D / 4) merge_kernel(const DecodeArgs a) {
+  constexpr int T = D / 4;
+  constexpr int kChunk = 256;   // splits whose weights are staged at a time
+  __shared__ float wgt[kChunk];
+  __shared__ float red[T / 32];
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t row = blockIdx.x;
   const int S = a.plan.n_splits;
-  const float* ml = a.ws_ml + row * S * 2;
-  float M = -INFINITY;
-  bool poisoned = false;
-  for (int i = 0; i < S; ++i) {
-    M = fmaxf(M, ml[2 * i]);
-    poisoned |= ml[2 * i + 1] < 0.0f;
+  const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row * S;
+  float M = -INFINITY, pois = 0.0f;
+  for (int i = threadIdx.x; i < S; i += T) {
+    const float2 v = ml[i];
+    M = fmaxf(M, v.x);
+    pois = fmaxf(pois, v.y < 0.0f ? 1.0f : 0.0f);
   }
-  for (int j = threadIdx.x; j < D; j += blockDim.x) {
-    float res = 0.0f;
-    if (!poisoned && M != -INFINITY) {
-      float num = 0.0f, den = 0.0f;
-      for (int i = 0; i < S; ++i) {
-        const float m = ml[2 * i];
-        if (m == -INFINITY) continue;
-        const float w = expf(m - M);
-        den = fmaf(ml[2 * i + 1], w, den);
-        num = fmaf(a.ws_o[(row * S + i) * D + j], w, num);
-      }
-      res = num / den;
+  M = block_reduce<T>(M, true, red);
+  pois = block_reduce<T>(pois, true, red);
+  float L = 0.0f;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  const float4* o = reinterpret_cast<const float4*>(a.ws_o + row * S * D) + threadIdx.x;
+  for (int c0 = 0; c0 < S; c0 += kChunk) {
+    const int n = min(kChunk, S - c0);
+    __syncthreads();   // the previous chunk's weights are consumed
+    for (int i = threadIdx.x; i < n; i += T) {
+      const float2 v = ml[c0 + i];
+      const float w = (M == -INFINITY || v.x == -INFINITY) ? 0.0f : expf(v.x - M);
+      wgt[i] = w;
+      L = fmaf(v.y, w, L);
     }
-    store_out(a.out, a.out_dtype, row * D + j, res);
+    __syncthreads();
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
+      const float w = wgt[i];
+      if (w == 0.0f) continue;   // an empty split adds nothing
+      const float4 x = o[static_cast<int64_t>(c0 + i) * T];
+      acc.x = fmaf(x.x, w, acc.x);
+      acc.y = fmaf(x.y, w, acc.y);
+      acc.z = fmaf(x.z, w, acc.z);
+      acc.w = fmaf(x.w, w, acc.w);
+    }
   }
+  L = block_reduce<T>(L, false, red);
+  const bool ok = pois == 0.0f && M != -INFINITY && L > 0.0f;
+  const int64_t base = row * D + 4 * threadIdx.x;
+  store_out(a.out, a.out_dtype, base, ok ? acc.x / L : 0.0f);
+  store_out(a.out, a.out_dtype, base + 1, ok ? acc.y / L : 0.0f);
+  store_out(a.out, a.out_dtype, base + 2, ok ? acc.z / L : 0.0f);
+  store_out(a.out, a.out_dtype, base + 3, ok ? acc.w / L : 0.0f);
 }
 
 }  // namespace
@@ -320,11 +368,8 @@ int device_sm_count() {
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream) {
   const q4kv_decode_plan& p = a.plan;
   const unsigned rows = static_cast<unsigned>(p.batch) * p.n_q_heads;
-  if (p.head_dim == 128)
-    merge_kernel<128><<<rows, 128, 0, stream>>>(a);
-  else
-    merge_kernel<256><<<rows, 128, 0, stream>>>(a);
-  return cudaGetLastError();
+  if (p.head_dim == 128) return launch_pdl(merge_kernel<128>, dim3(rows), dim3(32), 0, stream, a);
+  return launch_pdl(merge_kernel<256>, dim3(rows), dim3(64), 0, stream, a);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {

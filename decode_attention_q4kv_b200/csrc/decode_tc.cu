@@ -345,7 +345,6 @@ __device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage
   using G = Geo<D, Q8>;
   using O = TileOffsets<D, Q8>;
   constexpr int kTileRows = kCW * 16;   // rows between a warp's tiles
-  const int t = lane & 3;
   // ---- keys ----
   float sk[NTILE][NT][4];
 #pragma unroll
@@ -504,12 +503,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   uint8_t* stages = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kNS * kStageBytes);
   uint64_t* empty = full + kNS;
-  float* qrot = reinterpret_cast<float*>(empty + kNS);                 // [G][D]
+  float* qrot = reinterpret_cast<float*>(empty + kNS);                 // query digit table, 2 G D bytes
   float* qsum = qrot + 8 * D;                                          // [8][4] sums, [32 + h] scales
   float* mrg_ml = qsum + 64;                                           // [kCW][8][2]
   float* mrg_o = mrg_ml + kCW * 16;                                    // [kCW][G][D]
   __shared__ int s_flags[2];                                            // poison, timeout
 
+  griddep_wait();   // earlier kernels in the stream (the encoder) have finished
+  griddep_launch_dependents();
   const PoolView& P = a.pool;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hkv = P.n_kv_heads, hq = a.plan.n_q_heads, G = hq / hkv;
@@ -679,12 +680,37 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       int ex = 0;
       if (mx > 0.0f) ex = static_cast<int>(floorf(log2f(32000.0f / mx)));
       ex = max(-100, min(100, ex));
+      // digits of the fixed-point query, written straight into the B-operand
+      // table: entry (h, kk, t) is 16 bytes = words (low digit, r = 0),
+      // (low, r = 1), (high, r = 0), (high, r = 1); byte e of word r is the
+      // digit of channel 128 (kk / 4) + 32 t + 8 (kk % 4) + r + 2 e.  With
+      // q = 256 hi + lo, lo in [-128, 127]: lo = q mod 256, hi = (q + 128) >> 8.
       float part = 0.0f;
+      uint32_t lo8[E], hi8[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const float qv = rintf(ldexpf(x[e], ex));
-        qrot[warp * D + E * lane + e] = qv;
-        part += qv;
+        const float qf = rintf(ldexpf(x[e], ex));
+        part += qf;
+        const int qv = static_cast<int>(qf);
+        lo8[e] = static_cast<uint32_t>(qv) & 255u;
+        hi8[e] = static_cast<uint32_t>((qv + 128) >> 8) & 255u;
+      }
+      uint8_t* tbl = reinterpret_cast<uint8_t*>(qrot) + warp * (D / 32) * 64;
+      if constexpr (E == 8) {   // lane = channels 8 lane + [0, 8): kk = 4 (lane / 16) + lane % 4, t = (lane / 4) % 4
+        const int kk = 4 * (lane >> 4) + (lane & 3), tt = (lane >> 2) & 3;
+        uint4 w;
+        w.x = lo8[0] | lo8[2] << 8 | lo8[4] << 16 | lo8[6] << 24;
+        w.y = lo8[1] | lo8[3] << 8 | lo8[5] << 16 | lo8[7] << 24;
+        w.z = hi8[0] | hi8[2] << 8 | hi8[4] << 16 | hi8[6] << 24;
+        w.w = hi8[1] | hi8[3] << 8 | hi8[5] << 16 | hi8[7] << 24;
+        *reinterpret_cast<uint4*>(tbl + (kk * 4 + tt) * 16) = w;
+      } else {        // lane = channels 4 lane + [0, 4): bytes 2 (lane % 2), +1 of each word
+        const int kk = (lane >> 1) & 3, tt = lane >> 3;
+        uint16_t* h16 = reinterpret_cast<uint16_t*>(tbl + (kk * 4 + tt) * 16) + (lane & 1);
+        h16[0] = static_cast<uint16_t>(lo8[0] | lo8[2] << 8);
+        h16[2] = static_cast<uint16_t>(lo8[1] | lo8[3] << 8);
+        h16[4] = static_cast<uint16_t>(hi8[0] | hi8[2] << 8);
+        h16[6] = static_cast<uint16_t>(hi8[1] | hi8[3] << 8);
       }
       // exact group sums: the 64 / E lanes of a group are consecutive
 #pragma unroll
@@ -697,24 +723,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int j = 0; j < NT; ++j) {
       const int col = 8 * j + g;                // this thread's B column
       const int h = col / NG, gr = col % NG;
+      const uint4* tbl = reinterpret_cast<const uint4*>(qrot) + (h < G ? h : 0) * (D / 32) * 4 + t;
 #pragma unroll
       for (int kk = 0; kk < D / 32; ++kk) {
-        const int base = 128 * (kk / 4) + 32 * t + 8 * (kk % 4);
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {           // register r: channels base + r + {0, 2, 4, 6}
-          uint32_t d0 = 0, d1 = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int ch = base + r + 2 * e;
-            const int qv = (h < G && ch / kGroup == gr) ? static_cast<int>(qrot[h * D + ch]) : 0;
-            const int q0 = ((qv + 128) & 255) - 128;     // balanced low digit
-            const int q1 = (qv - q0) >> 8;               // high digit, |q1| <= 125
-            d0 |= static_cast<uint32_t>(q0 & 255) << (8 * e);
-            d1 |= static_cast<uint32_t>(q1 & 255) << (8 * e);
-          }
-          bq[kk][j][0][r] = d0;
-          bq[kk][j][1][r] = d1;
-        }
+        // channels of step kk for this t lie in group 2 (kk / 4) + t / 2
+        const bool use = h < G && 2 * (kk / 4) + (t >> 1) == gr;
+        uint4 w = tbl[kk * 4];
+        if (!use) w = make_uint4(0u, 0u, 0u, 0u);
+        bq[kk][j][0][0] = w.x;
+        bq[kk][j][0][1] = w.y;
+        bq[kk][j][1][0] = w.z;
+        bq[kk][j][1][1] = w.w;
       }
       {
         const int c2 = 8 * j + 2 * t;             // the thread's accumulator columns c2, c2 + 1
@@ -895,7 +914,8 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
     e = cudaFuncSetAttribute(decode_tc_kernel<DD, NN>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(smem));                                             \
     if (e == cudaSuccess)                                                                         \
-      decode_tc_kernel<DD, NN><<<grid, kThreadsTC, smem, stream>>>(a, maps, n_items);             \
+      e = launch_pdl(decode_tc_kernel<DD, NN>, dim3(grid), dim3(kThreadsTC), smem, stream, a, maps, \
+                     n_items);                                                                    \
   } while (0)
   if (p.head_dim == 128 && nt == 1) Q4KV_TC(128, 1);
   else if (p.head_dim == 128) Q4KV_TC(128, 2);

@@ -74,6 +74,35 @@ __device__ __forceinline__ float to_float<__nv_bfloat16>(__nv_bfloat16 x) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  The hot kernels (encoder, tensor-core
+// decode, split merge) are launched so that they may start while the kernel
+// before them in the stream drains, and each lets its own successor start
+// early.  Such a kernel executes griddep_wait() before it touches any global
+// memory: that returns once every earlier grid has completed and its writes
+// are visible, so the stream order of results is unchanged.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// ---------------------------------------------------------------------------
 // launchers (each returns cudaGetLastError() of its launch)
 // ---------------------------------------------------------------------------
 cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, int in_dtype,

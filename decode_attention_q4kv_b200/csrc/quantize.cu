@@ -253,6 +253,8 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(PoolView pool, const I
   const uint32_t hkv = pool.n_kv_heads;
   const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
   uint32_t item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  griddep_wait();   // the inputs may come from the kernel before in the stream
+  griddep_launch_dependents();
   if (item >= n_items) return;
 
   ItemLoad<InT> cur, nxt;
@@ -468,16 +470,14 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
   if (g > cap) g = cap;
   const dim3 grid(static_cast<unsigned>(g < 1 ? 1 : g)), block(256);
   const uint32_t nt = static_cast<uint32_t>(n_tokens), ni = static_cast<uint32_t>(n_items);
-#define Q4KV_LAUNCH_Q(DD, T)                                                          \
-  quantize_kernel<DD, T><<<grid, block, 0, stream>>>(pool, static_cast<const T*>(k),  \
-                                                     static_cast<const T*>(v), nt,    \
-                                                     token_stride, block_ids, ni)
-  if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(128, __half);
-  else if (d == 128) Q4KV_LAUNCH_Q(128, __nv_bfloat16);
-  else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(256, __half);
-  else Q4KV_LAUNCH_Q(256, __nv_bfloat16);
+#define Q4KV_LAUNCH_Q(DD, T)                                                                 \
+  launch_pdl(quantize_kernel<DD, T>, grid, block, 0, stream, pool, static_cast<const T*>(k), \
+             static_cast<const T*>(v), nt, token_stride, block_ids, ni)
+  if (d == 128 && in_dtype == Q4KV_F16) return Q4KV_LAUNCH_Q(128, __half);
+  if (d == 128) return Q4KV_LAUNCH_Q(128, __nv_bfloat16);
+  if (in_dtype == Q4KV_F16) return Q4KV_LAUNCH_Q(256, __half);
+  return Q4KV_LAUNCH_Q(256, __nv_bfloat16);
 #undef Q4KV_LAUNCH_Q
-  return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,
