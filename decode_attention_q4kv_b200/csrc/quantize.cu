@@ -20,6 +20,7 @@
 // subtraction and division for each code, round-half-even to an integer,
 // clamp.  Dequantisation is fma(code, s, z), equal to code*s + z because the
 // product is exact.
+#include "async_copy.cuh"
 #include "q4kv_internal.cuh"
 
 namespace q4kv {
@@ -92,6 +93,8 @@ __device__ __forceinline__ void rotate_pairs(float2 (&x)[8], int j) {
   for (int p = 0; p < 8; ++p) x[p] = __fmul2_rn(x[p], make_float2(c, c));
 }
 
+__device__ __forceinline__ uint4 lds16(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+
 template <typename T>
 __device__ __forceinline__ void unpack16(const uint4& w0, const uint4& w1, float2 (&x)[8]) {
   static_assert(sizeof(T) == 2, "16-bit inputs");
@@ -116,23 +119,37 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // the low mantissa bits.
 constexpr float kRoundMagic = 12582912.0f;
 
+// Correctly rounded quotient RN(u / s) for a divisor s whose significand
+// has at most 11 bits (every fp16 value, and the constants 15 and 255), from
+// r = RN(1/s): q0 = RN(u r), the residual u - q0 s is exact under an FMA, and
+// one correction q1 = RN(q0 + (u - q0 s) r) gives RN(u / s).  This is
+// Markstein's correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990); the quotient is checked exhaustively for every 11-bit divisor
+// significand against every binary32 dividend significand (the steps scale
+// exactly with the exponents), and the codes it produces are checked
+// bit-exact against the oracle's IEEE division.
+__device__ __forceinline__ float quot(float u, float s, float r) {
+  const float q0 = __fmul_rn(u, r);
+  return __fmaf_rn(__fmaf_rn(-q0, s, u), r, q0);
+}
+
 // Encode the lane's 16 values (one quarter of a 64-value group) and store its
 // codes and, from the group's first lane, the group's (scale, zero).
 //
-// Codes are defined as clamp(rne(fl(fl(x - z) / s)), 0, L).  Fast path:
-// y = fl(x * r + (-z * r)) with r = fl(1/s), then k = rne(y).  With
-// |y - fl(fl(x - z)/s)| <= B = (4 (L + 1) + |z r|) 2^-24, k is the defined
-// code whenever y lies more than 2B away from a half-integer.  The fast path
-// is taken for a group only when |z r| <= 2^10 (so B < 2^-13) and every
-// value's quotient stays inside [-0.49, L + 0.49] (so no clamp is needed);
-// a lane whose values come within 2^-13 (4-bit) or 2^-12 (8-bit) of a
-// half-integer recomputes its codes with IEEE division.  Either way the codes
-// equal the definition.
+// Codes are defined as clamp(rne(fl(fl(x - z) / s)), 0, L): u = fl(x - z),
+// then the correctly rounded quotient above, then round-half-even to an
+// integer by adding 1.5 * 2^23.  The quotient is monotone in x, so when the
+// group's extremes give quotients in [-0.5, L + 0.5) no code needs the
+// clamp; other groups (a zero far outside the fp16 grid of the values) take
+// IEEE division and an integer clamp.
 template <int BITS>
 __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool valid,
                                              uint8_t* __restrict__ code_dst,
                                              __half2* __restrict__ param_dst) {
   constexpr int L = (1 << BITS) - 1;
+  // RN(1/L); 15 and 255 have 11-bit significands
+  constexpr float kRecipL = BITS == 4 ? 0x1.111112p-4f : 0x1.010102p-8f;
   float mn = min3(min3(min3(x[0].x, x[0].y, x[1].x), min3(x[1].y, x[2].x, x[2].y),
                        min3(x[3].x, x[3].y, x[4].x)),
                   min3(x[4].y, x[5].x, x[5].y), min3(x[6].x, x[6].y, min(x[7].x, x[7].y)));
@@ -146,58 +163,74 @@ __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool v
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
   mx = __fadd_rn(mx, 0.0f);
-  const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(L));
+  const float s = quot(__fsub_rn(mx, mn), static_cast<float>(L), kRecipL);
   const __half sh = __float2half_rn(s);
   const __half zh = __float2half_rn(mn);
   const float sf = __half2float(sh);
   const float zf = __half2float(zh);
 
-  uint32_t q[kEPL];   // code e in the low bits of q[e]; lane element e = pair e%8, half e/8
-  bool exact = true;
+  // Codes as floats.  4-bit: ke[i] = code of register pair 2i plus 1.5 * 2^23,
+  // ko[i] = code of pair 2i + 1, so ko * 16 + ke holds the byte of channels
+  // (2i, 2i + 1) (.x) and (2i + 8, 2i + 9) (.y) in its low bits.  8-bit:
+  // q[p] = codes of pair p (.x, .y) in the low bits.
+  float2 ke[4], ko[4];
+  uint32_t q[kEPL];
+  const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
   if (sf != 0.0f) {
     const float r = __frcp_rn(sf);
-    const float nzr = __fmul_rn(-zf, r);
-    const float t_lo = __fmaf_rn(mn, r, nzr), t_hi = __fmaf_rn(mx, r, nzr);
-    exact = fabsf(nzr) > 1024.0f || t_lo < -0.49f || t_hi > L + 0.49f;
-    if (!exact) {
-      constexpr float thr = 0.5f - (BITS == 4 ? 0x1p-13f : 0x1p-12f);
-      const float2 r2 = make_float2(r, r), n2 = make_float2(nzr, nzr);
-      const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
+    const float q_lo = quot(__fsub_rn(mn, zf), sf, r), q_hi = quot(__fsub_rn(mx, zf), sf, r);
+    if (q_lo >= -0.5f && q_hi < L + 0.5f) {
+      const float2 r2 = make_float2(r, r), ns2 = make_float2(-sf, -sf), nz2 = make_float2(-zf, -zf);
       const float2 mm2 = make_float2(-kRoundMagic, -kRoundMagic);
-      const float2 t2 = make_float2(-thr * thr, -thr * thr);
-      uint32_t all_neg = 0xffffffffu;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        const float2 y = __ffma2_rn(x[p], r2, n2);
-        const float2 yk = __fadd2_rn(y, m2);        // integer in the low bits
-        const float2 k = __fadd2_rn(yk, mm2);       // that integer as a float
-        const float2 d = sub2(y, k);                // distance to it, |d| <= 0.5
-        const float2 e = __ffma2_rn(d, d, t2);      // < 0 iff |d| < thr
-        all_neg &= __float_as_uint(e.x) & __float_as_uint(e.y);
-        q[p] = __float_as_uint(yk.x);
-        q[p + 8] = __float_as_uint(yk.y);
+        const float2 u = __fadd2_rn(x[p], nz2);            // fl(x - z)
+        const float2 q0 = __fmul2_rn(u, r2);
+        const float2 q1 = __ffma2_rn(__ffma2_rn(q0, ns2, u), r2, q0);   // fl(u / s)
+        const float2 yk = __fadd2_rn(q1, m2);              // rne(q1) in the low bits
+        if (BITS == 4) {
+          if (p % 2 == 0) ke[p / 2] = yk;
+          else ko[p / 2] = __fadd2_rn(yk, mm2);
+        } else {
+          q[p] = __float_as_uint(yk.x);
+          q[p + 8] = __float_as_uint(yk.y);
+        }
       }
-      exact = (all_neg >> 31) == 0;
-    }
-    if (exact) {
+    } else {
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        int r0 = __float2int_rn(__fdiv_rn(__fsub_rn(x[p].x, zf), sf));
-        int r1 = __float2int_rn(__fdiv_rn(__fsub_rn(x[p].y, zf), sf));
-        q[p] = static_cast<uint32_t>(min(max(r0, 0), L));
-        q[p + 8] = static_cast<uint32_t>(min(max(r1, 0), L));
+        const int r0 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].x, zf), sf)), 0), L);
+        const int r1 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].y, zf), sf)), 0), L);
+        if (BITS == 4) {
+          const float2 c = make_float2(static_cast<float>(r0), static_cast<float>(r1));
+          if (p % 2 == 0) ke[p / 2] = __fadd2_rn(c, m2);
+          else ko[p / 2] = c;
+        } else {
+          q[p] = static_cast<uint32_t>(r0);
+          q[p + 8] = static_cast<uint32_t>(r1);
+        }
       }
     }
   } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ke[i] = m2;
+      ko[i] = make_float2(0.0f, 0.0f);
+    }
 #pragma unroll
     for (int e = 0; e < kEPL; ++e) q[e] = 0;
   }
   if (!valid) return;
   if (BITS == 4) {
-    // byte b holds elements 2b (low nibble) and 2b+1 (high nibble)
+    // byte b holds elements 2b (low nibble) and 2b+1 (high nibble); the sums
+    // are exact (integers below 2^24)
     uint32_t b[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = (q[2 * i] & 15u) | ((q[2 * i + 1] & 15u) << 4);
+    for (int i = 0; i < 4; ++i) {
+      const float2 w = __ffma2_rn(ko[i], make_float2(16.0f, 16.0f), ke[i]);
+      b[i] = __float_as_uint(w.x);
+      b[i + 4] = __float_as_uint(w.y);
+    }
     const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
     *reinterpret_cast<uint2*>(code_dst + j * 8) = make_uint2(lo, hi);
@@ -212,88 +245,162 @@ __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool v
   if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(sh, zh);
 }
 
-// One warp item = (group of VPW consecutive tokens, KV head).  Items are
-// walked with a grid stride; the next item's K/V rows are loaded before the
-// current one is encoded, so every warp keeps two items of loads in flight.
-template <typename InT>
-struct ItemLoad {
-  uint4 k0, k1, v0, v1;
-  int32_t blk;
+// ---------------------------------------------------------------------------
+// Encoder kernel.  Persistent CTAs (one per SM): one producer warp streams
+// the K and V rows of a unit -- T consecutive tokens x a run of H' heads,
+// 16 KB of input per tensor -- into a 4-deep ring of shared-memory stages
+// with bulk copies (one copy per token row, or one per tensor when the run
+// is contiguous in memory); 16 consumer warps each encode one warp item of
+// the stage: VPW tokens of one head, a lane holding 16 channels.  T and H'
+// are chosen so that every full unit holds exactly 16 warp items.
+// ---------------------------------------------------------------------------
+constexpr int kQConsumers = 16;
+constexpr int kQThreads = (kQConsumers + 1) * 32;
+constexpr int kQStages = 4;
+constexpr int kQHalf = 16384;                 // input bytes of one tensor per stage
+constexpr int kQStageBytes = 2 * kQHalf;
+
+struct EncodeGeometry {
+  uint32_t n_tokens;
+  int64_t stride;        // elements between consecutive tokens
+  int32_t unit_tokens;   // T
+  int32_t unit_heads;    // H'
+  int32_t head_chunks;   // ceil(Hkv / H')
+  uint32_t n_chunks;     // ceil(n_tokens / T)
 };
 
 template <int D, typename InT>
-__device__ __forceinline__ void load_item(uint32_t item, uint32_t hkv, int r, int j, uint32_t n_tokens,
-                                          int64_t stride, const InT* __restrict__ k,
-                                          const InT* __restrict__ v,
-                                          const int32_t* __restrict__ block_ids, ItemLoad<InT>& L) {
+__global__ void __launch_bounds__(kQThreads, 1)
+    quantize_kernel(const __grid_constant__ PoolView pool, const InT* __restrict__ k,
+                    const InT* __restrict__ v, const __grid_constant__ EncodeGeometry geo,
+                    const int32_t* __restrict__ block_ids) {
   using S = Shape<D>;
-  const uint32_t grp = item / hkv, h = item - grp * hkv;
-  const uint32_t t0 = grp * S::VPW, t = t0 + r;
-  L.blk = __ldg(block_ids + t0 / kBlockTokens);
-  L.k0 = L.k1 = L.v0 = L.v1 = make_uint4(0, 0, 0, 0);
-  if (t < n_tokens) {
-    const int64_t src = static_cast<int64_t>(t) * stride + h * D + j * kEPL;
-    L.k0 = __ldg(reinterpret_cast<const uint4*>(k + src));
-    L.k1 = __ldg(reinterpret_cast<const uint4*>(k + src) + 1);
-    L.v0 = __ldg(reinterpret_cast<const uint4*>(v + src));
-    L.v1 = __ldg(reinterpret_cast<const uint4*>(v + src) + 1);
-  }
-}
+  extern __shared__ __align__(128) uint8_t qsmem[];
+  uint8_t* stages = qsmem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + kQStages * kQStageBytes);
+  uint64_t* empty = full + kQStages;
+  __shared__ int s_timeout;
 
-template <int D, typename InT>
-__global__ void __launch_bounds__(256, 2) quantize_kernel(PoolView pool, const InT* __restrict__ k,
-                                                          const InT* __restrict__ v,
-                                                          uint32_t n_tokens, int64_t stride,
-                                                          const int32_t* __restrict__ block_ids,
-                                                          uint32_t n_items) {
-  using S = Shape<D>;
-  const int lane = threadIdx.x & 31;
-  const int r = lane / S::LPV;
-  const int j = lane % S::LPV;
-  const uint32_t hkv = pool.n_kv_heads;
-  const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
-  uint32_t item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   griddep_wait();   // the inputs may come from the kernel before in the stream
   griddep_launch_dependents();
-  if (item >= n_items) return;
-
-  ItemLoad<InT> cur, nxt;
-  load_item<D, InT>(item, hkv, r, j, n_tokens, stride, k, v, block_ids, cur);
-  for (; item < n_items; item += n_warps) {
-    const uint32_t next = item + n_warps;
-    if (next < n_items) load_item<D, InT>(next, hkv, r, j, n_tokens, stride, k, v, block_ids, nxt);
-
-    const uint32_t grp = item / hkv, h = item - grp * hkv;
-    const uint32_t t0 = grp * S::VPW, t = t0 + r;
-    const bool valid = t < n_tokens;
-    const int32_t blk = cur.blk;
-    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
-      if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
-    } else {
-      const int slot = static_cast<int>(t % kBlockTokens);
-      const bool is8 = blk >= pool.n_q4;
-      const int64_t phys = is8 ? blk - pool.n_q4 : blk;
-      const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
-      float2 x[8];
-      // keys: rotate, then code
-      unpack16<InT>(cur.k0, cur.k1, x);
-      if (pool.k_rotated) rotate_pairs<D>(x, j);
-      if (is8)
-        encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
-      else
-        encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
-      // values: code unrotated
-      unpack16<InT>(cur.v0, cur.v1, x);
-      if (is8)
-        encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
-      else
-        encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
-      // a freshly written slot is live
-      if (valid && h == 0 && j == 0)
-        atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32,
-                  ~(1u << (slot % 32)));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hkv = pool.n_kv_heads;
+  const int T = geo.unit_tokens, HP = geo.unit_heads, HC = geo.head_chunks;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kQConsumers);
     }
-    cur = nxt;
+    s_timeout = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kQConsumers) {
+    // ---------------- producer ----------------
+    if (lane != 0) return;
+    uint32_t it = 0;
+    bool stop = false;
+    for (uint32_t c = blockIdx.x; c < geo.n_chunks && !stop; c += gridDim.x) {
+      const uint32_t t0 = c * T;
+      const int nvalid = static_cast<int>(umin(static_cast<uint32_t>(T), geo.n_tokens - t0));
+      for (int hc = 0; hc < HC; ++hc, ++it) {
+        const int s = it % kQStages;
+        if (!mbar_wait(&empty[s], ((it / kQStages) & 1) ^ 1)) {
+          s_timeout = 1;
+          mbar_arrive(&full[s]);   // release the consumers; they see the flag
+          stop = true;
+          break;
+        }
+        const int h0 = hc * HP, nh = min(HP, hkv - h0);
+        const uint32_t row = static_cast<uint32_t>(nh) * D * sizeof(InT);   // bytes per token
+        uint8_t* dst = stages + s * kQStageBytes;
+        mbar_arrive_tx(&full[s], 2u * nvalid * row);
+        const InT* ks = k + static_cast<int64_t>(t0) * geo.stride + h0 * D;
+        const InT* vs = v + static_cast<int64_t>(t0) * geo.stride + h0 * D;
+        if (nh == hkv && geo.stride == static_cast<int64_t>(hkv) * D) {
+          bulk_g2s(dst, ks, nvalid * row, &full[s]);
+          bulk_g2s(dst + kQHalf, vs, nvalid * row, &full[s]);
+        } else {
+          for (int t = 0; t < nvalid; ++t) {
+            bulk_g2s(dst + t * row, ks + t * geo.stride, row, &full[s]);
+            bulk_g2s(dst + kQHalf + t * row, vs + t * geo.stride, row, &full[s]);
+          }
+        }
+      }
+    }
+    // no copy may still be landing when the CTA exits
+    for (uint32_t q = (it > kQStages ? it - kQStages : 0); q < it; ++q)
+      if (!mbar_wait(&full[q % kQStages], (q / kQStages) & 1)) break;
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  // warp w takes warp item w of each unit: head hh = w / tpi of the unit's
+  // run, tokens (w % tpi) * VPW .. + VPW - 1 of its T
+  const int r = lane / S::LPV;       // token of the warp item
+  const int j = lane % S::LPV;       // 16-channel run of the lane
+  const int tpi = T / S::VPW;        // warp items per head in a unit
+  const int hh = warp / tpi;
+  const int ti = (warp - hh * tpi) * S::VPW;   // first token of the item in the unit
+  const int tt = ti + r;
+  uint32_t it = 0;
+  bool dead = false;
+  int32_t blk_next = blockIdx.x < geo.n_chunks ? __ldg(block_ids + (blockIdx.x * T) / kBlockTokens) : 0;
+  for (uint32_t c = blockIdx.x; c < geo.n_chunks && !dead; c += gridDim.x) {
+    const uint32_t t0 = c * T;
+    const int32_t blk = blk_next;
+    if (c + gridDim.x < geo.n_chunks) blk_next = __ldg(block_ids + ((c + gridDim.x) * T) / kBlockTokens);
+    const uint32_t t = t0 + tt;
+    const bool valid = t < geo.n_tokens;
+    const int slot = static_cast<int>(t % kBlockTokens);
+    const bool bad_blk = blk < 0 || blk >= pool.n_q4 + pool.n_q8;
+    const bool is8 = blk >= pool.n_q4;
+    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+    for (int hc = 0; hc < HC; ++hc, ++it) {
+      const int s = it % kQStages;
+      if (!mbar_wait(&full[s], (it / kQStages) & 1) || s_timeout) {
+        if (lane == 0 && warp == 0) raise_error(pool.error_word, Q4KV_DEVERR_TIMEOUT);
+        dead = true;
+        break;
+      }
+      const int h0 = hc * HP, nh = min(HP, hkv - h0);
+      if (hh < nh) {
+        const uint8_t* src = stages + s * kQStageBytes + ((tt * nh + hh) * D + j * kEPL) * sizeof(InT);
+        const uint4 k0 = lds16(src), k1 = lds16(src + 16);
+        const uint4 v0 = lds16(src + kQHalf), v1 = lds16(src + kQHalf + 16);
+        const int h = h0 + hh;
+        if (bad_blk) {
+          if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
+        } else {
+          const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
+          float2 x[8];
+          // keys: rotate, then code
+          unpack16<InT>(k0, k1, x);
+          if (pool.k_rotated) rotate_pairs<D>(x, j);
+          if (is8)
+            encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
+          else
+            encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
+          // values: code unrotated
+          unpack16<InT>(v0, v1, x);
+          if (is8)
+            encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+          else
+            encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+          // freshly written slots are live: one word update for the item's tokens
+          const uint32_t tf = t0 + ti;
+          if (h == 0 && lane == 0 && tf < geo.n_tokens) {
+            const int nv = static_cast<int>(umin(static_cast<uint32_t>(S::VPW), geo.n_tokens - tf));
+            const int sf = static_cast<int>(tf % kBlockTokens);
+            atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + sf / 32,
+                      ~(((1u << nv) - 1u) << (sf % 32)));
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
   }
 }
 
@@ -459,25 +566,43 @@ inline int grid_for(int64_t n_items) {
 cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, int in_dtype,
                             int64_t n_tokens, int64_t token_stride, const int32_t* block_ids,
                             cudaStream_t stream) {
-  const int d = pool.head_dim;
+  const int d = pool.head_dim, hkv = pool.n_kv_heads;
+  if (n_tokens >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
+  // a unit holds T tokens x H' heads with T * H' * D = 8192 elements (16 KB of
+  // 16-bit input per tensor): H' the largest power of two <= Hkv that leaves
+  // T >= VPW, so a full unit is 16 warp items
   const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;
-  const int64_t n_items = ((n_tokens + vpw - 1) / vpw) * pool.n_kv_heads;
-  if (n_items >= (int64_t{1} << 32) || n_tokens >= (int64_t{1} << 32)) return cudaErrorInvalidValue;
-  // two CTAs of 8 warps per SM, each warp with two items of loads in flight
-  const int sms = device_sm_count();
-  int64_t g = (n_items + 7) / 8;
-  const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 2;
-  if (g > cap) g = cap;
-  const dim3 grid(static_cast<unsigned>(g < 1 ? 1 : g)), block(256);
-  const uint32_t nt = static_cast<uint32_t>(n_tokens), ni = static_cast<uint32_t>(n_items);
-#define Q4KV_LAUNCH_Q(DD, T)                                                                 \
-  launch_pdl(quantize_kernel<DD, T>, grid, block, 0, stream, pool, static_cast<const T*>(k), \
-             static_cast<const T*>(v), nt, token_stride, block_ids, ni)
-  if (d == 128 && in_dtype == Q4KV_F16) return Q4KV_LAUNCH_Q(128, __half);
-  if (d == 128) return Q4KV_LAUNCH_Q(128, __nv_bfloat16);
-  if (in_dtype == Q4KV_F16) return Q4KV_LAUNCH_Q(256, __half);
-  return Q4KV_LAUNCH_Q(256, __nv_bfloat16);
+  const int per_unit = 8192 / d;   // T * H'
+  int hp = 1;
+  while (hp * 2 <= hkv && per_unit / (hp * 2) >= vpw) hp *= 2;
+  EncodeGeometry geo;
+  geo.n_tokens = static_cast<uint32_t>(n_tokens);
+  geo.stride = token_stride;
+  geo.unit_tokens = per_unit / hp;
+  geo.unit_heads = hp;
+  geo.head_chunks = (hkv + hp - 1) / hp;
+  const int64_t n_chunks = (n_tokens + geo.unit_tokens - 1) / geo.unit_tokens;
+  geo.n_chunks = static_cast<uint32_t>(n_chunks);
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+  const int64_t grid = n_chunks < sms ? n_chunks : sms;
+  const size_t smem = kQStages * kQStageBytes + 2 * kQStages * sizeof(uint64_t);
+  cudaError_t e = cudaSuccess;
+#define Q4KV_LAUNCH_Q(DD, T)                                                                     \
+  do {                                                                                           \
+    e = cudaFuncSetAttribute(quantize_kernel<DD, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(smem));                                            \
+    if (e == cudaSuccess)                                                                        \
+      e = launch_pdl(quantize_kernel<DD, T>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),  \
+                     smem, stream, pool, static_cast<const T*>(k), static_cast<const T*>(v), geo,  \
+                     block_ids);                                                                 \
+  } while (0)
+  if (n_chunks == 0) return cudaSuccess;
+  if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(128, __half);
+  else if (d == 128) Q4KV_LAUNCH_Q(128, __nv_bfloat16);
+  else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(256, __half);
+  else Q4KV_LAUNCH_Q(256, __nv_bfloat16);
 #undef Q4KV_LAUNCH_Q
+  return e;
 }
 
 cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,

@@ -41,6 +41,32 @@ def test_ragged_tokens_permuted_blocks(d, dtype, hkv, rotated):
     assert_pool_equal(pool, ref)
 
 
+@pytest.mark.parametrize("d,hkv,n", [(128, 5, 1000), (256, 6, 777), (256, 16, 515), (128, 16, 3),
+                                     (256, 3, 1), (128, 2, 261)])
+@pytest.mark.parametrize("strided", [False, True])
+def test_encoder_unit_shapes(d, hkv, n, strided):
+    # head counts that leave a partial head chunk per unit, token tails shorter
+    # than a unit, one-token calls, and rows that are not contiguous in memory
+    k, v = W.random_small(n, hkv, d, "bf16", seed=70 + d + hkv + n)
+    nb = nblocks(n)
+    ids = list(range(nb - 1, -1, -1))
+    dev = cuda()
+    if strided:   # token stride Hkv*D + 8: each token's heads are copied on their own
+        kk = torch.zeros(n, hkv * d + 8, dtype=k.dtype, device=dev)
+        vv = torch.zeros(n, hkv * d + 8, dtype=v.dtype, device=dev)
+        kk[:, :hkv * d] = k.reshape(n, -1).to(dev)
+        vv[:, :hkv * d] = v.reshape(n, -1).to(dev)
+        kk = kk[:, :hkv * d].view(n, hkv, d)
+        vv = vv[:, :hkv * d].view(n, hkv, d)
+    else:
+        kk, vv = k.to(dev), v.to(dev)
+    pool = q4.Q4KVPool(hkv, d, nb, 0, device=dev)
+    pool.quantize(kk, vv, torch.tensor(ids, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    assert pool.read_device_error() == 0
+    assert_pool_equal(pool, oracle_pool(k, v, ids, nb, 0))
+
+
 def test_mixed_widths_and_strided_input():
     n, hkv, d = 700, 4, 128
     k, v = W.random_small(n, hkv, d, "fp16", seed=3)
