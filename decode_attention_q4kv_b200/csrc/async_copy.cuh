@@ -7,7 +7,8 @@
 
 namespace q4kv {
 
-constexpr unsigned kSpinLimit = 1u << 26;   // bounded mbarrier waits (~2 s with back-off)
+constexpr unsigned kSpinLimit = 1u << 21;   // bounded mbarrier waits: ~2 s or more in all
+constexpr unsigned kSuspendNs = 1000;       // hardware suspend hint of one try_wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -25,20 +26,26 @@ __device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+// One try_wait: the thread is suspended (issuing nothing) until the phase
+// completes or the hint runs out; true when the phase has completed.
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
-// Bounded wait; false when the limit ran out.
+// Bounded wait; false when the limit ran out.  The suspend hint is only an
+// upper bound, so between tries the thread also sleeps, backing off from
+// 32 ns to 1 us; the whole wait stays above two seconds before it gives up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  unsigned ns = 32;
   for (unsigned i = 0; i < kSpinLimit; ++i) {
-    if (mbar_test(bar, parity)) return true;
-    if (i > 64) __nanosleep(32);
+    if (mbar_try(bar, parity)) return true;
+    __nanosleep(ns);
+    ns = ns < 1024 ? 2 * ns : 1024;
   }
   return false;
 }

@@ -134,19 +134,27 @@ __device__ __forceinline__ float quot(float u, float s, float r) {
   return __fmaf_rn(__fmaf_rn(-q0, s, u), r, q0);
 }
 
-// Encode the lane's 16 values (one quarter of a 64-value group) and store its
-// codes and, from the group's first lane, the group's (scale, zero).
+// Encoding of one lane's 16 values (a quarter of a 64-value group).
 //
 // Codes are defined as clamp(rne(fl(fl(x - z) / s)), 0, L): u = fl(x - z),
 // then the correctly rounded quotient above, then round-half-even to an
 // integer by adding 1.5 * 2^23.  The quotient is monotone in x, so when the
 // group's extremes give quotients in [-0.5, L + 0.5) no code needs the
-// clamp; other groups (a zero far outside the fp16 grid of the values) take
-// IEEE division and an integer clamp.
+// clamp; other groups (a zero far outside the fp16 grid of the values) are
+// recomputed with IEEE division and an integer clamp.  s = 0 (a constant
+// group) is handled by r = 0, which makes every quotient 0.
+//
+// The steps are split so that the K and V encodings of a warp item form one
+// branch-free stretch of code the compiler can interleave: group statistics,
+// codes, then the rare clamp path and the stores.
+struct GroupParams {
+  __half sh, zh;   // stored scale and zero
+  float s, z, r;   // the same as binary32, and RN(1/s) (0 when s = 0)
+  bool fast;       // every code of the group is rne(quotient) without a clamp
+};
+
 template <int BITS>
-__device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool valid,
-                                             uint8_t* __restrict__ code_dst,
-                                             __half2* __restrict__ param_dst) {
+__device__ __forceinline__ GroupParams group_params(const float2 (&x)[8]) {
   constexpr int L = (1 << BITS) - 1;
   // RN(1/L); 15 and 255 have 11-bit significands
   constexpr float kRecipL = BITS == 4 ? 0x1.111112p-4f : 0x1.010102p-8f;
@@ -163,71 +171,70 @@ __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool v
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
   mx = __fadd_rn(mx, 0.0f);
-  const float s = quot(__fsub_rn(mx, mn), static_cast<float>(L), kRecipL);
-  const __half sh = __float2half_rn(s);
-  const __half zh = __float2half_rn(mn);
-  const float sf = __half2float(sh);
-  const float zf = __half2float(zh);
+  GroupParams g;
+  g.sh = __float2half_rn(quot(__fsub_rn(mx, mn), static_cast<float>(L), kRecipL));
+  g.zh = __float2half_rn(mn);
+  g.s = __half2float(g.sh);
+  g.z = __half2float(g.zh);
+  g.r = g.s != 0.0f ? __frcp_rn(g.s) : 0.0f;
+  const float q_lo = quot(__fsub_rn(mn, g.z), g.s, g.r), q_hi = quot(__fsub_rn(mx, g.z), g.s, g.r);
+  g.fast = q_lo >= -0.5f && q_hi < L + 0.5f;
+  return g;
+}
 
-  // Codes as floats.  4-bit: ke[i] = code of register pair 2i plus 1.5 * 2^23,
-  // ko[i] = code of pair 2i + 1, so ko * 16 + ke holds the byte of channels
-  // (2i, 2i + 1) (.x) and (2i + 8, 2i + 9) (.y) in its low bits.  8-bit:
-  // q[p] = codes of pair p (.x, .y) in the low bits.
-  float2 ke[4], ko[4];
-  uint32_t q[kEPL];
+// Codes as floats.  4-bit: c[i] = code of register pair 2i plus 1.5 * 2^23
+// (i < 4) and c[4 + i] = code of pair 2i + 1, so c[4 + i] * 16 + c[i] holds
+// the byte of channels (2i, 2i + 1) (.x) and (2i + 8, 2i + 9) (.y) in its low
+// bits.  8-bit: c[p] = code of pair p plus 1.5 * 2^23.
+template <int BITS>
+__device__ __forceinline__ void fast_codes(const float2 (&x)[8], const GroupParams& g, float2 (&c)[8]) {
   const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
-  if (sf != 0.0f) {
-    const float r = __frcp_rn(sf);
-    const float q_lo = quot(__fsub_rn(mn, zf), sf, r), q_hi = quot(__fsub_rn(mx, zf), sf, r);
-    if (q_lo >= -0.5f && q_hi < L + 0.5f) {
-      const float2 r2 = make_float2(r, r), ns2 = make_float2(-sf, -sf), nz2 = make_float2(-zf, -zf);
-      const float2 mm2 = make_float2(-kRoundMagic, -kRoundMagic);
+  const float2 mm2 = make_float2(-kRoundMagic, -kRoundMagic);
+  const float2 r2 = make_float2(g.r, g.r), ns2 = make_float2(-g.s, -g.s), nz2 = make_float2(-g.z, -g.z);
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const float2 u = __fadd2_rn(x[p], nz2);            // fl(x - z)
-        const float2 q0 = __fmul2_rn(u, r2);
-        const float2 q1 = __ffma2_rn(__ffma2_rn(q0, ns2, u), r2, q0);   // fl(u / s)
-        const float2 yk = __fadd2_rn(q1, m2);              // rne(q1) in the low bits
-        if (BITS == 4) {
-          if (p % 2 == 0) ke[p / 2] = yk;
-          else ko[p / 2] = __fadd2_rn(yk, mm2);
-        } else {
-          q[p] = __float_as_uint(yk.x);
-          q[p + 8] = __float_as_uint(yk.y);
-        }
-      }
+  for (int p = 0; p < 8; ++p) {
+    const float2 u = __fadd2_rn(x[p], nz2);                              // fl(x - z)
+    const float2 q0 = __fmul2_rn(u, r2);
+    const float2 q1 = __ffma2_rn(__ffma2_rn(q0, ns2, u), r2, q0);        // fl(u / s)
+    const float2 yk = __fadd2_rn(q1, m2);                                // rne(q1) in the low bits
+    if (BITS == 4) {
+      if (p % 2 == 0) c[p / 2] = yk;
+      else c[4 + p / 2] = __fadd2_rn(yk, mm2);
     } else {
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const int r0 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].x, zf), sf)), 0), L);
-        const int r1 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].y, zf), sf)), 0), L);
-        if (BITS == 4) {
-          const float2 c = make_float2(static_cast<float>(r0), static_cast<float>(r1));
-          if (p % 2 == 0) ke[p / 2] = __fadd2_rn(c, m2);
-          else ko[p / 2] = c;
-        } else {
-          q[p] = static_cast<uint32_t>(r0);
-          q[p + 8] = static_cast<uint32_t>(r1);
-        }
-      }
+      c[p] = yk;
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ke[i] = m2;
-      ko[i] = make_float2(0.0f, 0.0f);
-    }
-#pragma unroll
-    for (int e = 0; e < kEPL; ++e) q[e] = 0;
   }
-  if (!valid) return;
+}
+
+template <int BITS>
+__device__ __forceinline__ void clamped_codes(const float2 (&x)[8], const GroupParams& g, float2 (&c)[8]) {
+  constexpr int L = (1 << BITS) - 1;
+  const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int r0 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].x, g.z), g.s)), 0), L);
+    const int r1 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].y, g.z), g.s)), 0), L);
+    const float2 k = make_float2(static_cast<float>(r0), static_cast<float>(r1));
+    if (BITS == 4) {
+      if (p % 2 == 0) c[p / 2] = __fadd2_rn(k, m2);
+      else c[4 + p / 2] = k;
+    } else {
+      c[p] = __fadd2_rn(k, m2);
+    }
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupParams& g, int j,
+                                            uint8_t* __restrict__ code_dst,
+                                            __half2* __restrict__ param_dst) {
   if (BITS == 4) {
     // byte b holds elements 2b (low nibble) and 2b+1 (high nibble); the sums
     // are exact (integers below 2^24)
     uint32_t b[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float2 w = __ffma2_rn(ko[i], make_float2(16.0f, 16.0f), ke[i]);
+      const float2 w = __ffma2_rn(c[4 + i], make_float2(16.0f, 16.0f), c[i]);
       b[i] = __float_as_uint(w.x);
       b[i + 4] = __float_as_uint(w.y);
     }
@@ -235,6 +242,13 @@ __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool v
     const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
     *reinterpret_cast<uint2*>(code_dst + j * 8) = make_uint2(lo, hi);
   } else {
+    // element e: pair e % 8, half e / 8
+    uint32_t q[kEPL];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      q[p] = __float_as_uint(c[p].x);
+      q[p + 8] = __float_as_uint(c[p].y);
+    }
     uint4 w;
     w.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
     w.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
@@ -242,7 +256,25 @@ __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool v
     w.w = __byte_perm(__byte_perm(q[12], q[13], 0x0040), __byte_perm(q[14], q[15], 0x0040), 0x5410);
     *reinterpret_cast<uint4*>(code_dst + j * 16) = w;
   }
-  if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(sh, zh);
+  if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(g.sh, g.zh);
+}
+
+// K (already rotated when the pool stores rotated keys) and V of one warp item.
+template <int BITS>
+__device__ __forceinline__ void encode_kv(const float2 (&xk)[8], const float2 (&xv)[8], int j, bool valid,
+                                          uint8_t* __restrict__ kc, __half2* __restrict__ kp,
+                                          uint8_t* __restrict__ vc, __half2* __restrict__ vp) {
+  const GroupParams gk = group_params<BITS>(xk);
+  const GroupParams gv = group_params<BITS>(xv);
+  float2 ck[8], cv[8];
+  fast_codes<BITS>(xk, gk, ck);
+  fast_codes<BITS>(xv, gv, cv);
+  if (!gk.fast) clamped_codes<BITS>(xk, gk, ck);
+  if (!gv.fast) clamped_codes<BITS>(xv, gv, cv);
+  if (valid) {
+    store_codes<BITS>(ck, gk, j, kc, kp);
+    store_codes<BITS>(cv, gv, j, vc, vp);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -250,15 +282,17 @@ __device__ __forceinline__ void encode_store(const float2 (&x)[8], int j, bool v
 // the K and V rows of a unit -- T consecutive tokens x a run of H' heads,
 // 16 KB of input per tensor -- into a 4-deep ring of shared-memory stages
 // with bulk copies (one copy per token row, or one per tensor when the run
-// is contiguous in memory); 16 consumer warps each encode one warp item of
-// the stage: VPW tokens of one head, a lane holding 16 channels.  T and H'
+// is contiguous in memory); 23 consumer warps encode its warp items: VPW
+// tokens of one head, a lane holding 16 channels.  T and H'
 // are chosen so that every full unit holds exactly 16 warp items.
 // ---------------------------------------------------------------------------
-constexpr int kQConsumers = 16;
+constexpr int kQConsumers = 23;                 // consumer warps (6 warps per scheduler)
+constexpr int kQItems = 16;                     // warp items in a full unit
 constexpr int kQThreads = (kQConsumers + 1) * 32;
 constexpr int kQStages = 4;
 constexpr int kQHalf = 16384;                 // input bytes of one tensor per stage
 constexpr int kQStageBytes = 2 * kQHalf;
+static_assert((kQStages & (kQStages - 1)) == 0, "stage index is a mask");
 
 struct EncodeGeometry {
   uint32_t n_tokens;
@@ -267,9 +301,10 @@ struct EncodeGeometry {
   int32_t unit_heads;    // H'
   int32_t head_chunks;   // ceil(Hkv / H')
   uint32_t n_chunks;     // ceil(n_tokens / T)
+  int32_t items_per_head_log2;   // log2(T / VPW)
 };
 
-template <int D, typename InT>
+template <int D, typename InT, bool ROT>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_kernel(const __grid_constant__ PoolView pool, const InT* __restrict__ k,
                     const InT* __restrict__ v, const __grid_constant__ EncodeGeometry geo,
@@ -289,7 +324,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kQConsumers);
+      mbar_init(&empty[i], kQItems);
     }
     s_timeout = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -336,71 +371,84 @@ __global__ void __launch_bounds__(kQThreads, 1)
   }
 
   // ---------------- consumers ----------------
-  // warp w takes warp item w of each unit: head hh = w / tpi of the unit's
-  // run, tokens (w % tpi) * VPW .. + VPW - 1 of its T
+  // The CTA's units come in the producer's order; their warp items (16 per
+  // unit, item w = head w / tpi of the unit's run, tokens (w % tpi) * VPW ..
+  // + VPW - 1 of its T) form one stream that warp w walks with stride 23.
+  // A stage is released after its 16 items have arrived.  The position
+  // (chunk c, head chunk hc, unit ul, item w16) advances without division.
   const int r = lane / S::LPV;       // token of the warp item
   const int j = lane % S::LPV;       // 16-channel run of the lane
-  const int tpi = T / S::VPW;        // warp items per head in a unit
-  const int hh = warp / tpi;
-  const int ti = (warp - hh * tpi) * S::VPW;   // first token of the item in the unit
-  const int tt = ti + r;
-  uint32_t it = 0;
-  bool dead = false;
-  int32_t blk_next = blockIdx.x < geo.n_chunks ? __ldg(block_ids + (blockIdx.x * T) / kBlockTokens) : 0;
-  for (uint32_t c = blockIdx.x; c < geo.n_chunks && !dead; c += gridDim.x) {
-    const uint32_t t0 = c * T;
-    const int32_t blk = blk_next;
-    if (c + gridDim.x < geo.n_chunks) blk_next = __ldg(block_ids + ((c + gridDim.x) * T) / kBlockTokens);
-    const uint32_t t = t0 + tt;
-    const bool valid = t < geo.n_tokens;
-    const int slot = static_cast<int>(t % kBlockTokens);
-    const bool bad_blk = blk < 0 || blk >= pool.n_q4 + pool.n_q8;
-    const bool is8 = blk >= pool.n_q4;
-    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
-    for (int hc = 0; hc < HC; ++hc, ++it) {
-      const int s = it % kQStages;
-      if (!mbar_wait(&full[s], (it / kQStages) & 1) || s_timeout) {
-        if (lane == 0 && warp == 0) raise_error(pool.error_word, Q4KV_DEVERR_TIMEOUT);
-        dead = true;
-        break;
+  const int tpi_log = geo.items_per_head_log2;   // tpi = T / VPW, a power of two
+  struct Pos {
+    uint32_t c, ul;
+    int hc, w16;
+  };
+  auto advance = [&](Pos& p, int by) {
+    p.w16 += by;
+    while (p.w16 >= kQItems) {
+      p.w16 -= kQItems;
+      ++p.ul;
+      if (++p.hc == HC) {
+        p.hc = 0;
+        p.c += gridDim.x;
       }
-      const int h0 = hc * HP, nh = min(HP, hkv - h0);
-      if (hh < nh) {
-        const uint8_t* src = stages + s * kQStageBytes + ((tt * nh + hh) * D + j * kEPL) * sizeof(InT);
-        const uint4 k0 = lds16(src), k1 = lds16(src + 16);
-        const uint4 v0 = lds16(src + kQHalf), v1 = lds16(src + kQHalf + 16);
-        const int h = h0 + hh;
-        if (bad_blk) {
-          if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
-        } else {
-          const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
-          float2 x[8];
-          // keys: rotate, then code
-          unpack16<InT>(k0, k1, x);
-          if (pool.k_rotated) rotate_pairs<D>(x, j);
-          if (is8)
-            encode_store<8>(x, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG);
-          else
-            encode_store<4>(x, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG);
-          // values: code unrotated
-          unpack16<InT>(v0, v1, x);
-          if (is8)
-            encode_store<8>(x, j, valid, pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
-          else
-            encode_store<4>(x, j, valid, pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
-          // freshly written slots are live: one word update for the item's tokens
-          const uint32_t tf = t0 + ti;
-          if (h == 0 && lane == 0 && tf < geo.n_tokens) {
-            const int nv = static_cast<int>(umin(static_cast<uint32_t>(S::VPW), geo.n_tokens - tf));
-            const int sf = static_cast<int>(tf % kBlockTokens);
-            atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + sf / 32,
-                      ~(((1u << nv) - 1u) << (sf % 32)));
-          }
+    }
+  };
+  Pos pos = {blockIdx.x, 0u, 0, 0};
+  advance(pos, warp);
+  int32_t blk = pos.c < geo.n_chunks ? __ldg(block_ids + (pos.c * T) / kBlockTokens) : 0;
+  while (pos.c < geo.n_chunks) {
+    Pos nxt = pos;
+    advance(nxt, kQConsumers);
+    const int32_t blk_next = nxt.c < geo.n_chunks ? __ldg(block_ids + (nxt.c * T) / kBlockTokens) : 0;
+    const int s = pos.ul & (kQStages - 1);
+    if (!mbar_wait(&full[s], (pos.ul / kQStages) & 1) || s_timeout) {
+      if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_TIMEOUT);
+      break;
+    }
+    const uint32_t t0 = pos.c * T;
+    const int h0 = pos.hc * HP, nh = min(HP, hkv - h0);
+    const int hh = pos.w16 >> tpi_log;
+    const int ti = (pos.w16 & ((1 << tpi_log) - 1)) * S::VPW;   // first token of the item in the unit
+    const int tt = ti + r;
+    if (hh < nh) {
+      const uint32_t t = t0 + tt;
+      const bool valid = t < geo.n_tokens;
+      const uint8_t* src = stages + s * kQStageBytes + ((tt * nh + hh) * D + j * kEPL) * sizeof(InT);
+      const uint4 k0 = lds16(src), k1 = lds16(src + 16);
+      const uint4 v0 = lds16(src + kQHalf), v1 = lds16(src + kQHalf + 16);
+      const int h = h0 + hh;
+      if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+        if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
+      } else {
+        const int slot = static_cast<int>(t % kBlockTokens);
+        const bool is8 = blk >= pool.n_q4;
+        const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+        const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
+        float2 xk[8], xv[8];
+        unpack16<InT>(k0, k1, xk);
+        unpack16<InT>(v0, v1, xv);
+        if (ROT) rotate_pairs<D>(xk, j);   // keys are coded rotated, values as they are
+        if (is8)
+          encode_kv<8>(xk, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
+                       pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+        else
+          encode_kv<4>(xk, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
+                       pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+        // freshly written slots are live: one word update for the item's tokens
+        const uint32_t tf = t0 + ti;
+        if (h == 0 && lane == 0 && tf < geo.n_tokens) {
+          const int nv = static_cast<int>(umin(static_cast<uint32_t>(S::VPW), geo.n_tokens - tf));
+          const int sf = static_cast<int>(tf % kBlockTokens);
+          atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + sf / 32,
+                    ~(((1u << nv) - 1u) << (sf % 32)));
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    pos = nxt;
+    blk = blk_next;
   }
 }
 
@@ -581,26 +629,36 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
   geo.unit_tokens = per_unit / hp;
   geo.unit_heads = hp;
   geo.head_chunks = (hkv + hp - 1) / hp;
+  geo.items_per_head_log2 = 0;
+  while ((vpw << (geo.items_per_head_log2 + 1)) <= geo.unit_tokens) ++geo.items_per_head_log2;
   const int64_t n_chunks = (n_tokens + geo.unit_tokens - 1) / geo.unit_tokens;
   geo.n_chunks = static_cast<uint32_t>(n_chunks);
   const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
   const int64_t grid = n_chunks < sms ? n_chunks : sms;
   const size_t smem = kQStages * kQStageBytes + 2 * kQStages * sizeof(uint64_t);
   cudaError_t e = cudaSuccess;
-#define Q4KV_LAUNCH_Q(DD, T)                                                                     \
-  do {                                                                                           \
-    e = cudaFuncSetAttribute(quantize_kernel<DD, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             static_cast<int>(smem));                                            \
-    if (e == cudaSuccess)                                                                        \
-      e = launch_pdl(quantize_kernel<DD, T>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),  \
-                     smem, stream, pool, static_cast<const T*>(k), static_cast<const T*>(v), geo,  \
-                     block_ids);                                                                 \
+#define Q4KV_LAUNCH_Q(DD, T, R)                                                                   \
+  do {                                                                                              \
+    e = cudaFuncSetAttribute(quantize_kernel<DD, T, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(smem));                                               \
+    if (e == cudaSuccess)                                                                           \
+      e = launch_pdl(quantize_kernel<DD, T, R>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),  \
+                     smem, stream, pool, static_cast<const T*>(k), static_cast<const T*>(v), geo,     \
+                     block_ids);                                                                    \
+  } while (0)
+#define Q4KV_LAUNCH_QR(DD, T)       \
+  do {                              \
+    if (pool.k_rotated)             \
+      Q4KV_LAUNCH_Q(DD, T, true);   \
+    else                            \
+      Q4KV_LAUNCH_Q(DD, T, false);  \
   } while (0)
   if (n_chunks == 0) return cudaSuccess;
-  if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(128, __half);
-  else if (d == 128) Q4KV_LAUNCH_Q(128, __nv_bfloat16);
-  else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(256, __half);
-  else Q4KV_LAUNCH_Q(256, __nv_bfloat16);
+  if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_QR(128, __half);
+  else if (d == 128) Q4KV_LAUNCH_QR(128, __nv_bfloat16);
+  else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_QR(256, __half);
+  else Q4KV_LAUNCH_QR(256, __nv_bfloat16);
+#undef Q4KV_LAUNCH_QR
 #undef Q4KV_LAUNCH_Q
   return e;
 }
