@@ -10,22 +10,24 @@
 // Why tensor cores: per (token, KV head) the g query heads of a GQA group do
 // g*D multiply-adds against the keys and g*D against the values, over 144
 // bytes of packed data (D = 128).  At HBM speed that is more fp32 FMA issue
-// than the SM has, so both contractions run as mma.sync.m16n8k16 (fp16 in,
-// fp32 accumulate) with the codes (exact small integers in fp16) as one
-// operand.  tcgen05 would need the unpacked codes in shared memory or TMEM
-// (4x the packed bytes of shared-memory traffic, N <= 16 columns), so the
-// register-fed mma.sync is the better fit for this N.
+// than the SM has, so both contractions run on the tensor cores with the
+// codes as one operand, unpacked in registers.  tcgen05 would need the
+// unpacked codes in shared memory or TMEM (2-4x the packed bytes of
+// shared-memory traffic, N <= 16 columns), so the register-fed mma.sync is
+// the better fit for this N.
 //
-//   keys:   S^T[16 tokens][8 cols] += Kcodes[16 tokens][16 ch] x Qm[16 ch][8 cols]
+//   keys:   S^T[16 tokens][8 cols] += Kcodes[16 tokens][32 ch] x Qm[32 ch][8 cols]
+//           (mma.sync.m16n8k32, u8 codes x s8 query digits, exact int32).
 //           A column of Qm is one (query head h, group gr) pair: q_rot[h] on
 //           the 64 channels of group gr and 0 elsewhere, so each thread gets
 //           the per-group partial dots and applies that token's (s, z) in
 //           registers: logit = sum_gr s_gr S_gr + z_gr sum(q_rot over gr).
-//           q_rot is split into fp16 hi + lo parts (two MMAs), so it is
-//           carried to ~22 bits.
+//           q_rot is scaled to 16-bit fixed point and split into two int8
+//           digits (two MMAs), exact up to the rounding of the scaled query.
 //   values: O^T[16 ch][8 cols] += Vcodes^T[16 ch][16 tokens] x W[16 tokens][8 cols]
-//           with W[t][(h, gr)] = p_t,h * s_t,gr (the value scale folded into
-//           the weight) and the zero term sum_t p_t,h z_t,gr added at the end;
+//           (mma.sync.m16n8k16, fp16 in, fp32 accumulate) with
+//           W[t][(h, gr)] = p_t,h * s_t,gr (the value scale folded into the
+//           weight) and the zero term sum_t p_t,h z_t,gr added at the end;
 //           a channel keeps only the column of its own group.  The softmax
 //           weights come out of the key MMA in the accumulator layout; one
 //           movmatrix.trans per 8x8 turns them into the B operand.
@@ -124,17 +126,21 @@ __device__ __forceinline__ uint32_t lop_or(uint32_t x, uint32_t mask, uint32_t b
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// 0x6400 is fp16 1024: (nibble | 0x6400) = 1024 + nibble, (nibble << 4 | 0x6400) = 1024 + 16 nibble.
-__device__ __forceinline__ uint32_t lo_nib(uint32_t x) {   // nibbles at bits 0-3, 16-19 -> exact codes
-  return h2u(__hsub2(u2h(lop_or(x, 0x000F000Fu, 0x64006400u)), u2h(0x64006400u)));
+// Value codes enter the fp16 MMA as exact fp16 numbers with no offset: a
+// nibble or byte c masked into the low mantissa bits of a zero-exponent fp16
+// is the subnormal c * 2^-24.  Rows of the value MMA for even channels carry
+// c * 2^-24, rows for odd channels c * 2^-20 (a 4-bit high nibble masked in
+// place is 16 c * 2^-24); each output channel therefore has one power-of-two
+// scale, undone exactly in the epilogue.
+__device__ __forceinline__ uint32_t lo_nib(uint32_t x) { return x & 0x000F000Fu; }   // c * 2^-24
+__device__ __forceinline__ uint32_t hi_nib(uint32_t x) { return x & 0x00F000F0u; }   // c * 2^-20
+__device__ __forceinline__ uint32_t byte_lo(uint32_t x) { return x & 0x00FF00FFu; }  // c * 2^-24
+__device__ __forceinline__ uint32_t byte_hi(uint32_t x) {   // c * 2^-20 = (1024 + c) 2^-20 - 2^-10, exact
+  return h2u(__hfma2(u2h((x & 0x00FF00FFu) | 0x64006400u), u2h(0x00100010u) /*2^-20*/,
+                     u2h(0x94009400u) /*-2^-10*/));
 }
-__device__ __forceinline__ uint32_t hi_nib(uint32_t x) {   // nibbles at bits 4-7, 20-23 -> exact codes
-  return h2u(__hfma2(u2h(lop_or(x, 0x00F000F0u, 0x64006400u)), u2h(0x2C002C00u) /*1/16*/,
-                     u2h(0xD400D400u) /*-64*/));
-}
-__device__ __forceinline__ uint32_t byte_pair(uint32_t x) {  // bytes at 0, 2 -> exact codes
-  return h2u(__hsub2(u2h(lop_or(x, 0x00FF00FFu, 0x64006400u)), u2h(0x64006400u)));
-}
+constexpr float kEvenScale = 16777216.0f;   // 2^24
+constexpr float kOddScale = 1048576.0f;     // 2^20
 
 template <typename T>
 __device__ __forceinline__ T lds(const void* p) { return *reinterpret_cast<const T*>(p); }
@@ -200,9 +206,9 @@ __device__ __forceinline__ int tok_perm(int r) { return r ^ ((r >> 1) & 1); }
 // Value A operands for one 16-token tile: tokens T = pi(2t), pi(2t+1),
 // pi(2t+8), pi(2t+9) of the tile, thread g's channels cb + [0, D/8).  Tile mv
 // (channels) uses rows g -> cb + 2 mv and g + 8 -> cb + 2 mv + 1.  The codes
-// enter the MMA as exact small integers: an offset form (1024 + code) would
-// save one instruction per register, but the accumulator would then carry
-// ~1024 x the weight sum and lose accuracy over long contexts.
+// enter the MMA as exact fp16 subnormals (see lo_nib); an offset form
+// (1024 + code) would make the accumulator carry ~1024 x the weight sum and
+// lose accuracy over long contexts.
 template <int D, bool Q8>
 __device__ __forceinline__ void value_a(const uint32_t* v0, const uint32_t* v1, const uint32_t* v8,
                                         const uint32_t* v9, int mv, uint32_t (&a)[4]) {
@@ -216,10 +222,10 @@ __device__ __forceinline__ void value_a(const uint32_t* v0, const uint32_t* v1, 
   } else {
     const int wi = (2 * mv) / 4, bp = (2 * mv) % 4;
     const uint32_t sa = bp | ((bp + 4) << 8), sb = (bp + 1) | ((bp + 5) << 8);
-    a[0] = byte_pair(__byte_perm(v0[wi], v1[wi], sa));
-    a[1] = byte_pair(__byte_perm(v0[wi], v1[wi], sb));
-    a[2] = byte_pair(__byte_perm(v8[wi], v9[wi], sa));
-    a[3] = byte_pair(__byte_perm(v8[wi], v9[wi], sb));
+    a[0] = byte_lo(__byte_perm(v0[wi], v1[wi], sa));
+    a[1] = byte_hi(__byte_perm(v0[wi], v1[wi], sb));
+    a[2] = byte_lo(__byte_perm(v8[wi], v9[wi], sa));
+    a[3] = byte_hi(__byte_perm(v8[wi], v9[wi], sb));
   }
 }
 
@@ -453,6 +459,22 @@ __device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage
   }
 }
 
+// Raw 16-bit query elements E*lane .. E*lane + E-1 of head `h` of item's
+// (sequence, KV head) group, as loaded (E = 4: 8 bytes, E = 8: 16 bytes).
+template <int E>
+__device__ __forceinline__ uint4 load_query(const DecodeArgs& a, int item, int S, int hkv, int hq, int G,
+                                            int h, int lane) {
+  const int kvh = (item / S) % hkv;
+  const int b = item / (S * hkv);
+  const int64_t qi = (static_cast<int64_t>(b) * hq + kvh * G + h) * (E * 32) + E * lane;
+  const uint8_t* p = static_cast<const uint8_t*>(a.q) + 2 * qi;
+  if (E == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    return make_uint4(w.x, w.y, 0u, 0u);
+  }
+  return *reinterpret_cast<const uint4*>(p);
+}
+
 template <int D, int NT>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     decode_tc_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ TileMaps maps,
@@ -579,6 +601,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   TileOffsets<D, false> off4;
   off4.init(warp, lane);
 
+  uint4 qraw = make_uint4(0u, 0u, 0u, 0u);   // raw query of the warp's head for the coming item
+  if (warp < G && blockIdx.x < n_items) qraw = load_query<D / 32>(a, blockIdx.x, S, hkv, hq, G, warp, lane);
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int split = item % S;
     const int kvh = (item / S) % hkv;
@@ -588,25 +612,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if (warp < G) {
       constexpr int E = D / 32;                   // lane holds channels E*lane .. E*lane + E-1
       float x[E];
-      const int64_t qi = ((static_cast<int64_t>(b) * hq + kvh * G + warp) * D + E * lane);
-      if (E == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(a.q) + 2 * qi);
-        const uint32_t ww[2] = {w.x, w.y};
+      const uint4 w = qraw;
+      // the next item's query is loaded now, behind this item's stages
+      const int nitem = item + gridDim.x;
+      if (nitem < n_items) qraw = load_query<E>(a, nitem, S, hkv, hq, G, warp, lane);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t h16 = (ww[e / 2] >> (16 * (e % 2))) & 0xFFFFu;
-          x[e] = a.q_dtype == Q4KV_F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(h16)))
-                                       : __uint_as_float(h16 << 16);
-        }
-      } else {
-        const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.q) + 2 * qi);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const uint32_t h16 = (ww[e / 2] >> (16 * (e % 2))) & 0xFFFFu;
-          x[e] = a.q_dtype == Q4KV_F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(h16)))
-                                       : __uint_as_float(h16 << 16);
-        }
+      for (int e = 0; e < E; ++e) {
+        const uint32_t h16 = (ww[e / 2] >> (16 * (e % 2))) & 0xFFFFu;
+        x[e] = a.q_dtype == Q4KV_F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(h16)))
+                                     : __uint_as_float(h16 << 16);
       }
       if (P.k_rotated) {   // c * H q: butterflies inside the lane, then across lanes (fp32)
 #pragma unroll
@@ -763,7 +778,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           const int col = c0 + (e & 1);
           const int hh = col / NG, gr = col % NG;
           if (hh < G && gr == ch / kGroup)
-            mrg_o[(warp * G + hh) * D + ch] = st.o[mv][j][e] + zz[e & 1];
+            mrg_o[(warp * G + hh) * D + ch] = __fmaf_rn(st.o[mv][j][e], e < 2 ? kEvenScale : kOddScale, zz[e & 1]);
         }
       }
     }
