@@ -85,12 +85,20 @@ __device__ __forceinline__ void fwht_pairs(float2 (&x)[8], int j) {
   }
 }
 
+// c * H x.  At D = 256 the constant c = 2^-4 is exact, so the multiply is
+// left to the encoder (kRotScale), which folds it into its first operations
+// without changing any rounding; at D = 128 it is applied here.
+template <int D>
+constexpr float kRotScale = D == 256 ? 0.0625f : 1.0f;
+
 template <int D>
 __device__ __forceinline__ void rotate_pairs(float2 (&x)[8], int j) {
   fwht_pairs<D>(x, j);
-  const float c = rotation_constant(D);
+  if (D != 256) {
+    const float c = rotation_constant(D);
 #pragma unroll
-  for (int p = 0; p < 8; ++p) x[p] = __fmul2_rn(x[p], make_float2(c, c));
+    for (int p = 0; p < 8; ++p) x[p] = __fmul2_rn(x[p], make_float2(c, c));
+  }
 }
 
 __device__ __forceinline__ uint4 lds16(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
@@ -153,8 +161,10 @@ struct GroupParams {
   bool fast;       // every code of the group is rne(quotient) without a clamp
 };
 
+// x holds the values divided by xs (a power of two): every use multiplies
+// by xs first, which is exact.
 template <int BITS>
-__device__ __forceinline__ GroupParams group_params(const float2 (&x)[8]) {
+__device__ __forceinline__ GroupParams group_params(const float2 (&x)[8], float xs) {
   constexpr int L = (1 << BITS) - 1;
   // RN(1/L); 15 and 255 have 11-bit significands
   constexpr float kRecipL = BITS == 4 ? 0x1.111112p-4f : 0x1.010102p-8f;
@@ -169,8 +179,8 @@ __device__ __forceinline__ GroupParams group_params(const float2 (&x)[8]) {
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
-  mx = __fadd_rn(mx, 0.0f);
+  mn = __fadd_rn(__fmul_rn(mn, xs), 0.0f);  // exact scaling; -0 -> +0
+  mx = __fadd_rn(__fmul_rn(mx, xs), 0.0f);
   GroupParams g;
   g.sh = __float2half_rn(quot(__fsub_rn(mx, mn), static_cast<float>(L), kRecipL));
   g.zh = __float2half_rn(mn);
@@ -187,13 +197,14 @@ __device__ __forceinline__ GroupParams group_params(const float2 (&x)[8]) {
 // the byte of channels (2i, 2i + 1) (.x) and (2i + 8, 2i + 9) (.y) in its low
 // bits.  8-bit: c[p] = code of pair p plus 1.5 * 2^23.
 template <int BITS>
-__device__ __forceinline__ void fast_codes(const float2 (&x)[8], const GroupParams& g, float2 (&c)[8]) {
+__device__ __forceinline__ void fast_codes(const float2 (&x)[8], float xs, const GroupParams& g, float2 (&c)[8]) {
   const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
   const float2 mm2 = make_float2(-kRoundMagic, -kRoundMagic);
   const float2 r2 = make_float2(g.r, g.r), ns2 = make_float2(-g.s, -g.s), nz2 = make_float2(-g.z, -g.z);
+  const float2 xs2 = make_float2(xs, xs);
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    const float2 u = __fadd2_rn(x[p], nz2);                              // fl(x - z)
+    const float2 u = __ffma2_rn(x[p], xs2, nz2);                         // fl(x xs - z), x xs exact
     const float2 q0 = __fmul2_rn(u, r2);
     const float2 q1 = __ffma2_rn(__ffma2_rn(q0, ns2, u), r2, q0);        // fl(u / s)
     const float2 yk = __fadd2_rn(q1, m2);                                // rne(q1) in the low bits
@@ -207,13 +218,13 @@ __device__ __forceinline__ void fast_codes(const float2 (&x)[8], const GroupPara
 }
 
 template <int BITS>
-__device__ __forceinline__ void clamped_codes(const float2 (&x)[8], const GroupParams& g, float2 (&c)[8]) {
+__device__ __forceinline__ void clamped_codes(const float2 (&x)[8], float xs, const GroupParams& g, float2 (&c)[8]) {
   constexpr int L = (1 << BITS) - 1;
   const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    const int r0 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].x, g.z), g.s)), 0), L);
-    const int r1 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(x[p].y, g.z), g.s)), 0), L);
+    const int r0 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(__fmul_rn(x[p].x, xs), g.z), g.s)), 0), L);
+    const int r1 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(__fmul_rn(x[p].y, xs), g.z), g.s)), 0), L);
     const float2 k = make_float2(static_cast<float>(r0), static_cast<float>(r1));
     if (BITS == 4) {
       if (p % 2 == 0) c[p / 2] = __fadd2_rn(k, m2);
@@ -259,18 +270,19 @@ __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupPar
   if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(g.sh, g.zh);
 }
 
-// K (already rotated when the pool stores rotated keys) and V of one warp item.
+// K (already rotated when the pool stores rotated keys; its values are the
+// rotated ones divided by ks) and V of one warp item.
 template <int BITS>
-__device__ __forceinline__ void encode_kv(const float2 (&xk)[8], const float2 (&xv)[8], int j, bool valid,
-                                          uint8_t* __restrict__ kc, __half2* __restrict__ kp,
+__device__ __forceinline__ void encode_kv(const float2 (&xk)[8], float ks, const float2 (&xv)[8], int j,
+                                          bool valid, uint8_t* __restrict__ kc, __half2* __restrict__ kp,
                                           uint8_t* __restrict__ vc, __half2* __restrict__ vp) {
-  const GroupParams gk = group_params<BITS>(xk);
-  const GroupParams gv = group_params<BITS>(xv);
+  const GroupParams gk = group_params<BITS>(xk, ks);
+  const GroupParams gv = group_params<BITS>(xv, 1.0f);
   float2 ck[8], cv[8];
-  fast_codes<BITS>(xk, gk, ck);
-  fast_codes<BITS>(xv, gv, cv);
-  if (!gk.fast) clamped_codes<BITS>(xk, gk, ck);
-  if (!gv.fast) clamped_codes<BITS>(xv, gv, cv);
+  fast_codes<BITS>(xk, ks, gk, ck);
+  fast_codes<BITS>(xv, 1.0f, gv, cv);
+  if (!gk.fast) clamped_codes<BITS>(xk, ks, gk, ck);
+  if (!gv.fast) clamped_codes<BITS>(xv, 1.0f, gv, cv);
   if (valid) {
     store_codes<BITS>(ck, gk, j, kc, kp);
     store_codes<BITS>(cv, gv, j, vc, vp);
@@ -429,11 +441,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
         unpack16<InT>(k0, k1, xk);
         unpack16<InT>(v0, v1, xv);
         if (ROT) rotate_pairs<D>(xk, j);   // keys are coded rotated, values as they are
+        constexpr float ks = ROT ? kRotScale<D> : 1.0f;
         if (is8)
-          encode_kv<8>(xk, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
+          encode_kv<8>(xk, ks, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
                        pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
         else
-          encode_kv<4>(xk, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
+          encode_kv<4>(xk, ks, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
                        pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
         // freshly written slots are live: one word update for the item's tokens
         const uint32_t tf = t0 + ti;
