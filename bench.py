@@ -142,7 +142,7 @@ class Job:
         import decode_attention_q4kv_b200 as q4
         from decode_attention_q4kv_b200 import workloads as W
 
-        self.w, self.dev, self.torch, self.q4 = w, device, torch, q4
+        self.w, self.dev, self.torch, self.q4, self.W = w, device, torch, q4, W
         if isinstance(layers, (list, tuple)):
             layer_ids = list(layers)
         else:
@@ -223,6 +223,20 @@ class Job:
     def decode_layer(self, L):
         self.q4.decode_attention(L["pool"], L["q"], L.get("tables", self.tables), self.lens,
                                  plan=self.plan, workspace=self.ws, out=L["out"])
+
+    def append_setup(self):
+        """One new token per sequence (seeded), written over each sequence's last slot."""
+        torch, W, w = self.torch, self.W, self.w
+        kn, vn = W.random_small(w.batch, w.n_kv_heads, w.head_dim, w.dtype, seed=w.seed + 77)
+        self.k_new = kn.view(w.batch, 1, w.n_kv_heads, w.head_dim).to(self.dev)
+        self.v_new = vn.view(w.batch, 1, w.n_kv_heads, w.head_dim).to(self.dev)
+        self.lens_before = (self.lens - 1).contiguous()
+        # algorithmic bytes of one append: K/V rows read, codes and params written
+        vec = 2 * w.head_dim * 2 + 2 * (w.head_dim // 2 + 4 * (w.head_dim // 64))
+        self.append_bytes = w.batch * w.n_kv_heads * vec
+
+    def append_layer(self, L):
+        L["pool"].append(self.k_new, self.v_new, L.get("tables", self.tables), self.lens_before)
 
     def step(self, events=None):
         for L in self.layers:
@@ -355,6 +369,22 @@ def run_gpu(args):
     torch.cuda.synchronize()
     d_cold_ms = statistics.median(a.elapsed_time(b) for a, b in cold)
 
+    # generation step: append one new token per sequence (over its last slot), then decode
+    job.append_setup()
+    gen = []
+    for _ in range(reps):
+        for L in job.layers:
+            a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a.record()
+            job.append_layer(L)
+            b.record()
+            job.decode_layer(L)
+            c.record()
+            gen.append((a, b, c))
+    torch.cuda.synchronize()
+    app_ms = statistics.median(a.elapsed_time(b) for a, b, _ in gen)
+    gen_ms = statistics.median(a.elapsed_time(c) for a, _, c in gen)
+
     e2e = run_e2e(job, args, dev, world) if not args.no_e2e else None
     if world > 1:
         dist.barrier()
@@ -399,6 +429,10 @@ def run_gpu(args):
                            "bytes_per_launch": job.decode_bytes,
                            "kv_tokens_per_s": round(kv_tok / (d_cold_ms * 1e-3), 1),
                            "frac_cold": round(d_cold_gbps / peak, 4)},
+                "append": {"us_per_launch": round(app_ms * 1e3, 2), "tokens_per_launch": w.batch,
+                           "bytes_per_launch": job.append_bytes,
+                           "append_then_decode_us": round(gen_ms * 1e3, 2),
+                           "note": "one new token per sequence written over its last slot, then decode"},
             },
             "roofline": roof,
             "gpu_launches": job.launches_per_layer * job.n_layers * args.steps,

@@ -126,6 +126,37 @@ class Q4KVPool:
                                          k.shape[0], k.stride(0), _ptr(ids), _stream(dev)),
               "q4kv_quantize_blocks")
 
+    def append(self, k: torch.Tensor, v: torch.Tensor, tables: torch.Tensor, seq_lens: torch.Tensor,
+               n_new: Optional[torch.Tensor] = None) -> None:
+        """Write new tokens k/v [B][T][Hkv][D] at each sequence's position.
+
+        Token i < n_new[b] (all T when n_new is None) of sequence b goes to
+        position seq_lens[b] + i through the block table tables [B][max_blocks];
+        seq_lens holds the lengths before the append and is not modified.
+        """
+        dev = _require_cuda(k, v, tables, seq_lens)
+        if k.dtype != v.dtype or k.dtype not in _IN_DTYPES:
+            raise ValueError("k and v must share dtype float16 or bfloat16")
+        if k.shape != v.shape or k.dim() != 4 or k.stride() != v.stride():
+            raise ValueError("k and v must be [B][T][Hkv][D] with equal strides")
+        if k.stride(3) != 1 or k.stride(2) != k.shape[3]:
+            raise ValueError("each token's [Hkv][D] row must be contiguous")
+        if tables.dim() != 2 or tables.shape[0] != k.shape[0] or seq_lens.shape != (k.shape[0],):
+            raise ValueError("tables must be [B][max_blocks] and seq_lens [B]")
+        tab = tables.to(torch.int32).contiguous()
+        lens = seq_lens.to(torch.int32).contiguous()
+        nn = None
+        if n_new is not None:
+            if n_new.shape != (k.shape[0],):
+                raise ValueError("n_new must be [B]")
+            _require_cuda(n_new)
+            nn = n_new.to(torch.int32).contiguous()
+        check(lib().q4kv_append_tokens(ctypes.byref(self.desc), _ptr(k), _ptr(v), _IN_DTYPES[k.dtype],
+                                       k.shape[0], k.shape[1], _ptr(nn) if nn is not None else None,
+                                       k.stride(0), k.stride(1), _ptr(tab), tab.shape[1], _ptr(lens),
+                                       _stream(dev)),
+              "q4kv_append_tokens")
+
     def invalidate(self, slot_ids: torch.Tensor) -> None:
         """Remap physical slots (block * 256 + offset) to the sentinel."""
         dev = _require_cuda(slot_ids)

@@ -45,6 +45,8 @@ _SIGNATURES = {
     "q4kv_pool_array_bytes": (c_int32, [c_int32, c_int32, c_int64, c_int32, P(c_size_t), P(c_size_t)]),
     "q4kv_quantize_blocks": (c_int32, [P(PoolDesc), c_void_p, c_void_p, c_int32, c_int64, c_int64,
                                        c_void_p, c_void_p]),
+    "q4kv_append_tokens": (c_int32, [P(PoolDesc), c_void_p, c_void_p, c_int32, c_int32, c_int32,
+                                     c_void_p, c_int64, c_int64, c_void_p, c_int32, c_void_p, c_void_p]),
     "q4kv_dequantize": (c_int32, [P(PoolDesc), c_void_p, c_int32, c_void_p, c_void_p, c_int32,
                                   c_int32, c_void_p]),
     "q4kv_invalidate_slots": (c_int32, [P(PoolDesc), c_void_p, c_int64, c_void_p]),

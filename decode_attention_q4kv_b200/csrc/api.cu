@@ -97,6 +97,28 @@ q4kv_status q4kv_quantize_blocks(const q4kv_pool* pool, const void* k, const voi
                                    block_ids, as_stream(stream)));
 }
 
+q4kv_status q4kv_append_tokens(const q4kv_pool* pool, const void* k, const void* v,
+                               int32_t in_dtype, int32_t batch, int32_t max_new,
+                               const int32_t* n_new, int64_t seq_stride, int64_t token_stride,
+                               const int32_t* tables, int32_t max_blocks, const int32_t* seq_lens,
+                               void* stream) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  if (batch < 0 || max_new < 0 || seq_stride < 0) return Q4KV_ERR_INVALID_ARG;
+  const int64_t rows = batch > 0 && max_new > 0 ? 1 : 0;
+  st = check_input(k, in_dtype, rows, token_stride, pool->n_kv_heads, pool->head_dim);
+  if (st != Q4KV_OK) return st;
+  st = check_input(v, in_dtype, rows, token_stride, pool->n_kv_heads, pool->head_dim);
+  if (st != Q4KV_OK) return st;
+  if ((seq_stride * 2) % 16 != 0) return Q4KV_ERR_INVALID_ARG;
+  if (rows == 0) return Q4KV_OK;
+  if (tables == nullptr || !aligned(tables, 4) || max_blocks < 1 || seq_lens == nullptr ||
+      !aligned(seq_lens, 4) || (n_new != nullptr && !aligned(n_new, 4)))
+    return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_append(view_of(*pool), k, v, in_dtype, batch, max_new, n_new, seq_stride,
+                                 token_stride, tables, max_blocks, seq_lens, as_stream(stream)));
+}
+
 q4kv_status q4kv_dequantize(const q4kv_pool* pool, const int32_t* block_ids, int32_t n_blocks,
                             void* k_out, void* v_out, int32_t out_dtype, int32_t unrotate_k,
                             void* stream) {

@@ -108,6 +108,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, int in_dtype,
                             int64_t n_tokens, int64_t token_stride, const int32_t* block_ids,
                             cudaStream_t stream);
+cudaError_t launch_append(const PoolView& pool, const void* k, const void* v, int in_dtype,
+                          int32_t batch, int32_t max_new, const int32_t* n_new, int64_t seq_stride,
+                          int64_t token_stride, const int32_t* tables, int32_t max_blocks,
+                          const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,
                               void* k_out, void* v_out, int out_dtype, int unrotate_k,
                               cudaStream_t stream);

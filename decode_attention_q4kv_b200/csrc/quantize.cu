@@ -467,6 +467,77 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
 // Scalar butterflies for the decoder's optional un-rotation (channels 16j ..
 // 16j+15 of the lane in order); same stage order and operations as above.
+// ---------------------------------------------------------------------------
+// Append kernel: new tokens of many sequences, each at its own position.  A
+// warp item is one (sequence, new token) and VPW consecutive KV heads (a lane
+// holds 16 channels of one head, as in the bulk encoder, so the rotation and
+// the group statistics are the same warp code); items are walked with a grid
+// stride.  The data are small (a few tokens per sequence), so rows are read
+// with plain 16-byte loads.
+// ---------------------------------------------------------------------------
+template <int D, typename InT, bool ROT>
+__global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ PoolView pool,
+                                                     const InT* __restrict__ k, const InT* __restrict__ v,
+                                                     int32_t batch, int32_t max_new,
+                                                     const int32_t* __restrict__ n_new, int64_t seq_stride,
+                                                     int64_t token_stride, const int32_t* __restrict__ tables,
+                                                     int32_t max_blocks, const int32_t* __restrict__ seq_lens) {
+  using S = Shape<D>;
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int r = lane / S::LPV, j = lane % S::LPV;
+  const int hkv = pool.n_kv_heads;
+  const int hgroups = (hkv + S::VPW - 1) / S::VPW;
+  const int64_t n_items = static_cast<int64_t>(batch) * max_new * hgroups;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; item < n_items;
+       item += n_warps) {
+    const int hg = static_cast<int>(item % hgroups);
+    const int64_t bi = item / hgroups;
+    const int i = static_cast<int>(bi % max_new);
+    const int b = static_cast<int>(bi / max_new);
+    if (n_new != nullptr && i >= __ldg(n_new + b)) continue;    // warp-uniform
+    const int len = __ldg(seq_lens + b);
+    const int64_t p = static_cast<int64_t>(len) + i;
+    if (len < 0 || p >= static_cast<int64_t>(max_blocks) * kBlockTokens) {
+      if (lane == 0 && hg == 0) raise_error(pool.error_word, Q4KV_DEVERR_SEQ_LEN);
+      continue;
+    }
+    const int32_t blk = __ldg(tables + static_cast<int64_t>(b) * max_blocks + p / kBlockTokens);
+    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+      if (lane == 0 && hg == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const int slot = static_cast<int>(p % kBlockTokens);
+    const int h = hg * S::VPW + r;
+    const bool valid = h < hkv;
+    const int hs = valid ? h : hkv - 1;   // lanes past the last head read a real row, store nothing
+    const int64_t src = static_cast<int64_t>(b) * seq_stride + static_cast<int64_t>(i) * token_stride +
+                        static_cast<int64_t>(hs) * D + j * kEPL;
+    const uint4 k0 = __ldg(reinterpret_cast<const uint4*>(k + src));
+    const uint4 k1 = __ldg(reinterpret_cast<const uint4*>(k + src) + 1);
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(v + src));
+    const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(v + src) + 1);
+    const bool is8 = blk >= pool.n_q4;
+    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+    const int64_t row = (phys * hkv + hs) * kBlockTokens + slot;   // (block, head, slot)
+    float2 xk[8], xv[8];
+    unpack16<InT>(k0, k1, xk);
+    unpack16<InT>(v0, v1, xv);
+    if (ROT) rotate_pairs<D>(xk, j);
+    constexpr float ks = ROT ? kRotScale<D> : 1.0f;
+    if (is8)
+      encode_kv<8>(xk, ks, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
+                   pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+    else
+      encode_kv<4>(xk, ks, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
+                   pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+    if (lane == 0 && hg == 0)
+      atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32, ~(1u << (slot % 32)));
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void fwht_vector(float (&x)[kEPL], int j) {
 #pragma unroll
@@ -674,6 +745,36 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
 #undef Q4KV_LAUNCH_QR
 #undef Q4KV_LAUNCH_Q
   return e;
+}
+
+cudaError_t launch_append(const PoolView& pool, const void* k, const void* v, int in_dtype,
+                          int32_t batch, int32_t max_new, const int32_t* n_new, int64_t seq_stride,
+                          int64_t token_stride, const int32_t* tables, int32_t max_blocks,
+                          const int32_t* seq_lens, cudaStream_t stream) {
+  const int d = pool.head_dim;
+  const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;
+  const int64_t items = static_cast<int64_t>(batch) * max_new * ((pool.n_kv_heads + vpw - 1) / vpw);
+  if (items == 0) return cudaSuccess;
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+  int64_t g = (items + 7) / 8;                   // 8 warps per CTA
+  if (g > static_cast<int64_t>(sms) * 8) g = static_cast<int64_t>(sms) * 8;
+  const dim3 grid(static_cast<unsigned>(g)), block(256);
+#define Q4KV_LAUNCH_A(DD, T, R)                                                                     \
+  return launch_pdl(append_kernel<DD, T, R>, grid, block, 0, stream, pool, static_cast<const T*>(k), \
+                    static_cast<const T*>(v), batch, max_new, n_new, seq_stride, token_stride,        \
+                    tables, max_blocks, seq_lens)
+#define Q4KV_LAUNCH_AR(DD, T)       \
+  if (pool.k_rotated) {             \
+    Q4KV_LAUNCH_A(DD, T, true);     \
+  } else {                          \
+    Q4KV_LAUNCH_A(DD, T, false);    \
+  }
+  if (d == 128 && in_dtype == Q4KV_F16) { Q4KV_LAUNCH_AR(128, __half) }
+  if (d == 128) { Q4KV_LAUNCH_AR(128, __nv_bfloat16) }
+  if (in_dtype == Q4KV_F16) { Q4KV_LAUNCH_AR(256, __half) }
+  Q4KV_LAUNCH_AR(256, __nv_bfloat16)
+#undef Q4KV_LAUNCH_AR
+#undef Q4KV_LAUNCH_A
 }
 
 cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,

@@ -9,7 +9,10 @@
  *          Sec. 2.1 item 2: 4-bit codes packed in uint32 words, one 16-bit
  *          scale and one 16-bit bias per group, read by attention directly
  *          ("direct restore").  Sec. 2.1 item 3: attention batched over many
- *          agents' quantised caches.  Sec. 2.2: GQA.
+ *          agents' quantised caches, one agent decoding while another's
+ *          cache is brought in.  Sec. 2.1 item 4: a prompt that extends a
+ *          cached prefix (EXTEND match) grows the cache instead of being
+ *          prefilled again.  Sec. 2.2: GQA.
  *   [UQ]   UltraQuant news item (poko-everyday.com, arXiv 2606.20474),
  *          section "技術/ビジネス面": Walsh-Hadamard rotation before 4-bit
  *          quantisation; keys and values treated asymmetrically.
@@ -150,6 +153,37 @@ q4kv_status q4kv_pool_array_bytes(int32_t head_dim, int32_t n_kv_heads, int64_t 
 q4kv_status q4kv_quantize_blocks(const q4kv_pool *pool, const void *k, const void *v,
                                  int32_t in_dtype, int64_t n_tokens, int64_t token_stride,
                                  const int32_t *block_ids, void *stream);
+
+/*
+ * Append new tokens to each sequence's cache at its own position ([AMBP]
+ * sec. 2.1 items 3-4: decoding and EXTEND both grow a cached sequence in
+ * place instead of prefilling it again).
+ *   k, v         device, dtype in_dtype (Q4KV_F16 or Q4KV_BF16); token i of
+ *                sequence b is the [Hkv][D] row at index
+ *                b*seq_stride + i*token_stride (elements), rows contiguous;
+ *                16-byte aligned, both strides * elem_size % 16 == 0,
+ *                token_stride >= Hkv*D.  Values must be finite.
+ *   batch, max_new  sequences and tokens per sequence in k / v.
+ *   n_new        device int32 [batch] with 0 <= n_new[b] <= max_new, the
+ *                tokens sequence b appends; NULL = every sequence appends
+ *                max_new.
+ *   tables       device int32 [batch][max_blocks]: logical block i of
+ *                sequence b is physical block tables[b*max_blocks + i].
+ *   seq_lens     device int32 [batch], lengths BEFORE the append (not
+ *                modified; the caller adds n_new afterwards).
+ *   Token i of sequence b is written to position p = seq_lens[b] + i, i.e.
+ *   slot p % 256 of block tables[b][p / 256], encoded exactly as
+ *   q4kv_quantize_blocks encodes the same row, and its remap bit is cleared.
+ *   The positions written must map to distinct slots.  A position at or
+ *   past max_blocks*256 (or a negative length) skips the token and raises
+ *   Q4KV_DEVERR_SEQ_LEN; a block id out of range skips it and raises
+ *   Q4KV_DEVERR_BLOCK_ID.  batch == 0 or max_new == 0 is a no-op.
+ */
+q4kv_status q4kv_append_tokens(const q4kv_pool *pool, const void *k, const void *v,
+                               int32_t in_dtype, int32_t batch, int32_t max_new,
+                               const int32_t *n_new, int64_t seq_stride, int64_t token_stride,
+                               const int32_t *tables, int32_t max_blocks, const int32_t *seq_lens,
+                               void *stream);
 
 /*
  * Dequantise whole blocks ([QKVS] "Méthodologie": dequantise before use).

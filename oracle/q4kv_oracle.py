@@ -15,7 +15,9 @@ What it computes, step by step, and where each step comes from:
           uint32 words with one 16-bit scale and one 16-bit bias per group,
           read directly by attention ("direct restore"), about 72 % smaller
           than FP16.  Section 2.1, item 3: attention batched over several
-          agents' quantised caches.  Section 2.2: GQA models.
+          agents' quantised caches.  Section 2.1, item 4: a prompt that
+          extends a cached prefix grows the cache instead of being
+          prefilled again.  Section 2.2: GQA models.
   [UQ]    UltraQuant news item (poko-everyday.com, arXiv 2606.20474),
           section "technology / business": a Walsh-Hadamard rotation before
           4-bit quantisation, with keys and values treated asymmetrically.
@@ -267,6 +269,39 @@ class OraclePool:
                     self.codes8[name][i8, :, : t1 - t0] = codes
                     self.params8[name][i8, :, : t1 - t0] = par
             for slot in range(t1 - t0):
+                self.mask[blk, slot // 32] &= np.uint32(~(1 << (slot % 32)) & 0xFFFFFFFF)
+
+    def append_tokens(self, k: np.ndarray, v: np.ndarray, dtype: str, tables: np.ndarray,
+                      seq_lens: Sequence[int], n_new: Optional[Sequence[int]] = None) -> None:
+        """Grow each sequence's cache in place [AMBP 2.1 items 3-4].
+
+        k, v: [B][T][Hkv][D].  Token i < n_new[b] (all T if None) of sequence
+        b is the token at position p = seq_lens[b] + i, stored in block
+        tables[b][p // 256], slot p % 256, with exactly the per-vector encoding
+        quantize_blocks gives it; the slot's mask bit is cleared.
+        """
+        kf = to_f32(k, dtype)
+        vf = to_f32(v, dtype)
+        nb, nt = kf.shape[0], kf.shape[1]
+        for b in range(nb):
+            for i in range(nt if n_new is None else int(n_new[b])):
+                p = int(seq_lens[b]) + i
+                blk = int(tables[b][p // BLOCK_TOKENS])
+                slot = p % BLOCK_TOKENS
+                bits = self.bits(blk)
+                kk = kf[b, i][None]                           # [1][Hkv][D]
+                if self.k_rotated:
+                    kk = rotate_f32(kk)
+                for name, x in (("k", kk), ("v", vf[b, i][None])):
+                    codes, s_h, z_h = quantize_groups(x, bits)
+                    par = np.stack([s_h[0], z_h[0]], axis=-1)  # [Hkv][D/64][2]
+                    if bits == 4:
+                        self.codes4[name][blk, :, slot] = pack_nibbles(codes[0])
+                        self.params4[name][blk, :, slot] = par
+                    else:
+                        i8 = blk - self.n_q4
+                        self.codes8[name][i8, :, slot] = codes[0]
+                        self.params8[name][i8, :, slot] = par
                 self.mask[blk, slot // 32] &= np.uint32(~(1 << (slot % 32)) & 0xFFFFFFFF)
 
     def invalidate_slots(self, slot_ids: Sequence[int]) -> None:

@@ -24,7 +24,7 @@ def _pool(**kw):
 
 def test_exports_every_declared_function():
     names = _lib.header_functions()
-    assert len(names) == 12
+    assert len(names) == 13
     for n in names:
         assert hasattr(L, n), n
     # the binding declares a signature for each of them
@@ -128,6 +128,28 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.q4kv_mixed_block_ids(FAKE, 70000, 1, 0, 0, FAKE, None) == _lib.ERR_INVALID_ARG
     assert L.q4kv_mixed_block_ids(FAKE, 10, 11, 0, 0, FAKE, None) == _lib.ERR_INVALID_ARG
     assert L.q4kv_mixed_block_ids(FAKE, 0, 0, 0, 0, FAKE, None) == 0
+
+
+def test_append_rejects_bad_arguments_without_launching():
+    p = _pool()
+    a = L.q4kv_append_tokens
+
+    def call(pool=p, k=FAKE, v=FAKE, dt=0, b=2, t=3, nn=None, ss=3 * 1024, ts=1024, tab=FAKE, mb=4, lens=FAKE):
+        return a(ctypes.byref(pool), k, v, dt, b, t, nn, ss, ts, tab, mb, lens, None)
+
+    assert call(dt=2) == _lib.ERR_INVALID_ARG                 # fp32 input
+    assert call(b=-1) == _lib.ERR_INVALID_ARG
+    assert call(t=-1) == _lib.ERR_INVALID_ARG
+    assert call(k=FAKE + 8) == _lib.ERR_INVALID_ARG           # misaligned rows
+    assert call(ts=1020) == _lib.ERR_INVALID_ARG              # token stride below Hkv*D
+    assert call(ts=1028) == _lib.ERR_INVALID_ARG              # token stride not a 16-byte multiple
+    assert call(ss=3 * 1024 + 4) == _lib.ERR_INVALID_ARG      # sequence stride not a 16-byte multiple
+    assert call(tab=None) == _lib.ERR_INVALID_ARG
+    assert call(lens=None) == _lib.ERR_INVALID_ARG
+    assert call(mb=0) == _lib.ERR_INVALID_ARG
+    assert call(nn=FAKE + 2) == _lib.ERR_INVALID_ARG
+    assert call(pool=_pool(head_dim=96)) != 0
+    assert call(b=0) == 0 and call(t=0) == 0                  # nothing to append: no launch
 
 
 def test_decode_rejects_bad_arguments_without_launching():

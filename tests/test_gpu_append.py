@@ -1,0 +1,117 @@
+"""Appending tokens in place ([AMBP] 2.1 items 3-4): the GPU encoder writes each
+new token at its sequence's position through the block table, bit-identical
+to the oracle; a generation step (append, then decode) matches the oracle's
+attention."""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_q4kv_b200 as q4
+from decode_attention_q4kv_b200 import _lib
+from decode_attention_q4kv_b200 import workloads as W
+from helpers import assert_close, assert_pool_equal, cuda, host
+from oracle import q4kv_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _grow(d, hkv, dtype, rotated, n_q4, n_q8, lens, new, tables, max_new, strided=False, seed=0):
+    """Prefill each sequence's first lens[b] tokens, then append; returns (gpu pool, oracle pool, k, v)."""
+    dev = cuda()
+    B = len(lens)
+    name = "fp16" if dtype == torch.float16 else "bf16"
+    pool = q4.Q4KVPool(hkv, d, n_q4, n_q8, k_rotated=rotated, device=dev)
+    ref = O.OraclePool(hkv, d, n_q4, n_q8, k_rotated=rotated)
+    for b in range(B):
+        if lens[b] == 0:
+            continue
+        k, v = W.random_small(lens[b], hkv, d, name, seed=seed + 10 * b)
+        nb = -(-lens[b] // 256)
+        ids = tables[b][:nb].tolist()
+        pool.quantize(k.to(dev), v.to(dev), torch.tensor(ids, dtype=torch.int32, device=dev))
+        kh, dt = host(k)
+        vh, _ = host(v)
+        ref.quantize_blocks(kh, vh, dt, ids)
+    kn, vn = W.random_small(B * max_new, hkv, d, name, seed=seed + 999)
+    kn = kn.view(B, max_new, hkv, d)
+    vn = vn.view(B, max_new, hkv, d)
+    if strided:   # each sequence's rows inside a wider buffer, tokens 2 rows apart
+        big_k = torch.zeros(B, 2 * max_new + 1, hkv, d, dtype=dtype)
+        big_v = torch.zeros_like(big_k)
+        big_k[:, 0:2 * max_new:2] = kn
+        big_v[:, 0:2 * max_new:2] = vn
+        kd, vd = big_k.to(dev)[:, 0:2 * max_new:2], big_v.to(dev)[:, 0:2 * max_new:2]
+    else:
+        kd, vd = kn.to(dev), vn.to(dev)
+    nn = None if new is None else torch.tensor(new, dtype=torch.int32, device=dev)
+    pool.append(kd, vd, torch.as_tensor(tables, dtype=torch.int32).to(dev),
+                torch.tensor(lens, dtype=torch.int32, device=dev), nn)
+    torch.cuda.synchronize()
+    kh, dt = host(kn.reshape(B * max_new, hkv, d))
+    vh, _ = host(vn.reshape(B * max_new, hkv, d))
+    ref.append_tokens(kh.reshape(B, max_new, hkv, d), vh.reshape(B, max_new, hkv, d), dt,
+                      np.asarray(tables), lens, new)
+    return pool, ref
+
+
+@pytest.mark.parametrize("d,hkv,dtype,rotated", [(128, 8, torch.float16, True), (256, 8, torch.bfloat16, True),
+                                                 (128, 3, torch.bfloat16, False), (256, 1, torch.float16, True),
+                                                 (256, 5, torch.bfloat16, False)])
+@pytest.mark.parametrize("strided", [False, True])
+def test_append_bit_exact(d, hkv, dtype, rotated, strided):
+    # ragged lengths: empty, mid-block, one token before a block boundary, a
+    # full block; ragged counts including 0; blocks of both widths
+    lens = [0, 100, 255, 256, 510]
+    new = [3, 1, 3, 0, 2]
+    tables = np.array([[0, 7], [2, 9], [4, 1], [6, 3], [5, 8]], dtype=np.int32)
+    pool, ref = _grow(d, hkv, dtype, rotated, 6, 4, lens, new, tables, 3, strided, seed=d + hkv)
+    assert pool.read_device_error() == 0
+    assert_pool_equal(pool, ref)
+
+
+def test_append_all_tokens_when_counts_omitted():
+    lens = [17, 300]
+    tables = np.array([[1, 0], [2, 3]], dtype=np.int32)
+    pool, ref = _grow(128, 8, torch.float16, True, 4, 0, lens, None, tables, 4)
+    assert pool.read_device_error() == 0
+    assert_pool_equal(pool, ref)
+
+
+def test_append_past_the_table_and_bad_block_raise_and_skip():
+    dev = cuda()
+    hkv, d = 2, 128
+    pool = q4.Q4KVPool(hkv, d, 4, device=dev)
+    before = [pool.k_codes4.clone(), pool.mask.clone()]
+    k, v = W.random_small(4, hkv, d, "fp16", seed=5)
+    k = k.view(2, 2, hkv, d).to(dev)
+    v = v.view(2, 2, hkv, d).to(dev)
+    tables = torch.tensor([[0], [1]], dtype=torch.int32, device=dev)
+    # sequence 0 is full (256 tokens, one block): both new tokens fall past the table
+    pool.append(k[:1], v[:1], tables[:1], torch.tensor([256], dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    assert pool.read_device_error() & _lib.DEVERR_SEQ_LEN
+    assert torch.equal(pool.k_codes4, before[0]) and torch.equal(pool.mask, before[1])
+    bad = torch.tensor([[7]], dtype=torch.int32, device=dev)
+    pool.append(k[1:], v[1:], bad, torch.tensor([0], dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    assert pool.read_device_error() & _lib.DEVERR_BLOCK_ID
+    assert torch.equal(pool.k_codes4, before[0])
+
+
+def test_generation_step_append_then_decode():
+    # one decode step of a batch: append the new token of every sequence, then
+    # attend over the grown cache with the new token included
+    dev = cuda()
+    hkv, hq, d = 8, 32, 128
+    lens = [700, 256, 1, 1023]
+    B = len(lens)
+    tables = np.arange(B * 4, dtype=np.int32)[::-1].copy().reshape(B, 4)
+    pool, ref = _grow(d, hkv, torch.float16, True, B * 4, 0, lens, [1] * B, tables, 1, seed=3)
+    assert pool.read_device_error() == 0
+    q = torch.randn(B, hq, d, generator=torch.Generator().manual_seed(4)).to(torch.float16)
+    grown = [n + 1 for n in lens]
+    out = q4.decode_attention(pool, q.to(dev), torch.as_tensor(tables).to(dev),
+                              torch.tensor(grown, dtype=torch.int32, device=dev), out_dtype=torch.float32)
+    qh, dt = host(q)
+    want = O.decode_attention(ref, qh, dt, tables, grown)
+    assert_close(out, want, what="append + decode")

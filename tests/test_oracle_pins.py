@@ -441,3 +441,39 @@ def test_bf16_conversion_is_exact():
     f = O.to_f32(bits, "bf16")
     assert list(f[:3]) == [1.0, -2.0, 0.25]
     assert f[3] == np.float32(2.0 ** -133)
+
+
+# ---------------------------------------------------------------------------
+# Appending tokens in place
+# ---------------------------------------------------------------------------
+
+def test_append_equals_bulk_encoding_of_whole_sequences():
+    # Growing sequences in place (ragged lengths, one crossing a block
+    # boundary, one not growing, appended slots previously remapped) must leave
+    # the pool exactly as encoding each whole sequence in one bulk call
+    # through its block table.
+    rng = np.random.default_rng(17)
+    hkv, d = 3, 128
+    lens, new = [300, 254, 40], [5, 4, 0]
+    tables = np.array([[3, 0], [1, 2], [4, 5]])
+    ks = [rng.standard_normal((lens[b] + new[b], hkv, d)).astype(np.float16) for b in range(3)]
+    vs = [rng.standard_normal((lens[b] + new[b], hkv, d)).astype(np.float16) for b in range(3)]
+    ref = O.OraclePool(hkv, d, 6)
+    grown = O.OraclePool(hkv, d, 6)
+    for b in range(3):
+        nb = -(-(lens[b] + new[b]) // O.BLOCK_TOKENS)
+        ref.quantize_blocks(ks[b], vs[b], "fp16", tables[b][:nb])
+        nb0 = -(-lens[b] // O.BLOCK_TOKENS)
+        grown.quantize_blocks(ks[b][:lens[b]], vs[b][:lens[b]], "fp16", tables[b][:nb0])
+        slots = [int(tables[b][p // 256]) * 256 + p % 256 for p in range(lens[b], lens[b] + new[b])]
+        grown.invalidate_slots(slots)
+    kn = np.zeros((3, 5, hkv, d), np.float16)
+    vn = np.zeros((3, 5, hkv, d), np.float16)
+    for b in range(3):
+        kn[b, :new[b]] = ks[b][lens[b]:]
+        vn[b, :new[b]] = vs[b][lens[b]:]
+    grown.append_tokens(kn, vn, "fp16", tables, lens, new)
+    for name in "kv":
+        np.testing.assert_array_equal(grown.codes4[name], ref.codes4[name])
+        np.testing.assert_array_equal(grown.params4[name].view(np.uint16), ref.params4[name].view(np.uint16))
+    np.testing.assert_array_equal(grown.mask, ref.mask)
