@@ -47,6 +47,7 @@ _SIGNATURES = {
                                        c_void_p, c_void_p]),
     "q4kv_append_tokens": (c_int32, [P(PoolDesc), c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                      c_void_p, c_int64, c_int64, c_void_p, c_int32, c_void_p, c_void_p]),
+    "q4kv_selftest_bounded_wait": (c_int32, [c_void_p, c_int32, c_void_p]),
     "q4kv_dequantize": (c_int32, [P(PoolDesc), c_void_p, c_int32, c_void_p, c_void_p, c_int32,
                                   c_int32, c_void_p]),
     "q4kv_invalidate_slots": (c_int32, [P(PoolDesc), c_void_p, c_int64, c_void_p]),

@@ -119,6 +119,12 @@ q4kv_status q4kv_append_tokens(const q4kv_pool* pool, const void* k, const void*
                                  token_stride, tables, max_blocks, seq_lens, as_stream(stream)));
 }
 
+q4kv_status q4kv_selftest_bounded_wait(uint32_t* error_word, int32_t tries, void* stream) {
+  if (error_word == nullptr || !aligned(error_word, 4) || tries < 1 || tries > (1 << 21))
+    return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_selftest_wait(error_word, static_cast<unsigned>(tries), as_stream(stream)));
+}
+
 q4kv_status q4kv_dequantize(const q4kv_pool* pool, const int32_t* block_ids, int32_t n_blocks,
                             void* k_out, void* v_out, int32_t out_dtype, int32_t unrotate_k,
                             void* stream) {

@@ -40,9 +40,9 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 // Bounded wait; false when the limit ran out.  The suspend hint is only an
 // upper bound, so between tries the thread also sleeps, backing off from
 // 32 ns to 1 us; the whole wait stays above two seconds before it gives up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned limit = kSpinLimit) {
   unsigned ns = 32;
-  for (unsigned i = 0; i < kSpinLimit; ++i) {
+  for (unsigned i = 0; i < limit; ++i) {
     if (mbar_try(bar, parity)) return true;
     __nanosleep(ns);
     ns = ns < 1024 ? 2 * ns : 1024;

@@ -299,6 +299,8 @@ __device__ __forceinline__ float block_reduce(float x, bool is_max, float* red) 
   return x;
 }
 
+constexpr int kFewSplits = 16;
+
 template <int D>
 __global__ void __launch_bounds__(D / 4) merge_kernel(const DecodeArgs a) {
   constexpr int T = D / 4;
@@ -310,6 +312,46 @@ __global__ void __launch_bounds__(D / 4) merge_kernel(const DecodeArgs a) {
   const int64_t row = blockIdx.x;
   const int S = a.plan.n_splits;
   const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row * S;
+  if (S <= kFewSplits) {
+    // few splits: every thread loads all (m, l) pairs and its partials in one
+    // round of loads and merges them itself, without a block reduction
+    const float4* op = reinterpret_cast<const float4*>(a.ws_o + row * S * D) + threadIdx.x;
+    float2 st[kFewSplits];
+    float4 ov[kFewSplits];
+#pragma unroll
+    for (int i = 0; i < kFewSplits; ++i)
+      if (i < S) {
+        st[i] = ml[i];
+        ov[i] = op[static_cast<int64_t>(i) * T];
+      }
+    float M = -INFINITY;
+    bool pois = false;
+#pragma unroll
+    for (int i = 0; i < kFewSplits; ++i)
+      if (i < S) {
+        M = fmaxf(M, st[i].x);
+        pois |= st[i].y < 0.0f;
+      }
+    float L = 0.0f;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int i = 0; i < kFewSplits; ++i)
+      if (i < S && M != -INFINITY && st[i].x != -INFINITY) {   // an empty split adds nothing
+        const float w = expf(st[i].x - M);
+        L = fmaf(st[i].y, w, L);
+        acc.x = fmaf(ov[i].x, w, acc.x);
+        acc.y = fmaf(ov[i].y, w, acc.y);
+        acc.z = fmaf(ov[i].z, w, acc.z);
+        acc.w = fmaf(ov[i].w, w, acc.w);
+      }
+    const bool ok = !pois && M != -INFINITY && L > 0.0f;
+    const int64_t base = row * D + 4 * threadIdx.x;
+    store_out(a.out, a.out_dtype, base, ok ? acc.x / L : 0.0f);
+    store_out(a.out, a.out_dtype, base + 1, ok ? acc.y / L : 0.0f);
+    store_out(a.out, a.out_dtype, base + 2, ok ? acc.z / L : 0.0f);
+    store_out(a.out, a.out_dtype, base + 3, ok ? acc.w / L : 0.0f);
+    return;
+  }
   float M = -INFINITY, pois = 0.0f;
   for (int i = threadIdx.x; i < S; i += T) {
     const float2 v = ml[i];

@@ -8,6 +8,7 @@
 // Mixed widths: QKVShare (arXiv 2605.03884 summary), "Méthodologie" -- bit
 // widths per token from {2, 4, 8, FP16}.  This library chooses 8 bits per
 // whole block for the blocks with the largest mean |K| and 4 bits elsewhere.
+#include "async_copy.cuh"
 #include "q4kv_internal.cuh"
 
 namespace q4kv {
@@ -121,6 +122,17 @@ __global__ void __launch_bounds__(1024) mixed_ids_kernel(int32_t n, int32_t q4_f
   }
 }
 
+// One barrier that no thread ever arrives on: the bounded wait must give up.
+__global__ void selftest_wait_kernel(uint32_t* error_word, unsigned tries) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (!mbar_wait(&bar, 0, tries)) raise_error(error_word, Q4KV_DEVERR_TIMEOUT);
+}
+
 }  // namespace
 
 cudaError_t launch_invalidate(const PoolView& pool, const int64_t* slot_ids, int64_t n,
@@ -149,6 +161,11 @@ cudaError_t launch_mixed_ids(const double* absmean, int32_t n, int32_t n_q8, int
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   mixed_ids_kernel<<<1, 1024, 0, stream>>>(n, q4_first, q8_first, ids);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(uint32_t* error_word, unsigned tries, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(error_word, tries);
   return cudaGetLastError();
 }
 

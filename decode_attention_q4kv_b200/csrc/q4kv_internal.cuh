@@ -112,6 +112,7 @@ cudaError_t launch_append(const PoolView& pool, const void* k, const void* v, in
                           int32_t batch, int32_t max_new, const int32_t* n_new, int64_t seq_stride,
                           int64_t token_stride, const int32_t* tables, int32_t max_blocks,
                           const int32_t* seq_lens, cudaStream_t stream);
+cudaError_t launch_selftest_wait(uint32_t* error_word, unsigned tries, cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,
                               void* k_out, void* v_out, int out_dtype, int unrotate_k,
                               cudaStream_t stream);

@@ -314,6 +314,16 @@ q4kv_status q4kv_decode_attention_static_scratch(const q4kv_pool *pool,
                                                  void *out, int32_t out_dtype, void *stream);
 
 /*
+ * Diagnostic (no counterpart on the pages): launch one CTA that waits on a
+ * shared-memory barrier nothing ever completes, with the bounded wait every
+ * kernel of this library uses, limited to `tries` rounds (1 <= tries <=
+ * 2^21; each round sleeps up to ~1 us).  When the limit runs out the kernel
+ * ORs Q4KV_DEVERR_TIMEOUT into *error_word (device uint32) and returns, so the
+ * context stays usable; tests use it to check that waits end.
+ */
+q4kv_status q4kv_selftest_bounded_wait(uint32_t *error_word, int32_t tries, void *stream);
+
+/*
  * Wait for `stream`, read pool->error_word into *bits, and zero it when
  * `clear` is nonzero.  Returns Q4KV_ERR_DEVICE when any bit was set,
  * Q4KV_OK otherwise (and *bits = 0 when pool->error_word is NULL).

@@ -24,7 +24,7 @@ def _pool(**kw):
 
 def test_exports_every_declared_function():
     names = _lib.header_functions()
-    assert len(names) == 13
+    assert len(names) == 14
     for n in names:
         assert hasattr(L, n), n
     # the binding declares a signature for each of them
@@ -179,6 +179,13 @@ def test_decode_rejects_bad_arguments_without_launching():
     st, empty = _plan(0, 32, 8, 128, 4, 0, 148)
     assert st == 0
     assert call(pl=empty, ws=0, wsb=0) == 0                              # batch 0: nothing to do
+
+
+def test_selftest_rejects_bad_arguments():
+    assert L.q4kv_selftest_bounded_wait(None, 10, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_selftest_bounded_wait(FAKE + 2, 10, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_selftest_bounded_wait(FAKE, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_selftest_bounded_wait(FAKE, (1 << 21) + 1, None) == _lib.ERR_INVALID_ARG
 
 
 def test_read_device_error_without_word():
