@@ -147,8 +147,9 @@ __device__ __forceinline__ float quot(float u, float s, float r) {
 // Codes are defined as clamp(rne(fl(fl(x - z) / s)), 0, L): u = fl(x - z),
 // then the correctly rounded quotient above, then round-half-even to an
 // integer by adding 1.5 * 2^23.  The quotient is monotone in x, so when the
-// group's extremes give quotients in [-0.5, L + 0.5) no code needs the
-// clamp; other groups (a zero far outside the fp16 grid of the values) are
+// group's extremes give quotients inside [-0.49, L + 0.49] (tested with the
+// uncorrected product (x - z) r, off by a few ulp) no code needs the clamp;
+// other groups (a zero far outside the fp16 grid of the values) are
 // recomputed with IEEE division and an integer clamp.  s = 0 (a constant
 // group) is handled by r = 0, which makes every quotient 0.
 //
@@ -179,16 +180,20 @@ __device__ __forceinline__ GroupParams group_params(const float2 (&x)[8], float 
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  mn = __fadd_rn(__fmul_rn(mn, xs), 0.0f);  // exact scaling; -0 -> +0
-  mx = __fadd_rn(__fmul_rn(mx, xs), 0.0f);
+  mn = __fmaf_rn(mn, xs, 0.0f);  // exact scaling, and -0 + 0 = +0
+  mx = __fmaf_rn(mx, xs, 0.0f);
   GroupParams g;
   g.sh = __float2half_rn(quot(__fsub_rn(mx, mn), static_cast<float>(L), kRecipL));
   g.zh = __float2half_rn(mn);
   g.s = __half2float(g.sh);
   g.z = __half2float(g.zh);
   g.r = g.s != 0.0f ? __frcp_rn(g.s) : 0.0f;
-  const float q_lo = quot(__fsub_rn(mn, g.z), g.s, g.r), q_hi = quot(__fsub_rn(mx, g.z), g.s, g.r);
-  g.fast = q_lo >= -0.5f && q_hi < L + 0.5f;
+  // fl(x r + fl(-z r)) differs from the defined quotient by at most
+  // (4 (L + 1) + |z r|) 2^-24 < 0.005 when |z r| <= 2^16, so the 0.01 margin
+  // keeps the test conservative; a group it rejects just takes the exact path
+  const float nzr = __fmul_rn(-g.z, g.r);
+  const float q_lo = __fmaf_rn(mn, g.r, nzr), q_hi = __fmaf_rn(mx, g.r, nzr);
+  g.fast = fabsf(nzr) <= 65536.0f && q_lo >= -0.49f && q_hi <= L + 0.49f;
   return g;
 }
 
@@ -316,7 +321,7 @@ struct EncodeGeometry {
   int32_t items_per_head_log2;   // log2(T / VPW)
 };
 
-template <int D, typename InT, bool ROT>
+template <int D, typename InT, bool ROT, bool MIXED>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_kernel(const __grid_constant__ PoolView pool, const InT* __restrict__ k,
                     const InT* __restrict__ v, const __grid_constant__ EncodeGeometry geo,
@@ -434,7 +439,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
       } else {
         const int slot = static_cast<int>(t % kBlockTokens);
-        const bool is8 = blk >= pool.n_q4;
+        const bool is8 = MIXED && blk >= pool.n_q4;   // a pool without 8-bit blocks drops that path
         const int64_t phys = is8 ? blk - pool.n_q4 : blk;
         const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
         float2 xk[8], xv[8];
@@ -721,21 +726,22 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
   const int64_t grid = n_chunks < sms ? n_chunks : sms;
   const size_t smem = kQStages * kQStageBytes + 2 * kQStages * sizeof(uint64_t);
   cudaError_t e = cudaSuccess;
-#define Q4KV_LAUNCH_Q(DD, T, R)                                                                   \
-  do {                                                                                              \
-    e = cudaFuncSetAttribute(quantize_kernel<DD, T, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             static_cast<int>(smem));                                               \
-    if (e == cudaSuccess)                                                                           \
-      e = launch_pdl(quantize_kernel<DD, T, R>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),  \
-                     smem, stream, pool, static_cast<const T*>(k), static_cast<const T*>(v), geo,     \
-                     block_ids);                                                                    \
+#define Q4KV_LAUNCH_Q(DD, T, R, M)                                                                   \
+  do {                                                                                                 \
+    e = cudaFuncSetAttribute(quantize_kernel<DD, T, R, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(smem));                                                  \
+    if (e == cudaSuccess)                                                                              \
+      e = launch_pdl(quantize_kernel<DD, T, R, M>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),  \
+                     smem, stream, pool, static_cast<const T*>(k), static_cast<const T*>(v), geo,        \
+                     block_ids);                                                                       \
   } while (0)
-#define Q4KV_LAUNCH_QR(DD, T)       \
-  do {                              \
-    if (pool.k_rotated)             \
-      Q4KV_LAUNCH_Q(DD, T, true);   \
-    else                            \
-      Q4KV_LAUNCH_Q(DD, T, false);  \
+#define Q4KV_LAUNCH_QR(DD, T)                                   \
+  do {                                                          \
+    const bool mixed = pool.n_q8 > 0;                           \
+    if (pool.k_rotated && mixed) Q4KV_LAUNCH_Q(DD, T, true, true);        \
+    else if (pool.k_rotated) Q4KV_LAUNCH_Q(DD, T, true, false);           \
+    else if (mixed) Q4KV_LAUNCH_Q(DD, T, false, true);                    \
+    else Q4KV_LAUNCH_Q(DD, T, false, false);                              \
   } while (0)
   if (n_chunks == 0) return cudaSuccess;
   if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_QR(128, __half);
