@@ -70,10 +70,13 @@ class Q4KVPool:
     """
 
     def __init__(self, n_kv_heads: int, head_dim: int, n_q4_blocks: int, n_q8_blocks: int = 0,
-                 k_rotated: bool = True, device="cuda"):
+                 k_rotated: bool = True, device="cuda", fp8: bool = False):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("Q4KVPool lives on a CUDA device")
+        if fp8 and (n_q4_blocks or k_rotated):
+            raise ValueError("an FP8 pool has only 8-bit blocks (n_q4_blocks = 0) and raw keys (k_rotated = False)")
+        self.fp8 = bool(fp8)
         self.n_kv_heads, self.head_dim = n_kv_heads, head_dim
         self.n_q4_blocks, self.n_q8_blocks = n_q4_blocks, n_q8_blocks
         self.k_rotated = bool(k_rotated)
@@ -89,11 +92,12 @@ class Q4KVPool:
         self.k_codes4, self.v_codes4 = codes(n_q4_blocks, head_dim // 2), codes(n_q4_blocks, head_dim // 2)
         self.k_params4, self.v_params4 = params(n_q4_blocks), params(n_q4_blocks)
         self.k_codes8, self.v_codes8 = codes(n_q8_blocks, head_dim), codes(n_q8_blocks, head_dim)
-        self.k_params8, self.v_params8 = params(n_q8_blocks), params(n_q8_blocks)
+        n_par8 = 0 if self.fp8 else n_q8_blocks                 # FP8 blocks carry no params
+        self.k_params8, self.v_params8 = params(n_par8), params(n_par8)
         self.mask = torch.zeros((n_q4_blocks + n_q8_blocks, 8), dtype=torch.int32, device=self.device)
         self.error_word = torch.zeros(4, dtype=torch.int32, device=self.device)
         self.desc = _lib.PoolDesc(
-            head_dim, n_kv_heads, int(self.k_rotated), n_q4_blocks, n_q8_blocks, 0,
+            head_dim, n_kv_heads, int(self.k_rotated), n_q4_blocks, n_q8_blocks, int(self.fp8),
             self.k_codes4.data_ptr(), self.v_codes4.data_ptr(),
             self.k_params4.data_ptr(), self.v_params4.data_ptr(),
             self.k_codes8.data_ptr() if n_q8_blocks else 0,

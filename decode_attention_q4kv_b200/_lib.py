@@ -24,7 +24,7 @@ DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT_ID, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 class PoolDesc(ctypes.Structure):
     _fields_ = [("head_dim", c_int32), ("n_kv_heads", c_int32), ("k_rotated", c_int32),
-                ("n_q4_blocks", c_int32), ("n_q8_blocks", c_int32), ("reserved", c_int32),
+                ("n_q4_blocks", c_int32), ("n_q8_blocks", c_int32), ("value_format", c_int32),
                 ("k_codes4", c_void_p), ("v_codes4", c_void_p),
                 ("k_params4", c_void_p), ("v_params4", c_void_p),
                 ("k_codes8", c_void_p), ("v_codes8", c_void_p),

@@ -14,9 +14,11 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 q4kv_status check_pool(const q4kv_pool* p) {
   if (p == nullptr) return Q4KV_ERR_INVALID_ARG;
-  if (p->reserved != 0 || p->n_kv_heads < 1 || p->n_q4_blocks < 0 || p->n_q8_blocks < 0 ||
-      (p->k_rotated != 0 && p->k_rotated != 1))
+  if ((p->value_format != Q4KV_FORMAT_INT && p->value_format != Q4KV_FORMAT_FP8) || p->n_kv_heads < 1 ||
+      p->n_q4_blocks < 0 || p->n_q8_blocks < 0 || (p->k_rotated != 0 && p->k_rotated != 1))
     return Q4KV_ERR_INVALID_ARG;
+  const bool fp8 = p->value_format == Q4KV_FORMAT_FP8;
+  if (fp8 && (p->n_q4_blocks != 0 || p->k_rotated != 0)) return Q4KV_ERR_INVALID_ARG;
   if (p->head_dim != 128 && p->head_dim != 256) return Q4KV_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(p->n_q4_blocks) + p->n_q8_blocks > (int64_t{1} << 31) / kBlockTokens)
     return Q4KV_ERR_INVALID_ARG;
@@ -27,8 +29,8 @@ q4kv_status check_pool(const q4kv_pool* p) {
   }
   if (p->n_q8_blocks > 0) {
     const void* a[4] = {p->k_codes8, p->v_codes8, p->k_params8, p->v_params8};
-    for (const void* x : a)
-      if (x == nullptr || !aligned(x, 16)) return Q4KV_ERR_INVALID_ARG;
+    for (int i = 0; i < (fp8 ? 2 : 4); ++i)   // an FP8 pool has no params
+      if (a[i] == nullptr || !aligned(a[i], 16)) return Q4KV_ERR_INVALID_ARG;
   }
   if (p->n_q4_blocks + p->n_q8_blocks > 0 &&
       (p->remap_mask == nullptr || !aligned(p->remap_mask, 16)))
@@ -274,6 +276,8 @@ q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan*
       static_cast<int64_t>(pool->n_q4_blocks > pool->n_q8_blocks ? pool->n_q4_blocks : pool->n_q8_blocks) *
       pool->n_kv_heads * kBlockTokens;
   if (code_rows >= (int64_t{1} << 31)) return Q4KV_ERR_UNSUPPORTED;
+  // the FP8 comparison cache is read by the tensor-core kernel only
+  if (pool->value_format == Q4KV_FORMAT_FP8 && plan->kernel != 1) return Q4KV_ERR_UNSUPPORTED;
   if (plan->workspace_bytes > 0 &&
       (workspace == nullptr || workspace_bytes < plan->workspace_bytes || !aligned(workspace, 256)))
     return Q4KV_ERR_WORKSPACE;

@@ -459,6 +459,159 @@ __device__ __forceinline__ void tiles(WarpState<D, NT>& st, const uint8_t* stage
   }
 }
 
+// ---------------------------------------------------------------------------
+// FP8 comparison cache: OCP E4M3 keys and values, no params, raw keys.  Both
+// contractions run as fp16 MMAs: a code pair becomes an exact f16x2 with one
+// conversion, the query (pre-scaled by scale * log2 e) enters as fp16 high +
+// low parts (two MMAs, ~22 bits), and a B column is one query head.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t pair16) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair16 & 0xFFFFu),
+                                                   __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+template <int D>
+struct Fp8State {
+  float o[D / 16][4];   // value accumulators (channels x heads)
+  float m[2];           // running max of the thread's two heads (columns 2t, 2t+1), log2 units
+  float l[2];           // this thread's share of their running sums
+};
+
+template <int D>
+__device__ __forceinline__ void reset(Fp8State<D>& st) {
+#pragma unroll
+  for (int mv = 0; mv < D / 16; ++mv)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) st.o[mv][e] = 0.0f;
+  st.m[0] = st.m[1] = -INFINITY;
+  st.l[0] = st.l[1] = 0.0f;
+}
+
+// NTILE tiles of an FP8 stage (8-bit geometry).  qtab: this thread's entries
+// of the query table, entry ks at qtab[ks * 4] = (high b0, high b1, low b0,
+// low b1) for channels 128 (ks / 8) + 32 t + 4 (ks % 8) + 0..3 of head g.
+template <int D, int NTILE>
+__device__ __forceinline__ void fp8_tiles(Fp8State<D>& st, const uint8_t* stage,
+                                          const TileOffsets<D, true>& o, int nvalid,
+                                          const uint4* __restrict__ qtab, int lane) {
+  using G = Geo<D, true>;
+  using O = TileOffsets<D, true>;
+  constexpr int kTileRows = kCW * 16;
+  float sk[NTILE][4];
+#pragma unroll
+  for (int i = 0; i < NTILE; ++i) {
+    uint32_t rg[G::KB / 4], rg8[G::KB / 4];
+    const uint8_t* base = stage + i * kTileRows * G::RB;
+#pragma unroll
+    for (int n = 0; n < O::NC * O::NQ; ++n) {
+      const uint4 u = lds<uint4>(base + o.k[0][n]), u8 = lds<uint4>(base + o.k[1][n]);
+      rg[4 * n] = u.x; rg[4 * n + 1] = u.y; rg[4 * n + 2] = u.z; rg[4 * n + 3] = u.w;
+      rg8[4 * n] = u8.x; rg8[4 * n + 1] = u8.y; rg8[4 * n + 2] = u8.z; rg8[4 * n + 3] = u8.w;
+    }
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a[4];
+      a[0] = e4m3x2_f16x2(rg[ks]);         // row g, channels +0, +1
+      a[1] = e4m3x2_f16x2(rg8[ks]);        // row g + 8
+      a[2] = e4m3x2_f16x2(rg[ks] >> 16);   // row g, channels +2, +3
+      a[3] = e4m3x2_f16x2(rg8[ks] >> 16);
+      const uint4 b = qtab[ks * 4];
+      mma16816(acc, a, b.x, b.y);
+      mma16816(acc, a, b.z, b.w);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sk[i][e] = acc[e];
+  }
+  // logits (log2 units; the query carries scale * log2 e): acc e = (row e / 2, column 2t + e % 2)
+  const uint32_t* mask = reinterpret_cast<const uint32_t*>(stage + kOffMask);
+  const int slot0 = reinterpret_cast<const StageMeta*>(stage + kOffMeta)->slot0;
+  float logit[NTILE][2][2];   // [tile][row][column]
+  bool live[NTILE][2];
+#pragma unroll
+  for (int i = 0; i < NTILE; ++i) {
+    const int s16 = slot0 + o.row[0] - tok_perm((lane >> 2)) + i * kTileRows;
+    const uint32_t mbits = mask[s16 >> 5] >> (s16 & 16);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int row = o.row[r] + i * kTileRows;
+      const bool valid = row < nvalid;
+      const bool masked = valid && ((mbits >> (row & 15)) & 1u);
+      live[i][r] = valid && !masked;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        logit[i][r][c] = !valid ? -INFINITY : (masked ? Q4KV_SENTINEL_LOGIT * kLog2e : sk[i][2 * r + c]);
+    }
+  }
+  // online softmax per column (head), lazy rescale
+  float alpha[2] = {1.0f, 1.0f};
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NTILE; ++i) mx = fmaxf(mx, fmaxf(logit[i][0][c], logit[i][1][c]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (mx > st.m[c] + kLazy) {
+      alpha[c] = ex2(st.m[c] - mx);
+      st.m[c] = mx;
+      st.l[c] *= alpha[c];
+    }
+  }
+  if (alpha[0] != 1.0f || alpha[1] != 1.0f) {
+#pragma unroll
+    for (int mv = 0; mv < D / 16; ++mv) {
+      st.o[mv][0] *= alpha[0];
+      st.o[mv][1] *= alpha[1];
+      st.o[mv][2] *= alpha[0];
+      st.o[mv][3] *= alpha[1];
+    }
+  }
+  constexpr int VW = G::VB / 4;
+#pragma unroll
+  for (int i = 0; i < NTILE; ++i) {
+    uint32_t wb[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float p[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        p[c] = logit[i][r][c] == -INFINITY ? 0.0f : ex2(logit[i][r][c] - st.m[c]);
+        st.l[c] += p[c];
+      }
+      // a remapped slot's value is 0 (its weight still counts in the sum);
+      // rows past the range may hold any bytes: selected away
+      wb[r] = live[i][r] ? h2u(__floats2half2_rn(p[0], p[1])) : 0u;
+    }
+    const uint32_t bw0 = movtrans(wb[0]), bw1 = movtrans(wb[1]);
+    uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
+    const uint8_t* vc = stage + kOffV + i * kTileRows * G::RB;
+#pragma unroll
+    for (int q = 0; q < VW; q += 4) {
+      const uint4 a0 = lds<uint4>(vc + o.v[0] + 4 * q), a1 = lds<uint4>(vc + o.v[1] + 4 * q);
+      const uint4 a8 = lds<uint4>(vc + o.v[2] + 4 * q), a9 = lds<uint4>(vc + o.v[3] + 4 * q);
+      v0[q] = a0.x; v0[q + 1] = a0.y; v0[q + 2] = a0.z; v0[q + 3] = a0.w;
+      v1[q] = a1.x; v1[q + 1] = a1.y; v1[q + 2] = a1.z; v1[q + 3] = a1.w;
+      v8[q] = a8.x; v8[q + 1] = a8.y; v8[q + 2] = a8.z; v8[q + 3] = a8.w;
+      v9[q] = a9.x; v9[q + 1] = a9.y; v9[q + 2] = a9.z; v9[q + 3] = a9.w;
+    }
+#pragma unroll
+    for (int mv = 0; mv < D / 16; ++mv) {
+      // byte 2 mv of the thread's run = channel cb + 2 mv, byte 2 mv + 1 = cb + 2 mv + 1
+      const int wi = (2 * mv) / 4, bp = (2 * mv) % 4;
+      const uint32_t sa = bp | ((bp + 4) << 4), sb = (bp + 1) | ((bp + 5) << 4);   // [T0.b, T1.b]
+      uint32_t a[4];
+      a[0] = e4m3x2_f16x2(__byte_perm(v0[wi], v1[wi], sa));
+      a[1] = e4m3x2_f16x2(__byte_perm(v0[wi], v1[wi], sb));
+      a[2] = e4m3x2_f16x2(__byte_perm(v8[wi], v9[wi], sa));
+      a[3] = e4m3x2_f16x2(__byte_perm(v8[wi], v9[wi], sb));
+      mma16816(st.o[mv], a, bw0, bw1);
+    }
+  }
+}
+
 // Raw 16-bit query elements E*lane .. E*lane + E-1 of head `h` of item's
 // (sequence, KV head) group, as loaded (E = 4: 8 bytes, E = 8: 16 bytes).
 template <int E>
@@ -475,7 +628,7 @@ __device__ __forceinline__ uint4 load_query(const DecodeArgs& a, int item, int S
   return *reinterpret_cast<const uint4*>(p);
 }
 
-template <int D, int NT>
+template <int D, int NT, bool FP8 = false>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     decode_tc_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ TileMaps maps,
                      int n_items) {
@@ -564,14 +717,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           const uint8_t* vpp = reinterpret_cast<const uint8_t*>(is8 ? P.v_params8 : P.v_params4) + row * pb;
           // codes: one TS-row box per tensor (the box never leaves the block)
           const int ts = is8 ? Geo<D, true>::TS : Geo<D, false>::TS;
-          const uint32_t cb = static_cast<uint32_t>(ts) * rb, prb = rows * pb;
+          const uint32_t cb = static_cast<uint32_t>(ts) * rb, prb = FP8 ? 0u : rows * pb;   // FP8: no params
           mbar_arrive_tx(&full[s], 2 * cb + 2 * prb + 32);
           tma_rows(stg, is8 ? &maps.k8 : &maps.k4, static_cast<int>(row), &full[s]);
           tma_rows(stg + kOffV, is8 ? &maps.v8 : &maps.v4, static_cast<int>(row), &full[s]);
           (void)kc;
           (void)vc;
-          bulk_g2s(stg + kOffKP, kpp, prb, &full[s]);
-          bulk_g2s(stg + kOffVP, vpp, prb, &full[s]);
+          if (!FP8) {
+            bulk_g2s(stg + kOffKP, kpp, prb, &full[s]);
+            bulk_g2s(stg + kOffVP, vpp, prb, &full[s]);
+          }
           bulk_g2s(stg + kOffMask, P.mask + static_cast<int64_t>(meta.blk) * kMaskWords, 32, &full[s]);
         } else {
           mbar_arrive(&full[s]);
@@ -600,6 +755,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   bool dead = false;
   TileOffsets<D, false> off4;
   off4.init(warp, lane);
+  // FP8: query table [head][ks][t] of (high b0, high b1, low b0, low b1);
+  // heads past G stay zero
+  Fp8State<D> fst;
+  TileOffsets<D, true> off8f;
+  uint4* qtab = reinterpret_cast<uint4*>(qrot);
+  const uint4* qtab_t = qtab + g * (D / 16) * 4 + t;
+  if constexpr (FP8) {
+    off8f.init(warp, lane);
+    for (int i = threadIdx.x; i < 8 * (D / 16) * 4; i += kCW * 32) qtab[i] = make_uint4(0u, 0u, 0u, 0u);
+    consumer_sync();
+  }
 
   uint4 qraw = make_uint4(0u, 0u, 0u, 0u);   // raw query of the warp's head for the coming item
   if (warp < G && blockIdx.x < n_items) qraw = load_query<D / 32>(a, blockIdx.x, S, hkv, hq, G, warp, lane);
@@ -623,6 +789,26 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         x[e] = a.q_dtype == Q4KV_F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(h16)))
                                      : __uint_as_float(h16 << 16);
       }
+      if constexpr (FP8) {
+        // q * scale * log2 e as fp16 high + low parts, in the B layout of the
+        // key MMA: entry (head, ks, t) covers channels 128 (ks / 8) + 32 t + 4 (ks % 8) + 0..3
+        uint32_t hw[E / 2], lw[E / 2];
+#pragma unroll
+        for (int p2 = 0; p2 < E / 2; ++p2) {
+          const float y0 = x[2 * p2] * sc2, y1 = x[2 * p2 + 1] * sc2;
+          const __half2 hi = __floats2half2_rn(y0, y1);
+          const float2 hf = __half22float2(hi);
+          hw[p2] = h2u(hi);
+          lw[p2] = h2u(__floats2half2_rn(y0 - hf.x, y1 - hf.y));
+        }
+        if constexpr (E == 4) {   // channels 4 lane + 0..3: ks = lane % 8, t = lane / 8
+          qtab[(warp * (D / 16) + (lane & 7)) * 4 + (lane >> 3)] = make_uint4(hw[0], hw[1], lw[0], lw[1]);
+        } else {                  // channels 8 lane + 0..7: two entries
+          const int ks0 = 8 * (lane >> 4) + 2 * (lane & 3), tt = (lane & 15) >> 2;
+          qtab[(warp * (D / 16) + ks0) * 4 + tt] = make_uint4(hw[0], hw[1], lw[0], lw[1]);
+          qtab[(warp * (D / 16) + ks0 + 1) * 4 + tt] = make_uint4(hw[2], hw[3], lw[2], lw[3]);
+        }
+      } else {
       if (P.k_rotated) {   // c * H q: butterflies inside the lane, then across lanes (fp32)
 #pragma unroll
         for (int h = 1; h < E; h <<= 1)
@@ -692,10 +878,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int off = 1; off < kGroup / E; off <<= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
       if (lane % (kGroup / E) == 0) qsum[warp * 4 + lane / (kGroup / E)] = part;
       if (lane == 0) qsum[32 + warp] = ldexpf(1.0f, -ex);        // 2^-E of head `warp`
+      }
     }
     consumer_sync();
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
+    for (int j = 0; j < (FP8 ? 0 : NT); ++j) {
       const int col = 8 * j + g;                // this thread's B column
       const int h = col / NG, gr = col % NG;
       const uint4* tbl = reinterpret_cast<const uint4*>(qrot) + (h < G ? h : 0) * (D / 32) * 4 + t;
@@ -722,7 +909,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       }
     }
-    reset(st);
+    if constexpr (FP8) reset(fst);
+    else reset(st);
     bool poison = false, timeout = false;
 
     // ---- the item's stages ----
@@ -736,7 +924,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       poison |= meta.poison;
       if (!dead && !meta.timeout && meta.blk >= 0 && warp * 16 < meta.ntok) {
         // warp w takes the stage's tiles w, w + 8, ... (rows past ntok are masked)
-        if (!meta.is8) {
+        if constexpr (FP8) {
+          constexpr int NTL = Geo<D, true>::MTILES >= kCW ? Geo<D, true>::MTILES / kCW : 1;
+          if (warp < Geo<D, true>::MTILES) fp8_tiles<D, NTL>(fst, stg, off8f, meta.ntok, qtab_t, lane);
+        } else if (!meta.is8) {
           constexpr int NTL = Geo<D, false>::MTILES / kCW;
           tiles<D, NT, false, NTL>(st, stg, off4, meta.ntok, bq, qs, ks, lane);
         } else if (warp < Geo<D, true>::MTILES) {
@@ -754,8 +945,31 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if (timeout && threadIdx.x == 0) raise_error(P.error_word, Q4KV_DEVERR_TIMEOUT);
 
     // ---- cross-warp merge of the item ----
+    if constexpr (FP8) {
+      float lt[2] = {fst.l[0], fst.l[1]};
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
+      for (int off = 4; off < 32; off <<= 1) {
+        lt[0] += __shfl_xor_sync(0xffffffffu, lt[0], off);
+        lt[1] += __shfl_xor_sync(0xffffffffu, lt[1], off);
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int h = 2 * t + c;
+        if (g == 0 && h < G) {
+          mrg_ml[(warp * 8 + h) * 2] = fst.m[c];
+          mrg_ml[(warp * 8 + h) * 2 + 1] = lt[c];
+        }
+      }
+#pragma unroll
+      for (int mv = 0; mv < D / 16; ++mv)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int ch = (D / 8) * g + 2 * mv + (e >> 1), h = 2 * t + (e & 1);
+          if (h < G) mrg_o[(warp * G + h) * D + ch] = fst.o[mv][e];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < (FP8 ? 0 : NT); ++j) {
       float lt = st.l[j], z0 = st.z[j][0], z1 = st.z[j][1];
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -884,18 +1098,20 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
     return cudaErrorInvalidValue;
 
   cudaError_t e = cudaSuccess;
-#define Q4KV_TC(DD, NN)                                                                           \
-  do {                                                                                            \
-    e = cudaFuncSetAttribute(decode_tc_kernel<DD, NN>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             static_cast<int>(smem));                                             \
-    if (e == cudaSuccess)                                                                         \
-      e = launch_pdl(decode_tc_kernel<DD, NN>, dim3(grid), dim3(kThreadsTC), smem, stream, a, maps, \
-                     n_items);                                                                    \
+#define Q4KV_TC(DD, NN, F8)                                                                        \
+  do {                                                                                             \
+    e = cudaFuncSetAttribute(decode_tc_kernel<DD, NN, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(smem));                                              \
+    if (e == cudaSuccess)                                                                          \
+      e = launch_pdl(decode_tc_kernel<DD, NN, F8>, dim3(grid), dim3(kThreadsTC), smem, stream, a, maps, \
+                     n_items);                                                                     \
   } while (0)
-  if (p.head_dim == 128 && nt == 1) Q4KV_TC(128, 1);
-  else if (p.head_dim == 128) Q4KV_TC(128, 2);
-  else if (nt == 1) Q4KV_TC(256, 1);
-  else Q4KV_TC(256, 2);
+  if (a.pool.fp8 && p.head_dim == 128) Q4KV_TC(128, 1, true);   // FP8 comparison cache: heads are the columns
+  else if (a.pool.fp8) Q4KV_TC(256, 1, true);
+  else if (p.head_dim == 128 && nt == 1) Q4KV_TC(128, 1, false);
+  else if (p.head_dim == 128) Q4KV_TC(128, 2, false);
+  else if (nt == 1) Q4KV_TC(256, 1, false);
+  else Q4KV_TC(256, 2, false);
 #undef Q4KV_TC
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -4,6 +4,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,6 +23,7 @@ struct PoolView {
   int32_t k_rotated;
   int32_t n_q4;
   int32_t n_q8;
+  int32_t fp8;        // Q4KV_FORMAT_FP8: every block holds OCP E4M3 bytes, no params
   uint8_t* k_codes4;
   uint8_t* v_codes4;
   __half2* k_params4;
@@ -41,6 +43,7 @@ inline PoolView view_of(const q4kv_pool& p) {
   v.k_rotated = p.k_rotated;
   v.n_q4 = p.n_q4_blocks;
   v.n_q8 = p.n_q8_blocks;
+  v.fp8 = p.value_format == Q4KV_FORMAT_FP8;
   v.k_codes4 = p.k_codes4;
   v.v_codes4 = p.v_codes4;
   v.k_params4 = reinterpret_cast<__half2*>(p.k_params4);

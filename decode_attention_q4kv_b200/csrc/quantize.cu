@@ -275,6 +275,22 @@ __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupPar
   if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(g.sh, g.zh);
 }
 
+// FP8 comparison cache: the lane's 16 values as OCP E4M3 bytes (round to
+// nearest even, saturated to +-448), channel order, one 16-byte store.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {   // lo -> low byte
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ void store_fp8(const float2 (&x)[8], uint8_t* __restrict__ dst) {
+  // pair p holds channels p (.x) and p + 8 (.y)
+  uint4 w;
+  w.x = e4m3x2(x[0].x, x[1].x) | e4m3x2(x[2].x, x[3].x) << 16;
+  w.y = e4m3x2(x[4].x, x[5].x) | e4m3x2(x[6].x, x[7].x) << 16;
+  w.z = e4m3x2(x[0].y, x[1].y) | e4m3x2(x[2].y, x[3].y) << 16;
+  w.w = e4m3x2(x[4].y, x[5].y) | e4m3x2(x[6].y, x[7].y) << 16;
+  *reinterpret_cast<uint4*>(dst) = w;
+}
+
 // K (already rotated when the pool stores rotated keys; its values are the
 // rotated ones divided by ks) and V of one warp item.
 template <int BITS>
@@ -321,7 +337,7 @@ struct EncodeGeometry {
   int32_t items_per_head_log2;   // log2(T / VPW)
 };
 
-template <int D, typename InT, bool ROT, bool MIXED>
+template <int D, typename InT, bool ROT, bool MIXED, bool FP8 = false>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_kernel(const __grid_constant__ PoolView pool, const InT* __restrict__ k,
                     const InT* __restrict__ v, const __grid_constant__ EncodeGeometry geo,
@@ -445,14 +461,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
         float2 xk[8], xv[8];
         unpack16<InT>(k0, k1, xk);
         unpack16<InT>(v0, v1, xv);
-        if (ROT) rotate_pairs<D>(xk, j);   // keys are coded rotated, values as they are
-        constexpr float ks = ROT ? kRotScale<D> : 1.0f;
-        if (is8)
-          encode_kv<8>(xk, ks, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
-                       pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
-        else
-          encode_kv<4>(xk, ks, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
-                       pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+        if constexpr (FP8) {
+          if (valid) {
+            store_fp8(xk, pool.k_codes8 + row * D + j * kEPL);
+            store_fp8(xv, pool.v_codes8 + row * D + j * kEPL);
+          }
+        } else {
+          if (ROT) rotate_pairs<D>(xk, j);   // keys are coded rotated, values as they are
+          constexpr float ks = ROT ? kRotScale<D> : 1.0f;
+          if (is8)
+            encode_kv<8>(xk, ks, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
+                         pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+          else
+            encode_kv<4>(xk, ks, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
+                         pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
+        }
         // freshly written slots are live: one word update for the item's tokens
         const uint32_t tf = t0 + ti;
         if (h == 0 && lane == 0 && tf < geo.n_tokens) {
@@ -530,6 +553,15 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ Poo
     float2 xk[8], xv[8];
     unpack16<InT>(k0, k1, xk);
     unpack16<InT>(v0, v1, xv);
+    if (pool.fp8) {   // FP8 comparison cache
+      if (valid) {
+        store_fp8(xk, pool.k_codes8 + row * D + j * kEPL);
+        store_fp8(xv, pool.v_codes8 + row * D + j * kEPL);
+      }
+      if (lane == 0 && hg == 0)
+        atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + slot / 32, ~(1u << (slot % 32)));
+      continue;
+    }
     if (ROT) rotate_pairs<D>(xk, j);
     constexpr float ks = ROT ? kRotScale<D> : 1.0f;
     if (is8)
@@ -609,6 +641,20 @@ __device__ __forceinline__ void decode_lane(const uint8_t* __restrict__ codes,
   }
 }
 
+// The lane's 16 E4M3 bytes as binary32 (every E4M3 value is exact in fp16).
+__device__ __forceinline__ void decode_fp8_lane(const uint8_t* __restrict__ codes, int j, float (&x)[kEPL]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(codes + j * kEPL);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+        static_cast<__nv_fp8x2_storage_t>(w[i / 2] >> (16 * (i % 2))), __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
 template <typename OutT>
 __device__ __forceinline__ void store16(OutT* dst, const float (&x)[kEPL]);
 template <>
@@ -668,7 +714,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
     const bool masked =
         (pool.mask[static_cast<int64_t>(blk) * kMaskWords + slot / 32] >> (slot % 32)) & 1u;
 
-    if (is8)
+    if (pool.fp8)
+      decode_fp8_lane(pool.k_codes8 + row * D, j, x);
+    else if (is8)
       decode_lane<8>(pool.k_codes8 + row * D, pool.k_params8 + row * S::NG, j, x);
     else
       decode_lane<4>(pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG, j, x);
@@ -679,7 +727,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
     }
     store16<OutT>(kd, x);
 
-    if (is8)
+    if (pool.fp8)
+      decode_fp8_lane(pool.v_codes8 + row * D, j, x);
+    else if (is8)
       decode_lane<8>(pool.v_codes8 + row * D, pool.v_params8 + row * S::NG, j, x);
     else
       decode_lane<4>(pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG, j, x);
@@ -726,12 +776,12 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
   const int64_t grid = n_chunks < sms ? n_chunks : sms;
   const size_t smem = kQStages * kQStageBytes + 2 * kQStages * sizeof(uint64_t);
   cudaError_t e = cudaSuccess;
-#define Q4KV_LAUNCH_Q(DD, T, R, M)                                                                   \
+#define Q4KV_LAUNCH_Q(DD, T, R, M, ...)                                                              \
   do {                                                                                                 \
-    e = cudaFuncSetAttribute(quantize_kernel<DD, T, R, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(quantize_kernel<DD, T, R, M, ##__VA_ARGS__>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(smem));                                                  \
     if (e == cudaSuccess)                                                                              \
-      e = launch_pdl(quantize_kernel<DD, T, R, M>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),  \
+      e = launch_pdl(quantize_kernel<DD, T, R, M, ##__VA_ARGS__>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),  \
                      smem, stream, pool, static_cast<const T*>(k), static_cast<const T*>(v), geo,        \
                      block_ids);                                                                       \
   } while (0)
@@ -744,6 +794,13 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
     else Q4KV_LAUNCH_Q(DD, T, false, false);                              \
   } while (0)
   if (n_chunks == 0) return cudaSuccess;
+  if (pool.fp8) {   // FP8 pools: raw keys, every block 8-bit
+    if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(128, __half, false, true, true);
+    else if (d == 128) Q4KV_LAUNCH_Q(128, __nv_bfloat16, false, true, true);
+    else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_Q(256, __half, false, true, true);
+    else Q4KV_LAUNCH_Q(256, __nv_bfloat16, false, true, true);
+    return e;
+  }
   if (d == 128 && in_dtype == Q4KV_F16) Q4KV_LAUNCH_QR(128, __half);
   else if (d == 128) Q4KV_LAUNCH_QR(128, __nv_bfloat16);
   else if (in_dtype == Q4KV_F16) Q4KV_LAUNCH_QR(256, __half);

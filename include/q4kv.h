@@ -68,7 +68,7 @@
 extern "C" {
 #endif
 
-#define Q4KV_ABI_VERSION 1
+#define Q4KV_ABI_VERSION 2
 #define Q4KV_BLOCK_TOKENS 256
 #define Q4KV_GROUP 64
 #define Q4KV_MASK_WORDS 8            /* uint32 words of remap mask per block */
@@ -92,6 +92,25 @@ typedef enum {
 typedef enum { Q4KV_F16 = 0, Q4KV_BF16 = 1, Q4KV_F32 = 2 } q4kv_dtype;
 
 /*
+ * Value formats of a pool (q4kv_pool.value_format).
+ *   Q4KV_FORMAT_INT  4-bit (and optional 8-bit) integer codes with a scale and
+ *                    a zero per group of 64, as described above.
+ *   Q4KV_FORMAT_FP8  the FP8 cache the 4-bit cache is compared against ([UQ]
+ *                    "技術/ビジネス面": TTFT and throughput are reported against
+ *                    an FP8 KV cache).  Every value is one OCP E4M3 byte
+ *                    (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ *                    no infinities; largest finite 448) holding the input value
+ *                    rounded to nearest, ties to even, saturated to +-448; no
+ *                    scale and no rotation.  Such a pool has n_q4_blocks = 0 and
+ *                    k_rotated = 0, keeps its codes in k_codes8 / v_codes8
+ *                    [n_q8][Hkv][256][D], and has no params (their pointers are
+ *                    ignored).  Quantise, append, dequantise, invalidate and
+ *                    decode all accept it.
+ */
+#define Q4KV_FORMAT_INT 0
+#define Q4KV_FORMAT_FP8 1
+
+/*
  * The paged pool ([AMBP] sec. 2.1 items 1-2; 8-bit blocks: [QKVS]).
  * Unified block ids: [0, n_q4_blocks) are 4-bit blocks, stored at index id
  * of the *4 arrays; [n_q4_blocks, n_q4_blocks + n_q8_blocks) are 8-bit blocks,
@@ -113,7 +132,7 @@ typedef struct {
   int32_t k_rotated;    /* 1 = K stored Walsh-Hadamard rotated ([UQ]); 0 = raw */
   int32_t n_q4_blocks;  /* >= 0 */
   int32_t n_q8_blocks;  /* >= 0 */
-  int32_t reserved;     /* must be 0 */
+  int32_t value_format; /* Q4KV_FORMAT_INT (0) or Q4KV_FORMAT_FP8 (1) */
   uint8_t *k_codes4, *v_codes4;
   void *k_params4, *v_params4;
   uint8_t *k_codes8, *v_codes8;

@@ -20,7 +20,8 @@ What it computes, step by step, and where each step comes from:
           prefilled again.  Section 2.2: GQA models.
   [UQ]    UltraQuant news item (poko-everyday.com, arXiv 2606.20474),
           section "technology / business": a Walsh-Hadamard rotation before
-          4-bit quantisation, with keys and values treated asymmetrically.
+          4-bit quantisation, with keys and values treated asymmetrically;
+          the 4-bit cache is measured against an FP8 KV cache.
   [IKV]   IntentKV article (Qiita), section "invalidate instead of
           compacting": an evicted slot is re-pointed to a sentinel slot
           whose key is -1e4, so its softmax weight collapses to zero while
@@ -46,7 +47,11 @@ design notes):
   * an evicted slot's *logit* is -1e4 and its value is 0; its stored bytes
     stay where they are; one 256-bit mask per physical block, shared by
     all KV heads; writing a token into a slot makes the slot live again;
-  * 8-bit blocks use the same steps with 255 levels, one code per byte.
+  * 8-bit blocks use the same steps with 255 levels, one code per byte;
+  * the FP8 comparison cache stores each raw value as one OCP E4M3 byte
+    (bias 7, 3 mantissa bits, no infinities, largest finite 448), rounded
+    to nearest with ties to even and saturated to +-448; no scale, no
+    rotation (the plainest FP8 KV cache).
 
 Precision: the encoding steps (rotation, min/max, scale/zero, codes,
 dequantisation) are binary32/binary16 by definition, so they are written
@@ -201,6 +206,45 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# FP8 E4M3 values of the comparison cache [UQ]
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """OCP E4M3 bytes of finite values x: round to nearest, ties to even, on
+    the E4M3 grid (spacing 2^(e-3) for |x| in [2^e, 2^(e+1)), e >= -6, and
+    2^-9 below 2^-6), then saturate to +-448."""
+    x = np.asarray(x, dtype=np.float32)
+    a = np.abs(x.astype(np.float64))
+    sign = np.signbit(x).astype(np.uint8) << np.uint8(7)
+    a = np.minimum(a, E4M3_MAX)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    quantum = np.exp2(e - 3.0)
+    r = np.minimum(np.rint(a / quantum) * quantum, E4M3_MAX)   # a / quantum is exact in fp64
+    with np.errstate(divide="ignore"):
+        er = np.floor(np.log2(np.where(r > 0, r, 1.0)))
+    normal = r >= 2.0 ** -6
+    exp_field = np.where(normal, er + 7.0, 0.0)
+    mant = np.where(normal, r / np.exp2(er) - 1.0, r / 2.0 ** -9 / 8.0) * 8.0
+    bits = (exp_field.astype(np.uint8) << np.uint8(3)) | np.rint(mant).astype(np.uint8)
+    return (bits | sign).astype(np.uint8)
+
+
+def e4m3_decode(b: np.ndarray) -> np.ndarray:
+    """binary32 value of OCP E4M3 bytes (every one is exact in binary32)."""
+    b = np.asarray(b, dtype=np.uint8).astype(np.int32)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    ef = (b >> 3) & 0xF
+    mf = b & 0x7
+    val = np.where(ef == 0, mf * 2.0 ** -9, (1.0 + mf / 8.0) * np.exp2(ef - 7.0))
+    return (sign * val).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
 # the paged pool [AMBP 2.1 items 1-2], eviction mask [IKV]
 # ---------------------------------------------------------------------------
 
@@ -215,7 +259,10 @@ class OraclePool:
     """
 
     def __init__(self, n_kv_heads: int, head_dim: int, n_q4: int, n_q8: int = 0,
-                 k_rotated: bool = True):
+                 k_rotated: bool = True, fp8: bool = False):
+        if fp8 and (n_q4 or k_rotated):
+            raise ValueError("an FP8 pool has only 8-bit blocks and raw keys")
+        self.fp8 = fp8
         self.hkv = n_kv_heads
         self.d = head_dim
         self.n_q4 = n_q4
@@ -258,6 +305,9 @@ class OraclePool:
             if self.k_rotated:
                 kk = rotate_f32(kk)
             for name, x in (("k", kk), ("v", vf[t0:t1])):
+                if self.fp8:
+                    self.codes8[name][blk, :, : t1 - t0] = e4m3_encode(x).transpose(1, 0, 2)
+                    continue
                 codes, s_h, z_h = quantize_groups(x, bits)       # [cnt][Hkv][D]
                 codes = codes.transpose(1, 0, 2)                  # [Hkv][cnt][D]
                 par = np.stack([s_h, z_h], axis=-1).transpose(1, 0, 2, 3)
@@ -293,6 +343,9 @@ class OraclePool:
                 if self.k_rotated:
                     kk = rotate_f32(kk)
                 for name, x in (("k", kk), ("v", vf[b, i][None])):
+                    if self.fp8:
+                        self.codes8[name][blk, :, slot] = e4m3_encode(x[0])
+                        continue
                     codes, s_h, z_h = quantize_groups(x, bits)
                     par = np.stack([s_h[0], z_h[0]], axis=-1)  # [Hkv][D/64][2]
                     if bits == 4:
@@ -338,6 +391,10 @@ class OraclePool:
         """
         out = []
         for name in "kv":
+            if self.fp8:
+                self.bits(blk)
+                out.append(e4m3_decode(self.codes8[name][blk]))
+                continue
             codes, s_h, z_h = self.codes_params(blk, name)
             x = dequantize_groups(codes, s_h, z_h)
             if name == "k" and unrotate_k and self.k_rotated:

@@ -12,7 +12,7 @@ FAKE = 0x7F0000000000     # 4 KiB-aligned address never dereferenced: every call
 
 
 def _pool(**kw):
-    d = dict(head_dim=128, n_kv_heads=8, k_rotated=1, n_q4_blocks=4, n_q8_blocks=0, reserved=0,
+    d = dict(head_dim=128, n_kv_heads=8, k_rotated=1, n_q4_blocks=4, n_q8_blocks=0, value_format=0,
              k_codes4=FAKE, v_codes4=FAKE, k_params4=FAKE, v_params4=FAKE,
              k_codes8=0, v_codes8=0, k_params8=0, v_params8=0, remap_mask=FAKE, error_word=0)
     d.update(kw)
@@ -32,7 +32,7 @@ def test_exports_every_declared_function():
 
 
 def test_abi_version_and_status_strings():
-    assert L.q4kv_abi_version() == 1
+    assert L.q4kv_abi_version() == 2
     assert L.q4kv_status_string(0) == b"ok"
     assert b"workspace" in L.q4kv_status_string(_lib.ERR_WORKSPACE)
     assert L.q4kv_status_string(99) == b"unknown status"
@@ -105,7 +105,7 @@ def test_quantize_rejects_bad_arguments_without_launching():
     assert q(ctypes.byref(p), FAKE, FAKE, 0, 10, 1028, FAKE, None) == _lib.ERR_INVALID_ARG       # stride not 16 B
     assert q(ctypes.byref(p), FAKE, FAKE, 0, -1, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
     assert q(ctypes.byref(p), FAKE, FAKE, 0, 10, 1024, None, None) == _lib.ERR_INVALID_ARG       # no block ids
-    assert q(ctypes.byref(_pool(reserved=1)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert q(ctypes.byref(_pool(value_format=2)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
     assert q(ctypes.byref(_pool(k_codes4=0)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
     assert q(ctypes.byref(_pool(n_q8_blocks=2)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG
     assert q(ctypes.byref(_pool(remap_mask=FAKE + 4)), FAKE, FAKE, 0, 10, 1024, FAKE, None) == _lib.ERR_INVALID_ARG

@@ -477,3 +477,48 @@ def test_append_equals_bulk_encoding_of_whole_sequences():
         np.testing.assert_array_equal(grown.codes4[name], ref.codes4[name])
         np.testing.assert_array_equal(grown.params4[name].view(np.uint16), ref.params4[name].view(np.uint16))
     np.testing.assert_array_equal(grown.mask, ref.mask)
+
+
+# ---------------------------------------------------------------------------
+# FP8 (OCP E4M3) comparison cache
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("x,byte", [
+    (1.0, 0x38), (-1.0, 0xB8), (448.0, 0x7E), (-448.0, 0xFE), (500.0, 0x7E), (464.0, 0x7E),
+    (2.0 ** -6, 0x08), (2.0 ** -9, 0x01), (0.0, 0x00), (-0.0, 0x80),
+    (1.0625, 0x38),           # halfway between 1 and 1.125: ties to the even mantissa (1)
+    (1.1875, 0x3A),           # halfway between 1.125 and 1.25: ties to 1.25
+    (1.5 * 2.0 ** -9, 0x02),  # subnormal tie goes to the even count (2)
+    (2.0 ** -10, 0x00),       # half the smallest subnormal rounds to +0
+    (240.0, 0x77), (0.1, 0x1D)])
+def test_e4m3_encoding_closed_forms(x, byte):
+    # OCP E4M3: value = (1 + m/8) 2^(e - 7) for e in 1..15 (m = 7 with e = 15
+    # is NaN, so the largest finite is 1.75 * 2^8 = 448), m/8 * 2^-6 for e = 0
+    assert int(O.e4m3_encode(np.array([x], np.float32))[0]) == byte
+
+
+def test_e4m3_round_trip_and_library_agreement():
+    every = np.array([b for b in range(256) if b not in (0x7F, 0xFF)], np.uint8)   # all but NaN
+    np.testing.assert_array_equal(O.e4m3_encode(O.e4m3_decode(every)), every)
+    # torch's float8_e4m3fn conversion rounds to nearest even inside the range
+    import torch
+    x = np.clip(np.random.default_rng(5).standard_normal(100000) * 60, -448, 448).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.e4m3_encode(x), ref)
+
+
+def test_fp8_pool_attention_matches_brute_force():
+    rng = np.random.default_rng(9)
+    hkv, hq, d, n = 1, 4, 128, 300
+    k = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    v = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    pool = O.OraclePool(hkv, d, 0, 2, k_rotated=False, fp8=True)
+    pool.quantize_blocks(k, v, "fp16", [1, 0])
+    q = rng.standard_normal((1, hq, d)).astype(np.float16)
+    out = O.decode_attention(pool, q, "fp16", np.array([[1, 0]]), [n])
+    kd = O.e4m3_decode(O.e4m3_encode(k.astype(np.float32)))[:, 0].astype(np.float64)
+    vd = O.e4m3_decode(O.e4m3_encode(v.astype(np.float32)))[:, 0].astype(np.float64)
+    for h in range(hq):
+        s = kd @ q[0, h].astype(np.float64) / math.sqrt(d)
+        p = scipy.special.softmax(s)
+        np.testing.assert_allclose(out[0, h], p @ vd, rtol=1e-12, atol=1e-12)
