@@ -49,7 +49,7 @@ def workload_by_name(name):
     return W.WORKLOADS[name]
 
 
-def bytes_per_layer(w):
+def bytes_per_layer(w, fp8=False):
     """Algorithmic HBM bytes of one layer: (quantise, decode)."""
     in_elem = 2
     vec = w.head_dim
@@ -61,8 +61,10 @@ def bytes_per_layer(w):
     n_blocks = w.n_blocks
     frac8 = n_q8 / n_blocks if n_blocks else 0.0
     row = (1 - frac8) * q4_row + frac8 * q8_row
+    if fp8:                              # the FP8 comparison cache: one byte per value, no params
+        row = vec
     quant = n_tok * w.n_kv_heads * (2 * vec * in_elem + 2 * row)
-    if w.q8_fraction:
+    if w.q8_fraction and not fp8:
         quant += n_tok * w.n_kv_heads * vec * in_elem        # mean |K| pass reads K once more
     dec_tok = w.batch * w.ctx
     decode = dec_tok * w.n_kv_heads * 2 * row + n_blocks * 32 + w.batch * w.blocks_per_seq * 4
@@ -136,7 +138,7 @@ class ClockSampler:
 class Job:
     """All layers of one workload resident on one GPU, ready to step."""
 
-    def __init__(self, w, device, rank=0, layers=None):
+    def __init__(self, w, device, rank=0, layers=None, fp8=False):
         import torch
 
         import decode_attention_q4kv_b200 as q4
@@ -151,14 +153,16 @@ class Job:
         self.n_layers = len(layer_ids)
         n_tok = w.prefill_tokens or w.n_tokens
         n_pool = max(w.n_blocks, n_tok // 256) if w.permuted_pool else w.n_blocks
-        self.n_q8 = w.n_q8_blocks
+        self.fp8 = fp8
+        self.n_q8 = n_pool if fp8 else w.n_q8_blocks
         self.n_q4 = n_pool - self.n_q8
         self.layers = []
         for l in layer_ids:
             lid = rank_layer_id(l, rank)
             k, v = W.kv_tokens(w, lid, n_tok, device)
             q = W.query(w, lid, device)
-            pool = q4.Q4KVPool(w.n_kv_heads, w.head_dim, self.n_q4, self.n_q8, device=device)
+            pool = q4.Q4KVPool(w.n_kv_heads, w.head_dim, self.n_q4, self.n_q8, k_rotated=not fp8,
+                               device=device, fp8=fp8)
             self.layers.append(dict(k=k, v=v, q=q, pool=pool,
                                     out=torch.empty((w.batch, w.n_q_heads, w.head_dim),
                                                     dtype=torch.float16, device=device)))
@@ -178,15 +182,16 @@ class Job:
             for L in self.layers:
                 L["pool"].quantize(L["k"], L["v"], self.prefill_ids)
                 self._tile(L["pool"], n_tok // 256)
-        self.quant_bytes, self.decode_bytes = bytes_per_layer(w)
+        self.quant_bytes, self.decode_bytes = bytes_per_layer(w, fp8)
         self.launches_per_layer = 1 + 1 + (1 if self.plan.n_splits > 1 else 0)
-        if w.q8_fraction:
+        if w.q8_fraction and not fp8:
             self.launches_per_layer += 3
         if self.evict is not None:
             self.launches_per_layer += 1
 
     def _tile(self, pool, n_src):
-        for name in ("k_codes4", "v_codes4", "k_params4", "v_params4"):
+        names = ("k_codes8", "v_codes8") if self.fp8 else ("k_codes4", "v_codes4", "k_params4", "v_params4")
+        for name in names:
             t = getattr(pool, name)
             for s in range(n_src, t.shape[0], n_src):
                 e = min(s + n_src, t.shape[0])
@@ -194,7 +199,7 @@ class Job:
 
     def quantize_layer(self, L):
         w, q4 = self.w, self.q4
-        if w.q8_fraction:
+        if w.q8_fraction and not self.fp8:
             am = q4.block_absmean(L["k"])
             ids = q4.mixed_block_ids(am, self.n_q8, 0, self.n_q4)
             L["ids"] = ids
@@ -329,7 +334,7 @@ def run_gpu(args):
                                 device_id=dev)
 
     w = workload_by_name(args.workload)
-    job = Job(w, dev, rank, args.layers)
+    job = Job(w, dev, rank, args.layers, fp8=args.fp8)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -416,8 +421,9 @@ def run_gpu(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "layers": job.n_layers, "batch": w.batch, "ctx": w.ctx,
                        "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
-                       "input_dtype": w.dtype, "storage": "int4 codes, group 64, fp16 scale+zero, 256-token blocks",
-                       "q8_fraction": w.q8_fraction, "evict_fraction": w.evict_fraction,
+                       "input_dtype": w.dtype, "storage": ("fp8 e4m3 codes (the comparison cache), no scale, 256-token blocks" if args.fp8 else
+                                   "int4 codes, group 64, fp16 scale+zero, 256-token blocks"),
+                       "q8_fraction": 0.0 if args.fp8 else w.q8_fraction, "evict_fraction": w.evict_fraction,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "decode_splits": job.plan.n_splits,
                        "l2": "step inputs larger than L2 (%.1f GB)" % (job.bytes_per_step / 1e9)},
@@ -440,7 +446,7 @@ def run_gpu(args):
         }
         if e2e is not None:
             line["e2e"] = e2e
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not args.fp8:   # the oracle leg times the Q4 path
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -600,6 +606,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="q4kv", choices=["q4kv", "reference"])
     ap.add_argument("--workload", default="gemma")
+    ap.add_argument("--fp8", action="store_true",
+                    help="run the same workload on the FP8 (E4M3) comparison cache instead of Q4")
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

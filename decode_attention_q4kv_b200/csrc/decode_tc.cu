@@ -79,7 +79,7 @@ struct StageMeta {
   uint8_t is8;
   uint8_t last;     // last stage of its work item
   uint8_t poison;   // the item touched a bad block id or a bad length
-  uint8_t timeout;  // the producer gave up waiting
+  uint8_t pad;
 };
 
 // ---------------------------------------------------------------------------
@@ -679,12 +679,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       int tok = t0;
       do {
         const int s = it % kNS;
-        if (!gave_up && !mbar_wait(&empty[s], ((it / kNS) & 1) ^ 1)) gave_up = true;
+        // A stage that stays taken past the limit ends production: writing
+        // the stage or arriving on its full barrier could then land in a
+        // phase the consumers have not finished.  Their own bounded waits
+        // run out in turn and they report the timeout.
+        if (!mbar_wait(&empty[s], ((it / kNS) & 1) ^ 1)) {
+          gave_up = true;
+          break;
+        }
         uint8_t* stg = stages + s * kStageBytes;
         StageMeta meta;
         meta.tok0 = tok;
         meta.poison = bad_seq;
-        meta.timeout = gave_up;
+        meta.pad = 0;
         meta.blk = -1;
         meta.is8 = 0;
         meta.slot0 = static_cast<int16_t>(tok % kBlockTokens);
@@ -705,7 +712,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         meta.ntok = static_cast<int16_t>(max(0, min(step, t1 - tok)));
         meta.last = (tok + step >= t1) ? 1 : 0;
         *reinterpret_cast<StageMeta*>(stg + kOffMeta) = meta;
-        if (meta.blk >= 0 && !gave_up) {
+        if (meta.blk >= 0) {
           const int rows = (meta.ntok + 15) & ~15;   // whole 16-token tiles, inside the block
           const bool is8 = meta.is8;
           const int64_t phys = is8 ? meta.blk - P.n_q4 : meta.blk;
@@ -734,6 +741,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         ++it;
         tok += step;
       } while (tok < t1);
+      if (gave_up) break;
     }
     // no copy may still be landing when the CTA exits: wait (bounded) for the
     // last stages issued to complete
@@ -920,9 +928,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const uint8_t* stg = stages + s * kStageBytes;
       const StageMeta meta = *reinterpret_cast<const StageMeta*>(stg + kOffMeta);
       const bool last = dead ? true : meta.last;
-      timeout |= dead || meta.timeout;
+      timeout |= dead;
       poison |= meta.poison;
-      if (!dead && !meta.timeout && meta.blk >= 0 && warp * 16 < meta.ntok) {
+      if (!dead && meta.blk >= 0 && warp * 16 < meta.ntok) {
         // warp w takes the stage's tiles w, w + 8, ... (rows past ntok are masked)
         if constexpr (FP8) {
           constexpr int NTL = Geo<D, true>::MTILES >= kCW ? Geo<D, true>::MTILES / kCW : 1;

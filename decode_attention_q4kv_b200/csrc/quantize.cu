@@ -323,6 +323,7 @@ constexpr int kQConsumers = 23;                 // consumer warps (6 warps per s
 constexpr int kQItems = 16;                     // warp items in a full unit
 constexpr int kQThreads = (kQConsumers + 1) * 32;
 constexpr int kQStages = 4;
+constexpr int kQFull = 2 * kQStages;            // full barriers: two per stage, by unit mod 8
 constexpr int kQHalf = 16384;                 // input bytes of one tensor per stage
 constexpr int kQStageBytes = 2 * kQHalf;
 static_assert((kQStages & (kQStages - 1)) == 0, "stage index is a mask");
@@ -345,8 +346,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   using S = Shape<D>;
   extern __shared__ __align__(128) uint8_t qsmem[];
   uint8_t* stages = qsmem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + kQStages * kQStageBytes);
-  uint64_t* empty = full + kQStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + kQStages * kQStageBytes);   // [kQFull]
+  uint64_t* empty = full + kQFull;                                                 // [kQStages]
   __shared__ int s_timeout;
 
   griddep_wait();   // the inputs may come from the kernel before in the stream
@@ -355,10 +356,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const int hkv = pool.n_kv_heads;
   const int T = geo.unit_tokens, HP = geo.unit_heads, HC = geo.head_chunks;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kQStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kQItems);
-    }
+    for (int i = 0; i < kQFull; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < kQStages; ++i) mbar_init(&empty[i], kQItems);
     s_timeout = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -374,32 +373,34 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const int nvalid = static_cast<int>(umin(static_cast<uint32_t>(T), geo.n_tokens - t0));
       for (int hc = 0; hc < HC; ++hc, ++it) {
         const int s = it % kQStages;
+        uint64_t* fb = &full[it % kQFull];
         if (!mbar_wait(&empty[s], ((it / kQStages) & 1) ^ 1)) {
+          // production ends; an arrival here could fall in a phase still in
+          // flight, so the consumers find out through their own bounded waits
           s_timeout = 1;
-          mbar_arrive(&full[s]);   // release the consumers; they see the flag
           stop = true;
           break;
         }
         const int h0 = hc * HP, nh = min(HP, hkv - h0);
         const uint32_t row = static_cast<uint32_t>(nh) * D * sizeof(InT);   // bytes per token
         uint8_t* dst = stages + s * kQStageBytes;
-        mbar_arrive_tx(&full[s], 2u * nvalid * row);
+        mbar_arrive_tx(fb, 2u * nvalid * row);
         const InT* ks = k + static_cast<int64_t>(t0) * geo.stride + h0 * D;
         const InT* vs = v + static_cast<int64_t>(t0) * geo.stride + h0 * D;
         if (nh == hkv && geo.stride == static_cast<int64_t>(hkv) * D) {
-          bulk_g2s(dst, ks, nvalid * row, &full[s]);
-          bulk_g2s(dst + kQHalf, vs, nvalid * row, &full[s]);
+          bulk_g2s(dst, ks, nvalid * row, fb);
+          bulk_g2s(dst + kQHalf, vs, nvalid * row, fb);
         } else {
           for (int t = 0; t < nvalid; ++t) {
-            bulk_g2s(dst + t * row, ks + t * geo.stride, row, &full[s]);
-            bulk_g2s(dst + kQHalf + t * row, vs + t * geo.stride, row, &full[s]);
+            bulk_g2s(dst + t * row, ks + t * geo.stride, row, fb);
+            bulk_g2s(dst + kQHalf + t * row, vs + t * geo.stride, row, fb);
           }
         }
       }
     }
     // no copy may still be landing when the CTA exits
     for (uint32_t q = (it > kQStages ? it - kQStages : 0); q < it; ++q)
-      if (!mbar_wait(&full[q % kQStages], (q / kQStages) & 1)) break;
+      if (!mbar_wait(&full[q % kQFull], (q / kQFull) & 1)) break;
     return;
   }
 
@@ -409,6 +410,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
   // + VPW - 1 of its T) form one stream that warp w walks with stride 23.
   // A stage is released after its 16 items have arrived.  The position
   // (chunk c, head chunk hc, unit ul, item w16) advances without division.
+  //
+  // A parity wait tells only two phases of a barrier apart.  With stride 23 a
+  // warp has no item in some units (never two in a row), so with one full
+  // barrier per stage it could wait for unit u without having seen unit u - 4
+  // (same stage) complete, and a copy of u - 4 landing after later units'
+  // copies would let that wait return on the earlier phase: the warp would
+  // read the wrong data and arrive on the wrong phase of the empty barrier,
+  // after which the producer can arrive twice on one full phase.  Unit u
+  // therefore completes full barrier u mod 8 (two per stage), whose previous
+  // phase is unit u - 8.  A warp that waits for u has seen its previous item's
+  // unit (u - 1 or u - 2) land, so the producer had issued u - 4, which it
+  // does only once the items of u - 8 are released, i.e. after u - 8 landed;
+  // and the barrier cannot be past u while this warp's item in u is held.
   const int r = lane / S::LPV;       // token of the warp item
   const int j = lane % S::LPV;       // 16-channel run of the lane
   const int tpi_log = geo.items_per_head_log2;   // tpi = T / VPW, a power of two
@@ -435,7 +449,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     advance(nxt, kQConsumers);
     const int32_t blk_next = nxt.c < geo.n_chunks ? __ldg(block_ids + (nxt.c * T) / kBlockTokens) : 0;
     const int s = pos.ul & (kQStages - 1);
-    if (!mbar_wait(&full[s], (pos.ul / kQStages) & 1) || s_timeout) {
+    if (!mbar_wait(&full[pos.ul % kQFull], (pos.ul / kQFull) & 1) || s_timeout) {
       if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_TIMEOUT);
       break;
     }
@@ -774,7 +788,7 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
   geo.n_chunks = static_cast<uint32_t>(n_chunks);
   const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
   const int64_t grid = n_chunks < sms ? n_chunks : sms;
-  const size_t smem = kQStages * kQStageBytes + 2 * kQStages * sizeof(uint64_t);
+  const size_t smem = kQStages * kQStageBytes + (kQFull + kQStages) * sizeof(uint64_t);
   cudaError_t e = cudaSuccess;
 #define Q4KV_LAUNCH_Q(DD, T, R, M, ...)                                                              \
   do {                                                                                                 \
