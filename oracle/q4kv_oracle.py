@@ -51,7 +51,12 @@ design notes):
   * the FP8 comparison cache stores each raw value as one OCP E4M3 byte
     (bias 7, 3 mantissa bits, no infinities, largest finite 448), rounded
     to nearest with ties to even and saturated to +-448; no scale, no
-    rotation (the plainest FP8 KV cache).
+    rotation (the plainest FP8 KV cache);
+  * paging a block out of and back into the device ([AMBP] section 2.1,
+    items 1 and 3: blocks move between memory and storage, one agent's
+    cache is brought in while another decodes) copies its bytes unchanged:
+    a block image is a 16-byte header followed by the block's sections in
+    the pool's own layout, and loading it restores the block exactly.
 
 Precision: the encoding steps (rotation, min/max, scale/zero, codes,
 dequantisation) are binary32/binary16 by definition, so they are written
@@ -69,6 +74,10 @@ BLOCK_TOKENS = 256          # [AMBP] 2.1 item 1
 GROUP = 64                  # values sharing one (scale, zero) pair
 SENTINEL_LOGIT = -1.0e4     # [IKV]
 MASK_WORDS = BLOCK_TOKENS // 32
+# Block images [AMBP 2.1 item 1: blocks are paged between memory and storage]:
+# a fixed 16-byte header, then the block's bytes as the pool holds them.
+IMAGE_MAGIC = b"Q4KB"
+IMAGE_HEADER_BYTES = 16
 
 
 def levels(bits: int) -> int:
@@ -364,6 +373,75 @@ class OraclePool:
             blk, slot = divmod(sid, BLOCK_TOKENS)
             self.bits(blk)
             self.mask[blk, slot // 32] |= np.uint32(1 << (slot % 32))
+
+    # -- block images: paging between device and host [AMBP 2.1 items 1, 3; 5] --
+    def block_class(self, blk: int) -> int:
+        """Class tag of a block's image: 4 (4-bit), 8 (8-bit) or 0x108 (FP8)."""
+        bits = self.bits(blk)
+        return 0x108 if self.fp8 else bits
+
+    def image_sections(self, cls: int):
+        """(name, bytes) of the sections of an image of class `cls`, in order."""
+        row = self.d // 2 if cls == 4 else self.d
+        codes = self.hkv * BLOCK_TOKENS * row
+        params = 0 if cls == 0x108 else self.hkv * BLOCK_TOKENS * (self.d // GROUP) * 4
+        secs = [("header", IMAGE_HEADER_BYTES), ("k_codes", codes), ("v_codes", codes)]
+        if params:
+            secs += [("k_params", params), ("v_params", params)]
+        return secs + [("mask", MASK_WORDS * 4)]
+
+    def image_stride(self) -> int:
+        """Bytes between consecutive images: the largest class of the pool."""
+        classes = [0x108] if self.fp8 else ([4] if self.n_q4 else []) + ([8] if self.n_q8 else [])
+        return max(sum(b for _, b in self.image_sections(c)) for c in classes or [4])
+
+    def _block_arrays(self, blk: int):
+        """The block's arrays (views) in image order, header excluded."""
+        if self.bits(blk) == 4:
+            arrs = [self.codes4["k"][blk], self.codes4["v"][blk],
+                    self.params4["k"][blk], self.params4["v"][blk]]
+        else:
+            i8 = blk - self.n_q4
+            arrs = [self.codes8["k"][i8], self.codes8["v"][i8]]
+            if not self.fp8:
+                arrs += [self.params8["k"][i8], self.params8["v"][i8]]
+        return arrs + [self.mask[blk]]
+
+    def block_image(self, blk: int) -> np.ndarray:
+        """uint8 image of block `blk`: a 16-byte header (magic 'Q4KB', class,
+        head_dim, Hkv, source block id; little-endian) and then the block's
+        bytes exactly as the pool holds them -- K codes, V codes, K params,
+        V params (not for FP8), remap mask -- each section contiguous."""
+        hdr = np.zeros(IMAGE_HEADER_BYTES, np.uint8)
+        hdr[0:4] = np.frombuffer(IMAGE_MAGIC, np.uint8)
+        hdr[4:6] = np.array([self.block_class(blk)], "<u2").view(np.uint8)
+        hdr[6:8] = np.array([self.d], "<u2").view(np.uint8)
+        hdr[8:12] = np.array([self.hkv], "<u4").view(np.uint8)
+        hdr[12:16] = np.array([blk], "<i4").view(np.uint8)
+        parts = [hdr] + [np.ascontiguousarray(a).reshape(-1).view(np.uint8) for a in self._block_arrays(blk)]
+        return np.concatenate(parts)
+
+    def image_matches(self, blk: int, image: np.ndarray) -> bool:
+        """True when the header fits block `blk` of this pool (magic, class,
+        head_dim, Hkv; the source id is not checked)."""
+        h = np.asarray(image[:IMAGE_HEADER_BYTES], np.uint8)
+        return (h[0:4].tobytes() == IMAGE_MAGIC
+                and int(h[4:6].view("<u2")[0]) == self.block_class(blk)
+                and int(h[6:8].view("<u2")[0]) == self.d
+                and int(h[8:12].view("<u4")[0]) == self.hkv)
+
+    def load_block_image(self, blk: int, image: np.ndarray) -> bool:
+        """Replace block `blk` (codes, params, mask) by an image; an image
+        whose header does not fit the block changes nothing (returns False)."""
+        image = np.asarray(image, np.uint8)
+        if not self.image_matches(blk, image):
+            return False
+        off = IMAGE_HEADER_BYTES
+        for a in self._block_arrays(blk):
+            nb = a.size * a.itemsize
+            a[...] = image[off:off + nb].view(a.dtype).reshape(a.shape)
+            off += nb
+        return True
 
     # -- reads -------------------------------------------------------------
     def masked(self, blk: int) -> np.ndarray:

@@ -522,3 +522,99 @@ def test_fp8_pool_attention_matches_brute_force():
         s = kd @ q[0, h].astype(np.float64) / math.sqrt(d)
         p = scipy.special.softmax(s)
         np.testing.assert_allclose(out[0, h], p @ vd, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# block images (paging between device and host)
+# ---------------------------------------------------------------------------
+
+def _mixed_pool(seed=11, hkv=2, d=128, fp8=False):
+    rng = np.random.default_rng(seed)
+    n = 3 * 256 - 40
+    k = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    v = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    if fp8:
+        pool = O.OraclePool(hkv, d, 0, 4, k_rotated=False, fp8=True)
+        pool.quantize_blocks(k, v, "fp16", [2, 0, 3])
+    else:
+        pool = O.OraclePool(hkv, d, 2, 2)
+        pool.quantize_blocks(k, v, "fp16", [1, 3, 0])           # 4-bit, 8-bit, 4-bit
+    pool.invalidate_slots([5, 300, 3 * 256 + 7])
+    return pool, rng
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_block_image_sizes_follow_the_per_token_byte_counts(fp8):
+    """Header 16 B + mask 32 B + the block's bytes: 144 B per (token, KV
+    head) for a 4-bit block at D = 128 (the page's ~72 % figure), 272 B for
+    an 8-bit block, 256 B for an FP8 block."""
+    pool, _ = _mixed_pool(fp8=fp8)
+    per = {4: 144, 8: 272, 0x108: 256}
+    for blk in range(pool.n_blocks):
+        img = pool.block_image(blk)
+        assert img.size == 48 + per[pool.block_class(blk)] * 256 * pool.hkv
+    assert pool.image_stride() == 48 + (256 if fp8 else 272) * 256 * pool.hkv
+
+
+def test_block_image_layout_by_independent_indexing():
+    """Sampled bytes of the image sit where the layout puts them: K codes of
+    (head h, slot t, byte i) at 16 + (h*256 + t)*row + i, V codes one section
+    later, then the fp16 (scale, zero) pairs and the mask words."""
+    pool, rng = _mixed_pool()
+    for blk in (0, 3):
+        img = pool.block_image(blk)
+        assert img[:4].tobytes() == b"Q4KB"
+        assert int.from_bytes(img[4:6].tobytes(), "little") == pool.block_class(blk)
+        assert int.from_bytes(img[6:8].tobytes(), "little") == 128
+        assert int.from_bytes(img[8:12].tobytes(), "little") == 2
+        assert int.from_bytes(img[12:16].tobytes(), "little") == blk
+        is4 = blk < pool.n_q4
+        row = 64 if is4 else 128
+        cbytes = 2 * 256 * row
+        pbytes = 2 * 256 * 2 * 4
+        kc = pool.codes4["k"][blk] if is4 else pool.codes8["k"][blk - 2]
+        vc = pool.codes4["v"][blk] if is4 else pool.codes8["v"][blk - 2]
+        vp = pool.params4["v"][blk] if is4 else pool.params8["v"][blk - 2]
+        for _ in range(50):
+            h, t, i = int(rng.integers(2)), int(rng.integers(256)), int(rng.integers(row))
+            assert img[16 + (h * 256 + t) * row + i] == kc[h, t, i]
+            assert img[16 + cbytes + (h * 256 + t) * row + i] == vc[h, t, i]
+            g, e = int(rng.integers(2)), int(rng.integers(2))
+            off = 16 + 2 * cbytes + pbytes + ((h * 256 + t) * 2 + g) * 4 + 2 * e
+            assert img[off:off + 2].view(np.float16)[0].view(np.uint16) == vp[h, t, g, e].view(np.uint16)
+        mask_off = 16 + 2 * cbytes + 2 * pbytes
+        for w in range(8):
+            assert int.from_bytes(img[mask_off + 4 * w:mask_off + 4 * w + 4].tobytes(), "little") == int(pool.mask[blk, w])
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_block_images_restore_blocks_exactly(fp8):
+    """Loading every block's image into a fresh pool at a permuted id of the
+    same class gives back the same dequantised blocks and the same attention."""
+    src, rng = _mixed_pool(fp8=fp8)
+    dst = (O.OraclePool(2, 128, 0, 4, k_rotated=False, fp8=True) if fp8 else O.OraclePool(2, 128, 2, 2))
+    perm = {2: 0, 0: 3, 3: 2, 1: 1} if fp8 else {0: 1, 1: 0, 2: 3, 3: 2}   # same class both sides
+    for a, b in perm.items():
+        assert dst.load_block_image(b, src.block_image(a))
+    for a, b in perm.items():
+        for x, y in zip(src.dequantize_block(a), dst.dequantize_block(b)):
+            np.testing.assert_array_equal(x, y)
+        np.testing.assert_array_equal(src.masked(a), dst.masked(b))
+    q = rng.standard_normal((1, 4, 128)).astype(np.float16)
+    tbl = [2, 0, 3] if fp8 else [1, 3, 0]
+    out_src = O.decode_attention(src, q, "fp16", np.array([tbl]), [3 * 256 - 40])
+    out_dst = O.decode_attention(dst, q, "fp16", np.array([[perm[t] for t in tbl]]), [3 * 256 - 40])
+    np.testing.assert_array_equal(out_src, out_dst)
+
+
+def test_block_image_of_another_class_or_shape_is_refused():
+    src, _ = _mixed_pool()
+    dst = O.OraclePool(2, 128, 2, 2)
+    before = dst.block_image(2).copy()
+    assert not dst.load_block_image(2, src.block_image(0))      # 4-bit image into an 8-bit block
+    np.testing.assert_array_equal(dst.block_image(2), before)
+    other = O.OraclePool(4, 128, 2, 2)                          # another Hkv
+    assert not other.load_block_image(0, src.block_image(0))
+    bad = src.block_image(0).copy()
+    bad[0] ^= 1                                                 # broken magic
+    assert not dst.load_block_image(0, bad)
