@@ -390,6 +390,8 @@ def run_gpu(args):
     app_ms = statistics.median(a.elapsed_time(b) for a, b, _ in gen)
     gen_ms = statistics.median(a.elapsed_time(c) for a, _, c in gen)
 
+    paging = measure_paging(job, dev, reps, d_cold_ms)
+
     e2e = run_e2e(job, args, dev, world) if not args.no_e2e else None
     if world > 1:
         dist.barrier()
@@ -439,6 +441,7 @@ def run_gpu(args):
                            "bytes_per_launch": job.append_bytes,
                            "append_then_decode_us": round(gen_ms * 1e3, 2),
                            "note": "one new token per sequence written over its last slot, then decode"},
+                "paging": paging,
             },
             "roofline": roof,
             "gpu_launches": job.launches_per_layer * job.n_layers * args.steps,
@@ -452,6 +455,80 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_paging(job, dev, reps, decode_ms):
+    """Block images of the first layer's whole pool to and from pinned host
+    memory: the export and import kernels alone, the copy engine moving the
+    same bytes (reference), and the import on a second stream beside a decode
+    of the same layer (the import targets a second pool, so decode reads
+    unchanged blocks)."""
+    import torch
+    import decode_attention_q4kv_b200 as q4
+    L = job.layers[0]
+    pool = L["pool"]
+    nb = pool.n_blocks
+    ids = torch.arange(nb, dtype=torch.int32, device=dev)
+    stride = pool.image_stride()
+    images = torch.empty((nb, stride), dtype=torch.uint8, pin_memory=True)
+    moved = pool.nbytes() + 16 * nb                       # every block's sections + its header
+    other = q4.Q4KVPool(pool.n_kv_heads, pool.head_dim, pool.n_q4_blocks, pool.n_q8_blocks,
+                        k_rotated=pool.k_rotated, device=dev, fp8=pool.fp8)
+    flat = images.view(-1)
+    dev_buf = torch.empty(flat.numel(), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        out = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            out.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in out)
+
+    host_ids = ids.cpu()
+    h2d_ms = timed(lambda: dev_buf.copy_(flat, non_blocking=True))
+    d2h_ms = timed(lambda: flat.copy_(dev_buf, non_blocking=True))
+    s_dec, s_copy = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def beside(import_ids):
+        spans = []
+        for _ in range(reps):
+            go = torch.cuda.Event()
+            go.record()
+            s_dec.wait_event(go)
+            s_copy.wait_event(go)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(s_dec)
+            with torch.cuda.stream(s_dec):
+                job.decode_layer(L)
+            e[1].record(s_dec)
+            e[2].record(s_copy)
+            with torch.cuda.stream(s_copy):
+                other.import_blocks(images, import_ids)
+            e[3].record(s_copy)
+            spans.append(e)
+        torch.cuda.synchronize()
+        return (round(statistics.median(a.elapsed_time(b) for a, b, _, _ in spans) * 1e3, 2),
+                round(statistics.median(c.elapsed_time(d) for _, _, c, d in spans) * 1e3, 1))
+
+    gbps = lambda ms: round(moved / (ms * 1e-3) / 1e9, 2)
+    out = {"blocks": nb, "bytes": moved, "image_stride": stride,
+           "copy_engine_h2d_gbps": round(flat.numel() / (h2d_ms * 1e-3) / 1e9, 2),
+           "copy_engine_d2h_gbps": round(flat.numel() / (d2h_ms * 1e-3) / 1e9, 2),
+           "decode_us_alone": round(decode_ms * 1e3, 2)}
+    for tag, the_ids in (("kernel", ids), ("copy_engine", host_ids)):
+        exp_ms = timed(lambda: pool.export_blocks(the_ids, images))
+        imp_ms = timed(lambda: other.import_blocks(images, the_ids))
+        dec_b, imp_b = beside(the_ids)
+        out[tag] = {"export_gbps": gbps(exp_ms), "export_us": round(exp_ms * 1e3, 1),
+                    "import_gbps": gbps(imp_ms), "import_us": round(imp_ms * 1e3, 1),
+                    "decode_us_beside_import": dec_b, "import_us_beside_decode": imp_b}
+    out["note"] = ("pinned host images of the first layer's whole pool; kernel = device block ids, one "
+                   "launch reading/writing host memory; copy_engine = host block ids, strided copies, no SM")
+    return out
 
 
 def run_e2e(job, args, dev, world):

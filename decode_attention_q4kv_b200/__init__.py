@@ -168,6 +168,55 @@ class Q4KVPool:
         check(lib().q4kv_invalidate_slots(ctypes.byref(self.desc), _ptr(ids), ids.numel(), _stream(dev)),
               "q4kv_invalidate_slots")
 
+    # -- paging between device and host -------------------------------------
+    def image_stride(self) -> int:
+        """Bytes between consecutive block images (the largest block class)."""
+        out = ctypes.c_size_t(0)
+        check(lib().q4kv_block_image_stride(ctypes.byref(self.desc), ctypes.byref(out)),
+              "q4kv_block_image_stride")
+        return int(out.value)
+
+    def export_blocks(self, block_ids: torch.Tensor, images: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Images of the blocks into pinned host memory, uint8 [n][stride].
+
+        Device ids: one kernel writes the images.  Host (CPU) ids: the copy
+        engines do, with no kernel.  Enqueued on the current stream; the bytes
+        are complete once that stream has passed the call."""
+        ids = block_ids.to(torch.int32).contiguous()
+        stride = self.image_stride()
+        if images is None:
+            images = torch.empty((ids.numel(), stride), dtype=torch.uint8, pin_memory=True)
+        _check_images(images, ids.numel(), stride)
+        if ids.device.type == "cpu":
+            check(lib().q4kv_export_blocks_host_ids(ctypes.byref(self.desc), _ptr(ids), ids.numel(),
+                                                    ctypes.c_void_p(images.data_ptr()), _stream(self.device)),
+                  "q4kv_export_blocks_host_ids")
+            return images
+        dev = _require_cuda(ids)
+        check(lib().q4kv_export_blocks(ctypes.byref(self.desc), _ptr(ids), ids.numel(),
+                                       ctypes.c_void_p(images.data_ptr()), _stream(dev)),
+              "q4kv_export_blocks")
+        return images
+
+    def import_blocks(self, images: torch.Tensor, block_ids: torch.Tensor) -> None:
+        """Load pinned host images (uint8 [n][stride]) into blocks block_ids[i].
+
+        Device ids: one kernel, headers checked on the device.  Host (CPU)
+        ids: the copy engines, headers checked here first.  Enqueued on the
+        current stream; `images` must stay unchanged until that stream has
+        passed the call."""
+        ids = block_ids.to(torch.int32).contiguous()
+        _check_images(images, ids.numel(), self.image_stride())
+        if ids.device.type == "cpu":
+            check(lib().q4kv_import_blocks_host_ids(ctypes.byref(self.desc), ctypes.c_void_p(images.data_ptr()),
+                                                    _ptr(ids), ids.numel(), _stream(self.device)),
+                  "q4kv_import_blocks_host_ids")
+            return
+        dev = _require_cuda(ids)
+        check(lib().q4kv_import_blocks(ctypes.byref(self.desc), ctypes.c_void_p(images.data_ptr()),
+                                       _ptr(ids), ids.numel(), _stream(dev)),
+              "q4kv_import_blocks")
+
     # -- reads --------------------------------------------------------------
     def dequantize(self, block_ids: torch.Tensor, out_dtype=torch.float32,
                    unrotate_k: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -190,6 +239,13 @@ class Q4KVPool:
         if st not in (_lib.OK, _lib.ERR_DEVICE):
             check(st, "q4kv_read_device_error")
         return int(bits.value)
+
+
+def _check_images(images: torch.Tensor, n: int, stride: int) -> None:
+    if images.device.type != "cpu" or not images.is_pinned():
+        raise ValueError("block images live in pinned host memory")
+    if images.dtype != torch.uint8 or not images.is_contiguous() or images.numel() < n * stride:
+        raise ValueError(f"block images must be contiguous uint8 of at least {n} x {stride} bytes")
 
 
 def block_absmean(k: torch.Tensor) -> torch.Tensor:

@@ -48,6 +48,24 @@ q4kv_status check_input(const void* x, int32_t dtype, int64_t n_tokens, int64_t 
   return Q4KV_OK;
 }
 
+// Host argument checks shared by export and import; *dev receives the
+// device's address of the host buffer.
+q4kv_status check_paging(const q4kv_pool* pool, const int32_t* ids, int32_t n, const void* host, void** dev) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  if (n < 0) return Q4KV_ERR_INVALID_ARG;
+  if (n == 0) return Q4KV_OK;
+  if (ids == nullptr || !aligned(ids, 4) || host == nullptr || !aligned(host, 16)) return Q4KV_ERR_INVALID_ARG;
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, host) != cudaSuccess) {
+    cudaGetLastError();
+    return Q4KV_ERR_INVALID_ARG;
+  }
+  if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr) return Q4KV_ERR_INVALID_ARG;
+  *dev = attr.devicePointer;
+  return Q4KV_OK;
+}
+
 q4kv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? Q4KV_OK : Q4KV_ERR_CUDA; }
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
@@ -119,6 +137,56 @@ q4kv_status q4kv_append_tokens(const q4kv_pool* pool, const void* k, const void*
     return Q4KV_ERR_INVALID_ARG;
   return from_cuda(launch_append(view_of(*pool), k, v, in_dtype, batch, max_new, n_new, seq_stride,
                                  token_stride, tables, max_blocks, seq_lens, as_stream(stream)));
+}
+
+q4kv_status q4kv_block_image_stride(const q4kv_pool* pool, size_t* stride_bytes) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  if (stride_bytes == nullptr) return Q4KV_ERR_INVALID_ARG;
+  *stride_bytes = static_cast<size_t>(image_stride_bytes(view_of(*pool)));
+  return Q4KV_OK;
+}
+
+
+q4kv_status q4kv_export_blocks(const q4kv_pool* pool, const int32_t* block_ids, int32_t n_blocks,
+                               void* host_images, void* stream) {
+  void* dev = nullptr;
+  q4kv_status st = check_paging(pool, block_ids, n_blocks, host_images, &dev);
+  if (st != Q4KV_OK || n_blocks == 0) return st;
+  return from_cuda(launch_page(view_of(*pool), block_ids, n_blocks, dev, true, as_stream(stream)));
+}
+
+q4kv_status q4kv_import_blocks(const q4kv_pool* pool, const void* host_images, const int32_t* block_ids,
+                               int32_t n_blocks, void* stream) {
+  void* dev = nullptr;
+  q4kv_status st = check_paging(pool, block_ids, n_blocks, host_images, &dev);
+  if (st != Q4KV_OK || n_blocks == 0) return st;
+  return from_cuda(launch_page(view_of(*pool), block_ids, n_blocks, dev, false, as_stream(stream)));
+}
+
+q4kv_status q4kv_export_blocks_host_ids(const q4kv_pool* pool, const int32_t* block_ids, int32_t n_blocks,
+                                        void* host_images, void* stream) {
+  void* dev = nullptr;
+  q4kv_status st = check_paging(pool, block_ids, n_blocks, host_images, &dev);
+  if (st != Q4KV_OK || n_blocks == 0) return st;
+  const PoolView v = view_of(*pool);
+  for (int32_t i = 0; i < n_blocks; ++i)
+    if (block_ids[i] < 0 || block_ids[i] >= v.n_q4 + v.n_q8) return Q4KV_ERR_INVALID_ARG;
+  host_headers(v, block_ids, n_blocks, static_cast<uint8_t*>(host_images), true);
+  return from_cuda(copy_pages(v, block_ids, n_blocks, static_cast<uint8_t*>(host_images), true, as_stream(stream)));
+}
+
+q4kv_status q4kv_import_blocks_host_ids(const q4kv_pool* pool, const void* host_images, const int32_t* block_ids,
+                                        int32_t n_blocks, void* stream) {
+  void* dev = nullptr;
+  q4kv_status st = check_paging(pool, block_ids, n_blocks, host_images, &dev);
+  if (st != Q4KV_OK || n_blocks == 0) return st;
+  const PoolView v = view_of(*pool);
+  for (int32_t i = 0; i < n_blocks; ++i)
+    if (block_ids[i] < 0 || block_ids[i] >= v.n_q4 + v.n_q8) return Q4KV_ERR_INVALID_ARG;
+  uint8_t* img = static_cast<uint8_t*>(const_cast<void*>(host_images));
+  if (!host_headers(v, block_ids, n_blocks, img, false)) return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(copy_pages(v, block_ids, n_blocks, img, false, as_stream(stream)));
 }
 
 q4kv_status q4kv_selftest_bounded_wait(uint32_t* error_word, int32_t tries, void* stream) {

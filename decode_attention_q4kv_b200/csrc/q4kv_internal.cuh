@@ -116,6 +116,15 @@ cudaError_t launch_append(const PoolView& pool, const void* k, const void* v, in
                           int64_t token_stride, const int32_t* tables, int32_t max_blocks,
                           const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_selftest_wait(uint32_t* error_word, unsigned tries, cudaStream_t stream);
+// Block images (paging.cu): stride of one image for this pool, and one
+// launch moving n blocks' images between the pool and host memory.
+int64_t image_stride_bytes(const PoolView& pool);
+cudaError_t launch_page(const PoolView& pool, const int32_t* ids, int32_t n, void* host, bool to_host,
+                        cudaStream_t stream);
+// Copy-engine paging with host block ids (paging.cu): headers, then copies.
+bool host_headers(const PoolView& pool, const int32_t* ids, int32_t n, uint8_t* host, bool write);
+cudaError_t copy_pages(const PoolView& pool, const int32_t* ids, int32_t n, uint8_t* host, bool to_host,
+                       cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,
                               void* k_out, void* v_out, int out_dtype, int unrotate_k,
                               cudaStream_t stream);

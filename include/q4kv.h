@@ -68,7 +68,7 @@
 extern "C" {
 #endif
 
-#define Q4KV_ABI_VERSION 2
+#define Q4KV_ABI_VERSION 3
 #define Q4KV_BLOCK_TOKENS 256
 #define Q4KV_GROUP 64
 #define Q4KV_MASK_WORDS 8            /* uint32 words of remap mask per block */
@@ -88,6 +88,7 @@ typedef enum {
 #define Q4KV_DEVERR_SEQ_LEN 2u   /* seq_len < 0 or > max_blocks_per_seq * 256 */
 #define Q4KV_DEVERR_SLOT_ID 4u   /* a slot id outside [0, 256 * (n_q4_blocks + n_q8_blocks)) */
 #define Q4KV_DEVERR_TIMEOUT 8u   /* a bounded device-side wait gave up */
+#define Q4KV_DEVERR_IMAGE 16u    /* a block image whose header does not fit its target block */
 
 typedef enum { Q4KV_F16 = 0, Q4KV_BF16 = 1, Q4KV_F32 = 2 } q4kv_dtype;
 
@@ -341,6 +342,77 @@ q4kv_status q4kv_decode_attention_static_scratch(const q4kv_pool *pool,
  * context stays usable; tests use it to check that waits end.
  */
 q4kv_status q4kv_selftest_bounded_wait(uint32_t *error_word, int32_t tries, void *stream);
+
+/*
+ * Block images: paging blocks between device and host memory ([AMBP] sec.
+ * 2.1 item 1: the pool pages 256-token blocks between fast memory and
+ * storage; item 3: one agent's cache is brought in while another agent
+ * decodes; sec. 5: storage as the cache's swap space).  The storage tier
+ * itself (files, safetensors) is the caller's.
+ *
+ * An image is one block in one contiguous run of bytes, every section a
+ * multiple of 16 bytes:
+ *   header  16 B: uint32 magic 0x424B3451 ("Q4KB"), uint16 class (4 = 4-bit,
+ *           8 = 8-bit, 0x108 = FP8), uint16 head_dim, uint32 n_kv_heads,
+ *           int32 the block id it was exported from (informational)
+ *   K codes [Hkv][256][row] bytes, row = D/2 (4-bit) or D (8-bit, FP8)
+ *   V codes the same
+ *   K params [Hkv][256][D/64] half2, then V params (absent for FP8 pools)
+ *   remap mask 8 uint32
+ * i.e. the block's bytes exactly as the pool holds them.  Images of one call
+ * sit at a fixed stride, the size of the pool's largest block class; a
+ * smaller class leaves the rest of its stride unused.
+ */
+q4kv_status q4kv_block_image_stride(const q4kv_pool *pool, size_t *stride_bytes);
+
+/*
+ * Write the images of blocks block_ids[0 .. n_blocks) to host memory.
+ *   block_ids    device int32 [n_blocks]
+ *   host_images  page-locked host memory the device can address
+ *                (cudaHostAlloc, or cudaHostRegister'ed), 16-byte aligned,
+ *                at least n_blocks * stride bytes; image i at i * stride.
+ * One kernel reads the pool and stores straight into host memory over the
+ * bus, so the call can run on a stream of its own beside other work.  The
+ * images are complete once `stream` has reached this point.  An
+ * out-of-range id leaves its image unwritten and raises
+ * Q4KV_DEVERR_BLOCK_ID.  n_blocks == 0 is a no-op.  Pageable host memory is
+ * refused with Q4KV_ERR_INVALID_ARG.
+ */
+q4kv_status q4kv_export_blocks(const q4kv_pool *pool, const int32_t *block_ids, int32_t n_blocks,
+                               void *host_images, void *stream);
+
+/*
+ * Load images from host memory into blocks block_ids[0 .. n_blocks): image i
+ * replaces block block_ids[i] entirely (codes, params, remap mask).  Each
+ * image's header must fit its target block (magic, class, head_dim, Hkv);
+ * one that does not leaves the block unchanged and raises Q4KV_DEVERR_IMAGE.
+ * Same memory rules as q4kv_export_blocks; the host bytes must stay
+ * unchanged until `stream` has passed the call.  Target ids must be distinct,
+ * and no other work may read or write those blocks while the copy runs
+ * (decode of other blocks may run concurrently on another stream).
+ */
+q4kv_status q4kv_import_blocks(const q4kv_pool *pool, const void *host_images, const int32_t *block_ids,
+                               int32_t n_blocks, void *stream);
+
+/*
+ * The same two moves with the block ids in HOST memory, done by the copy
+ * engines: no kernel runs and no SM is used, so a block can page in while
+ * decode keeps every SM (the way [AMBP] sec. 2.1 item 3 hides loading).
+ *   block_ids    host int32 [n_blocks], each in range (else
+ *                Q4KV_ERR_INVALID_ARG before anything is enqueued)
+ *   host_images  as above (page-locked, 16-byte aligned, image i at i*stride)
+ * Export writes every image's header from the host at call time and
+ * enqueues the section copies; import reads and checks every header at call
+ * time (so the images must already be complete then) and returns
+ * Q4KV_ERR_INVALID_ARG, enqueuing nothing, if one does not fit its target
+ * block.  Each run of consecutive ids of one block class, at consecutive
+ * images, moves as one strided 2-D copy per section.  The results equal those
+ * of q4kv_export_blocks / q4kv_import_blocks.
+ */
+q4kv_status q4kv_export_blocks_host_ids(const q4kv_pool *pool, const int32_t *block_ids, int32_t n_blocks,
+                                        void *host_images, void *stream);
+q4kv_status q4kv_import_blocks_host_ids(const q4kv_pool *pool, const void *host_images,
+                                        const int32_t *block_ids, int32_t n_blocks, void *stream);
 
 /*
  * Wait for `stream`, read pool->error_word into *bits, and zero it when

@@ -24,7 +24,7 @@ def _pool(**kw):
 
 def test_exports_every_declared_function():
     names = _lib.header_functions()
-    assert len(names) == 14
+    assert len(names) == 19
     for n in names:
         assert hasattr(L, n), n
     # the binding declares a signature for each of them
@@ -32,7 +32,7 @@ def test_exports_every_declared_function():
 
 
 def test_abi_version_and_status_strings():
-    assert L.q4kv_abi_version() == 2
+    assert L.q4kv_abi_version() == 3
     assert L.q4kv_status_string(0) == b"ok"
     assert b"workspace" in L.q4kv_status_string(_lib.ERR_WORKSPACE)
     assert L.q4kv_status_string(99) == b"unknown status"
@@ -194,3 +194,47 @@ def test_read_device_error_without_word():
     assert L.q4kv_read_device_error(ctypes.byref(p), ctypes.byref(bits), 1, None) == 0
     assert bits.value == 0
     assert L.q4kv_read_device_error(None, ctypes.byref(bits), 1, None) == _lib.ERR_INVALID_ARG
+
+
+def _stride(pool):
+    out = ctypes.c_size_t(0)
+    st = L.q4kv_block_image_stride(ctypes.byref(pool), ctypes.byref(out))
+    return st, out.value
+
+
+@pytest.mark.parametrize("d,hkv,n_q8,fp8", [(128, 8, 0, 0), (128, 8, 3, 0), (256, 4, 0, 0), (128, 2, 4, 1),
+                                            (256, 8, 2, 0)])
+def test_block_image_stride_matches_the_oracle(d, hkv, n_q8, fp8):
+    from oracle import q4kv_oracle as O
+    n_q4 = 0 if fp8 else 4
+    kw = dict(head_dim=d, n_kv_heads=hkv, n_q4_blocks=n_q4, n_q8_blocks=n_q8, value_format=fp8,
+              k_rotated=0 if fp8 else 1)
+    if n_q8:
+        kw.update(k_codes8=FAKE, v_codes8=FAKE, k_params8=FAKE, v_params8=FAKE)
+    if fp8:
+        kw.update(k_codes4=0, v_codes4=0, k_params4=0, v_params4=0, k_params8=0, v_params8=0)
+    st, stride = _stride(_pool(**kw))
+    assert st == 0
+    ref = O.OraclePool(hkv, d, n_q4, n_q8, k_rotated=not fp8, fp8=bool(fp8))
+    assert stride == ref.image_stride() and stride % 16 == 0
+
+
+def test_paging_rejects_bad_arguments_without_launching():
+    p = _pool()
+    e, i = L.q4kv_export_blocks, L.q4kv_import_blocks
+    assert _stride(_pool(head_dim=64))[0] == _lib.ERR_UNSUPPORTED
+    assert L.q4kv_block_image_stride(ctypes.byref(p), None) == _lib.ERR_INVALID_ARG
+    host = ctypes.create_string_buffer(1 << 16)                # pageable host memory
+    addr = (ctypes.addressof(host) + 15) // 16 * 16
+    eh, ih = L.q4kv_export_blocks_host_ids, L.q4kv_import_blocks_host_ids
+    for call in (lambda ids, n, h: e(ctypes.byref(p), ids, n, h, None),
+                 lambda ids, n, h: i(ctypes.byref(p), h, ids, n, None),
+                 lambda ids, n, h: eh(ctypes.byref(p), ids, n, h, None),
+                 lambda ids, n, h: ih(ctypes.byref(p), h, ids, n, None)):
+        assert call(FAKE, -1, addr) == _lib.ERR_INVALID_ARG
+        assert call(None, 2, addr) == _lib.ERR_INVALID_ARG
+        assert call(FAKE + 2, 2, addr) == _lib.ERR_INVALID_ARG
+        assert call(FAKE, 2, None) == _lib.ERR_INVALID_ARG
+        assert call(FAKE, 2, addr + 8) == _lib.ERR_INVALID_ARG          # misaligned images
+        assert call(FAKE, 2, addr) == _lib.ERR_INVALID_ARG              # not page-locked
+        assert call(FAKE, 0, None) == 0                                 # nothing to move
