@@ -56,7 +56,13 @@ design notes):
     items 1 and 3: blocks move between memory and storage, one agent's
     cache is brought in while another decodes) copies its bytes unchanged:
     a block image is a 16-byte header followed by the block's sections in
-    the pool's own layout, and loading it restores the block exactly.
+    the pool's own layout, and loading it restores the block exactly;
+  * per-token widths from {2, 4, 8, FP16} in one cache ([QKVS]
+    "Methodologie": the CacheCard carries quantised groups and per-token
+    widths, and the receiver rebuilds FP16 keys and values before use): a
+    card holds each token at its own width with the pool's group coding
+    (L = 2^w - 1; 2-bit codes four to a byte in the nibble order, generalised)
+    or as its raw 16-bit rows, and decoding it dequantises and un-rotates.
 
 Precision: the encoding steps (rotation, min/max, scale/zero, codes,
 dequantisation) are binary32/binary16 by definition, so they are written
@@ -585,3 +591,155 @@ def bytes_per_token_head(head_dim: int, bits: int) -> int:
     code_bytes = head_dim * bits // 8
     param_bytes = (head_dim // GROUP) * 2 * 2
     return 2 * (code_bytes + param_bytes)
+
+
+# ---------------------------------------------------------------------------
+# per-token widths {2, 4, 8, FP16} in one cache: the card [QKVS "Methodologie"]
+# ---------------------------------------------------------------------------
+# QKVS gives every token a width from {2, 4, 8, FP16} and ships the cache as
+# a compact artifact holding the quantised groups, the per-token widths and
+# metadata; the receiver rebuilds FP16 keys and values from it before use.
+# Reading: the card is a 64-byte header, the widths (one byte per token), the
+# byte offset of every token's record, then the records.  A token's record is,
+# for every KV head in order, its K codes, V codes, K (s, z) pairs and V (s, z)
+# pairs at its width (the pool's group coding with L = 2^w - 1, K rotated when
+# the card says so), or for an FP16 token its raw 16-bit K and V rows.
+CARD_MAGIC = b"QKVC"
+CARD_VERSION = 1
+CARD_HEADER_BYTES = 64
+CARD_WIDTHS = (2, 4, 8, 16)
+
+
+def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
+    """bits-wide codes [..., D] -> bytes: element e sits at bits
+    bits*(e mod 8/bits) of byte e*bits/8 (the nibble order, generalised)."""
+    per = 8 // bits
+    c = np.asarray(codes, np.uint32).reshape(codes.shape[:-1] + (codes.shape[-1] // per, per))
+    out = np.zeros(c.shape[:-1], np.uint32)
+    for e in range(per):
+        out |= c[..., e] << np.uint32(bits * e)
+    return out.astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray, bits: int) -> np.ndarray:
+    per = 8 // bits
+    p = np.asarray(packed, np.uint32)[..., None]
+    shifts = np.arange(per, dtype=np.uint32) * np.uint32(bits)
+    out = (p >> shifts) & np.uint32((1 << bits) - 1)
+    return out.reshape(packed.shape[:-1] + (packed.shape[-1] * per,)).astype(np.uint8)
+
+
+def card_record_bytes(head_dim: int, bits: int) -> int:
+    """Bytes of one (token, KV head) record at width `bits`; 0 for a width
+    outside {2, 4, 8, 16} (such a token is skipped)."""
+    if bits == 16:
+        return 4 * head_dim
+    if bits in (2, 4, 8):
+        return bytes_per_token_head(head_dim, bits)
+    return 0
+
+
+def _round16(x: int) -> int:
+    return (x + 15) // 16 * 16
+
+
+def card_layout(head_dim: int, n_kv_heads: int, widths: Sequence[int]):
+    """(offsets of each token's record from the payload start, int64 [n + 1];
+    byte offsets of the widths, the offsets table and the payload; total
+    card bytes)."""
+    n = len(widths)
+    rec = np.array([n_kv_heads * card_record_bytes(head_dim, int(w)) for w in widths], np.int64)
+    offs = np.zeros(n + 1, np.int64)
+    offs[1:] = np.cumsum(rec)
+    widths_at = CARD_HEADER_BYTES
+    offsets_at = widths_at + _round16(n)
+    payload_at = offsets_at + _round16(8 * (n + 1))
+    return offs, widths_at, offsets_at, payload_at, payload_at + int(offs[-1])
+
+
+def card_encode(k: np.ndarray, v: np.ndarray, dtype: str, widths: Sequence[int],
+                k_rotated: bool = True) -> np.ndarray:
+    """The card (uint8) of tokens k, v [n][Hkv][D] at per-token widths."""
+    n, hkv, d = np.asarray(k).shape
+    kf, vf = to_f32(k, dtype), to_f32(v, dtype)
+    raw_k = np.asarray(k).view(np.uint16) if dtype == "fp16" else np.asarray(k, np.uint16)
+    raw_v = np.asarray(v).view(np.uint16) if dtype == "fp16" else np.asarray(v, np.uint16)
+    offs, w_at, o_at, p_at, total = card_layout(d, hkv, widths)
+    card = np.zeros(total, np.uint8)
+    hdr = card[:CARD_HEADER_BYTES]
+    hdr[0:4] = np.frombuffer(CARD_MAGIC, np.uint8)
+    hdr[4:24] = np.array([CARD_VERSION, d, hkv, n & 0xFFFFFFFF, n >> 32], "<u4").view(np.uint8)
+    hdr[24:32] = np.array([int(k_rotated), 0 if dtype == "fp16" else 1], "<u4").view(np.uint8)
+    hdr[32:40] = np.array([offs[-1]], "<i8").view(np.uint8)
+    card[w_at:w_at + n] = np.asarray(widths, np.uint8)
+    card[o_at:o_at + 8 * (n + 1)] = offs.astype("<i8").view(np.uint8)
+    for t in range(n):
+        w = int(widths[t])
+        at = p_at + int(offs[t])
+        if w == 16:
+            for h in range(hkv):
+                rec = np.concatenate([raw_k[t, h].astype("<u2").view(np.uint8),
+                                      raw_v[t, h].astype("<u2").view(np.uint8)])
+                card[at:at + rec.size] = rec
+                at += rec.size
+            continue
+        if w not in (2, 4, 8):
+            continue
+        kk = rotate_f32(kf[t:t + 1])[0] if k_rotated else kf[t]
+        ck, sk, zk = quantize_groups(kk, w)          # [Hkv][D], [Hkv][D/64]
+        cv, sv, zv = quantize_groups(vf[t], w)
+        for h in range(hkv):
+            pk = np.stack([sk[h], zk[h]], axis=-1).reshape(-1).view(np.uint8)
+            pv = np.stack([sv[h], zv[h]], axis=-1).reshape(-1).view(np.uint8)
+            rec = np.concatenate([pack_codes(ck[h], w), pack_codes(cv[h], w), pk, pv])
+            card[at:at + rec.size] = rec
+            at += rec.size
+    return card
+
+
+def card_header(card: np.ndarray) -> dict:
+    h = np.asarray(card[:CARD_HEADER_BYTES], np.uint8)
+    u = h[4:32].view("<u4")
+    return dict(magic=h[0:4].tobytes(), version=int(u[0]), head_dim=int(u[1]), n_kv_heads=int(u[2]),
+                n_tokens=int(u[3]) | (int(u[4]) << 32), k_rotated=int(u[5]), raw_dtype=int(u[6]),
+                payload_bytes=int(h[32:40].view("<i8")[0]))
+
+
+def card_decode(card: np.ndarray):
+    """Binary32 K_hat, V_hat [n][Hkv][D] of a card: x_hat = fl(code s + z),
+    K un-rotated by c*H when stored rotated; FP16 tokens exactly; a token of
+    an invalid width reads 0."""
+    hd = card_header(card)
+    n, hkv, d = hd["n_tokens"], hd["n_kv_heads"], hd["head_dim"]
+    widths = np.asarray(card[CARD_HEADER_BYTES:CARD_HEADER_BYTES + n], np.uint8)
+    offs, _, o_at, p_at, _ = card_layout(d, hkv, widths)
+    stored = np.asarray(card[o_at:o_at + 8 * (n + 1)]).view("<i8")
+    assert np.array_equal(stored, offs), "offset table does not match the widths"
+    k_hat = np.zeros((n, hkv, d), np.float32)
+    v_hat = np.zeros((n, hkv, d), np.float32)
+    raw = "fp16" if hd["raw_dtype"] == 0 else "bf16"
+    ng = d // GROUP
+    for t in range(n):
+        w = int(widths[t])
+        at = p_at + int(offs[t])
+        for h in range(hkv):
+            if w == 16:
+                rk = np.asarray(card[at:at + 2 * d]).view("<u2")
+                rv = np.asarray(card[at + 2 * d:at + 4 * d]).view("<u2")
+                k_hat[t, h] = to_f32(rk.view(np.float16) if raw == "fp16" else rk, raw)
+                v_hat[t, h] = to_f32(rv.view(np.float16) if raw == "fp16" else rv, raw)
+                at += 4 * d
+                continue
+            if w not in (2, 4, 8):
+                continue
+            cb = d * w // 8
+            ck = unpack_codes(card[at:at + cb], w)
+            cv = unpack_codes(card[at + cb:at + 2 * cb], w)
+            pk = np.asarray(card[at + 2 * cb:at + 2 * cb + 4 * ng]).view(np.float16).reshape(ng, 2)
+            pv = np.asarray(card[at + 2 * cb + 4 * ng:at + 2 * cb + 8 * ng]).view(np.float16).reshape(ng, 2)
+            k_hat[t, h] = dequantize_groups(ck, pk[:, 0], pk[:, 1])
+            v_hat[t, h] = dequantize_groups(cv, pv[:, 0], pv[:, 1])
+            at += card_record_bytes(d, w)
+        if w in (2, 4, 8) and hd["k_rotated"]:
+            k_hat[t] = rotate_f32(k_hat[t:t + 1])[0]
+    return k_hat, v_hat

@@ -618,3 +618,111 @@ def test_block_image_of_another_class_or_shape_is_refused():
     bad = src.block_image(0).copy()
     bad[0] ^= 1                                                 # broken magic
     assert not dst.load_block_image(0, bad)
+
+
+# ---------------------------------------------------------------------------
+# the mixed-width card (per-token widths {2, 4, 8, FP16})
+# ---------------------------------------------------------------------------
+
+def test_code_packing_generalises_the_nibble_order():
+    rng = np.random.default_rng(21)
+    c4 = rng.integers(0, 16, (3, 128)).astype(np.uint8)
+    np.testing.assert_array_equal(O.pack_codes(c4, 4), O.pack_nibbles(c4))
+    assert O.pack_codes(np.array([[0, 1, 2, 3]], np.uint8), 2)[0, 0] == 0b11100100
+    for bits in (2, 4, 8):
+        c = rng.integers(0, 1 << bits, (5, 256)).astype(np.uint8)
+        np.testing.assert_array_equal(O.unpack_codes(O.pack_codes(c, bits), bits), c)
+
+
+def test_card_record_sizes():
+    # per (token, KV head): K and V codes plus an fp16 (s, z) pair per group, or two raw 16-bit rows
+    assert [O.card_record_bytes(128, w) for w in (2, 4, 8, 16)] == [80, 144, 272, 512]
+    assert [O.card_record_bytes(256, w) for w in (2, 4, 8, 16)] == [160, 288, 544, 1024]
+    assert O.card_record_bytes(128, 3) == 0
+    offs, w_at, o_at, p_at, total = O.card_layout(128, 8, [2, 16, 4, 8, 5])
+    assert list(offs) == [0, 640, 640 + 4096, 640 + 4096 + 1152, 640 + 4096 + 1152 + 2176,
+                          640 + 4096 + 1152 + 2176]
+    assert (w_at, o_at, p_at) == (64, 80, 128) and total == 128 + offs[-1]
+
+
+def test_card_2bit_ramp_closed_form():
+    x = np.zeros((1, 1, 128), np.float32)
+    x[0, 0, :64] = np.arange(64)                 # s = 63 / 3 = 21, z = 0
+    x[0, 0, 64:] = np.arange(64) * 0.5 - 7.0     # s = 31.5 / 3 = 10.5, z = -7
+    card = O.card_encode(x.astype(np.float16), x.astype(np.float16), "fp16", [2], k_rotated=False)
+    p_at = O.card_layout(128, 1, [2])[3]
+    assert p_at == 64 + 16 + 16                  # header, one width byte, two offsets (each padded to 16)
+    rec = card[p_at:p_at + 80]
+    codes_v = O.unpack_codes(rec[32:64], 2)
+    np.testing.assert_array_equal(codes_v[:64], np.floor(np.arange(64) / 21.0 + 0.5))
+    np.testing.assert_array_equal(codes_v[64:], np.floor(np.arange(64) * 0.5 / 10.5 + 0.5))
+    par = rec[64 + 8:80].view(np.float16)        # V (s, z) of both groups
+    np.testing.assert_array_equal(par, np.array([21.0, 0.0, 10.5, -7.0], np.float16))
+
+
+def test_card_4_and_8_bit_records_are_the_pool_encoding():
+    rng = np.random.default_rng(23)
+    n, hkv, d = 256, 2, 128
+    k = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    v = rng.standard_normal((n, hkv, d)).astype(np.float16)
+    widths = rng.choice([4, 8], n)
+    card = O.card_encode(k, v, "fp16", widths)
+    offs, _, _, p_at, _ = O.card_layout(d, hkv, widths)
+    pool = O.OraclePool(hkv, d, 1, 1)
+    pool.quantize_blocks(k, v, "fp16", [0])
+    pool.quantize_blocks(k, v, "fp16", [1])
+    for t in range(n):
+        w, at = int(widths[t]), p_at + int(offs[t])
+        blk = 0 if w == 4 else 1
+        for h in range(hkv):
+            rec = card[at:at + O.card_record_bytes(d, w)]
+            cb = d * w // 8
+            kc = pool.codes4["k"][0, h, t] if w == 4 else pool.codes8["k"][0, h, t]
+            vc = pool.codes4["v"][0, h, t] if w == 4 else pool.codes8["v"][0, h, t]
+            kp = (pool.params4 if w == 4 else pool.params8)["k"][0, h, t]
+            vp = (pool.params4 if w == 4 else pool.params8)["v"][0, h, t]
+            np.testing.assert_array_equal(rec[:cb], kc)
+            np.testing.assert_array_equal(rec[cb:2 * cb], vc)
+            np.testing.assert_array_equal(rec[2 * cb:].view(np.uint16),
+                                          np.concatenate([kp.reshape(-1), vp.reshape(-1)]).view(np.uint16))
+            at += O.card_record_bytes(d, w)
+        assert blk in (0, 1)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_card_round_trip_bounds(dtype):
+    rng = np.random.default_rng(29)
+    n, hkv, d = 64, 2, 256
+    kf = (rng.standard_normal((n, hkv, d)) * 3).astype(np.float32)
+    vf = (rng.standard_normal((n, hkv, d)) * 3).astype(np.float32)
+    if dtype == "fp16":
+        k, v = kf.astype(np.float16), vf.astype(np.float16)
+    else:   # bf16 as raw bits (truncated fp32 is an exact bf16 value)
+        k = (kf.view(np.uint32) >> 16).astype(np.uint16)
+        v = (vf.view(np.uint32) >> 16).astype(np.uint16)
+    x_k, x_v = O.to_f32(k, dtype), O.to_f32(v, dtype)
+    widths = np.array([(2, 4, 8, 16, 7)[t % 5] for t in range(n)])
+    card = O.card_encode(k, v, dtype, widths)
+    hd = O.card_header(card)
+    assert hd["magic"] == b"QKVC" and hd["n_tokens"] == n and hd["raw_dtype"] == (0 if dtype == "fp16" else 1)
+    k_hat, v_hat = O.card_decode(card)
+    for t in range(n):
+        w = int(widths[t])
+        if w == 16:
+            np.testing.assert_array_equal(k_hat[t], x_k[t])
+            np.testing.assert_array_equal(v_hat[t], x_v[t])
+            continue
+        if w == 7:
+            assert not k_hat[t].any() and not v_hat[t].any()
+            continue
+        L = (1 << w) - 1
+        g = x_v[t].reshape(hkv, d // 64, 64)
+        s = (g.max(-1) - g.min(-1)) / L
+        bound = 0.5 * s + L * s * 2.0 ** -10 + np.abs(g.min(-1)) * 2.0 ** -10 + 1e-6
+        err = np.abs(v_hat[t] - x_v[t]).reshape(hkv, d // 64, 64).max(-1)
+        assert (err <= bound).all(), (w, err.max(), bound.min())
+        # keys: the rotation is orthonormal, so the l2 error stays within the rotated one's bound
+        kr = O.rotate_f32(x_k[t:t + 1])[0].reshape(hkv, d // 64, 64)
+        sk = (kr.max(-1) - kr.min(-1)) / L
+        lim = np.sqrt(64 * ((0.5 * sk + L * sk * 2.0 ** -10 + np.abs(kr.min(-1)) * 2.0 ** -10) ** 2).sum(-1))
+        assert (np.linalg.norm(k_hat[t] - x_k[t], axis=-1) <= lim * 1.001 + 1e-4).all()
