@@ -391,6 +391,7 @@ def run_gpu(args):
     gen_ms = statistics.median(a.elapsed_time(c) for a, _, c in gen)
 
     paging = measure_paging(job, dev, reps, d_cold_ms)
+    card = measure_card(job, dev, reps) if not args.fp8 else None
 
     e2e = run_e2e(job, args, dev, world) if not args.no_e2e else None
     if world > 1:
@@ -442,6 +443,7 @@ def run_gpu(args):
                            "append_then_decode_us": round(gen_ms * 1e3, 2),
                            "note": "one new token per sequence written over its last slot, then decode"},
                 "paging": paging,
+                "card": card,
             },
             "roofline": roof,
             "gpu_launches": job.launches_per_layer * job.n_layers * args.steps,
@@ -455,6 +457,45 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_card(job, dev, reps):
+    """Per-token mixed widths {2, 4, 8, FP16} (the synthetic mix of
+    workloads.CARD_WIDTH_MIX): encode the first layer's tokens into one card
+    and rebuild fp16 K/V from it.  Algorithmic bytes: encode reads K/V and
+    writes the card; decode reads the card and writes K/V."""
+    import torch
+    import decode_attention_q4kv_b200 as q4
+    from decode_attention_q4kv_b200 import workloads as W
+    L = job.layers[0]
+    k, v = L["k"], L["v"]
+    n, hkv, d = k.shape
+    widths = W.token_widths(n, job.w.seed, device=dev)
+    card = q4.card_encode(k, v, widths)
+    torch.cuda.synchronize()
+    payload = int(card[32:40].cpu().numpy().view("<i8")[0])
+    card_bytes = 64 + (n + 15) // 16 * 16 + (8 * (n + 1) + 15) // 16 * 16 + payload
+    kv_bytes = 2 * n * hkv * d * k.element_size()
+
+    def timed(fn):
+        out = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            out.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in out)
+
+    enc_ms = timed(lambda: q4.card_encode(k, v, widths))
+    dec_ms = timed(lambda: q4.card_decode(card, n, hkv, d, out_dtype=torch.float16))
+    counts = {int(w_): int((widths == w_).sum()) for w_ in (2, 4, 8, 16)}
+    return {"tokens": n, "width_counts": counts, "card_bytes": card_bytes,
+            "bits_per_value": round(8 * payload / (2 * n * hkv * d), 3),
+            "encode_us": round(enc_ms * 1e3, 1), "encode_gbps": round((kv_bytes + card_bytes) / (enc_ms * 1e-3) / 1e9, 1),
+            "decode_us": round(dec_ms * 1e3, 1), "decode_gbps": round((kv_bytes + card_bytes) / (dec_ms * 1e-3) / 1e9, 1),
+            "note": "card = per-token widths {2,4,8,FP16}; decode rebuilds fp16 K/V"}
 
 
 def measure_paging(job, dev, reps, decode_ms):

@@ -241,6 +241,42 @@ class Q4KVPool:
         return int(bits.value)
 
 
+def card_max_bytes(head_dim: int, n_kv_heads: int, n_tokens: int) -> int:
+    out = ctypes.c_size_t(0)
+    check(lib().q4kv_card_max_bytes(head_dim, n_kv_heads, n_tokens, ctypes.byref(out)), "q4kv_card_max_bytes")
+    return int(out.value)
+
+
+def card_encode(k: torch.Tensor, v: torch.Tensor, widths: torch.Tensor, k_rotated: bool = True,
+                error_word: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Card (device uint8) of K/V [n][Hkv][D] at per-token widths {2, 4, 8, 16}."""
+    dev = _require_cuda(k, v, widths)
+    if k.dtype != v.dtype or k.dtype not in _IN_DTYPES or k.shape != v.shape or k.dim() != 3:
+        raise ValueError("k and v must be [n][Hkv][D] of one dtype, float16 or bfloat16")
+    if k.stride() != v.stride() or k.stride(2) != 1 or k.stride(1) != k.shape[2]:
+        raise ValueError("each token's [Hkv][D] row must be contiguous, with equal strides for k and v")
+    n, hkv, d = k.shape
+    w = widths.to(torch.uint8).contiguous()
+    card = torch.empty(card_max_bytes(d, hkv, n), dtype=torch.uint8, device=dev)
+    check(lib().q4kv_card_encode(d, hkv, int(k_rotated), _ptr(k), _ptr(v), _IN_DTYPES[k.dtype], n, k.stride(0),
+                                 _ptr(w), _ptr(card), card.numel(), _ptr(error_word), _stream(dev)),
+          "q4kv_card_encode")
+    return card
+
+
+def card_decode(card: torch.Tensor, n_tokens: int, n_kv_heads: int, head_dim: int, out_dtype=torch.float32,
+                error_word: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """K_hat, V_hat [n][Hkv][D] rebuilt from a card."""
+    dev = _require_cuda(card)
+    shape = (n_tokens, n_kv_heads, head_dim)
+    k = torch.empty(shape, dtype=out_dtype, device=dev)
+    v = torch.empty(shape, dtype=out_dtype, device=dev)
+    check(lib().q4kv_card_decode(_ptr(card), card.numel(), head_dim, n_kv_heads, n_tokens, _ptr(k), _ptr(v),
+                                 _OUT_DTYPES[out_dtype], _ptr(error_word), _stream(dev)),
+          "q4kv_card_decode")
+    return k, v
+
+
 def _check_images(images: torch.Tensor, n: int, stride: int) -> None:
     if images.device.type != "cpu" or not images.is_pinned():
         raise ValueError("block images live in pinned host memory")
@@ -319,4 +355,4 @@ def decode_attention(pool: Q4KVPool, q: torch.Tensor, block_tables: torch.Tensor
 
 
 __all__ = ["Q4KVPool", "Q4KVError", "DecodePlan", "decode_attention", "block_absmean",
-           "mixed_block_ids", "BLOCK_TOKENS", "GROUP"]
+           "mixed_block_ids", "card_max_bytes", "card_encode", "card_decode", "BLOCK_TOKENS", "GROUP"]

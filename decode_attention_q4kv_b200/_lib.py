@@ -19,7 +19,7 @@ HEADER = os.path.join(_build.INCLUDE, "q4kv.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_DEVICE = range(6)
 F16, BF16, F32 = 0, 1, 2
-DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT_ID, DEVERR_TIMEOUT, DEVERR_IMAGE = 1, 2, 4, 8, 16
+DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT_ID, DEVERR_TIMEOUT, DEVERR_IMAGE, DEVERR_WIDTH = 1, 2, 4, 8, 16, 32
 
 
 class PoolDesc(ctypes.Structure):
@@ -51,6 +51,11 @@ _SIGNATURES = {
     "q4kv_block_image_stride": (c_int32, [P(PoolDesc), P(c_size_t)]),
     "q4kv_export_blocks": (c_int32, [P(PoolDesc), c_void_p, c_int32, c_void_p, c_void_p]),
     "q4kv_import_blocks": (c_int32, [P(PoolDesc), c_void_p, c_void_p, c_int32, c_void_p]),
+    "q4kv_card_max_bytes": (c_int32, [c_int32, c_int32, c_int64, P(c_size_t)]),
+    "q4kv_card_encode": (c_int32, [c_int32, c_int32, c_int32, c_void_p, c_void_p, c_int32, c_int64, c_int64,
+                                   c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "q4kv_card_decode": (c_int32, [c_void_p, c_size_t, c_int32, c_int32, c_int64, c_void_p, c_void_p, c_int32,
+                                   c_void_p, c_void_p]),
     "q4kv_export_blocks_host_ids": (c_int32, [P(PoolDesc), c_void_p, c_int32, c_void_p, c_void_p]),
     "q4kv_import_blocks_host_ids": (c_int32, [P(PoolDesc), c_void_p, c_void_p, c_int32, c_void_p]),
     "q4kv_dequantize": (c_int32, [P(PoolDesc), c_void_p, c_int32, c_void_p, c_void_p, c_int32,

@@ -189,6 +189,52 @@ q4kv_status q4kv_import_blocks_host_ids(const q4kv_pool* pool, const void* host_
   return from_cuda(copy_pages(v, block_ids, n_blocks, img, false, as_stream(stream)));
 }
 
+q4kv_status q4kv_card_max_bytes(int32_t head_dim, int32_t n_kv_heads, int64_t n_tokens, size_t* bytes) {
+  if (bytes == nullptr || n_kv_heads < 1 || n_tokens < 0 || n_tokens > (int64_t{1} << 31))
+    return Q4KV_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return Q4KV_ERR_UNSUPPORTED;
+  *bytes = static_cast<size_t>(card_max_bytes(head_dim, n_kv_heads, n_tokens));
+  return Q4KV_OK;
+}
+
+q4kv_status q4kv_card_encode(int32_t head_dim, int32_t n_kv_heads, int32_t k_rotated, const void* k,
+                             const void* v, int32_t in_dtype, int64_t n_tokens, int64_t token_stride,
+                             const uint8_t* widths, void* card, size_t card_bytes, uint32_t* error_word,
+                             void* stream) {
+  size_t need = 0;
+  q4kv_status st = q4kv_card_max_bytes(head_dim, n_kv_heads, n_tokens, &need);
+  if (st != Q4KV_OK) return st;
+  if (k_rotated != 0 && k_rotated != 1) return Q4KV_ERR_INVALID_ARG;
+  st = check_input(k, in_dtype, n_tokens, token_stride, n_kv_heads, head_dim);
+  if (st != Q4KV_OK) return st;
+  st = check_input(v, in_dtype, n_tokens, token_stride, n_kv_heads, head_dim);
+  if (st != Q4KV_OK) return st;
+  if ((n_tokens > 0 && widths == nullptr) || card == nullptr || !aligned(card, 16) || card_bytes < need ||
+      (error_word != nullptr && !aligned(error_word, 4)))
+    return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_card_encode(head_dim, n_kv_heads, k_rotated, k, v, in_dtype, n_tokens, token_stride,
+                                      widths, static_cast<uint8_t*>(card), error_word, as_stream(stream)));
+}
+
+q4kv_status q4kv_card_decode(const void* card, size_t card_bytes, int32_t head_dim, int32_t n_kv_heads,
+                             int64_t n_tokens, void* k_out, void* v_out, int32_t out_dtype, uint32_t* error_word,
+                             void* stream) {
+  size_t least = 0;
+  q4kv_status st = q4kv_card_max_bytes(head_dim, n_kv_heads, 0, &least);
+  if (st != Q4KV_OK) return st;
+  if (n_tokens < 0 || n_tokens > (int64_t{1} << 31)) return Q4KV_ERR_INVALID_ARG;
+  if (out_dtype != Q4KV_F32 && out_dtype != Q4KV_F16) return Q4KV_ERR_INVALID_ARG;
+  if (error_word != nullptr && !aligned(error_word, 4)) return Q4KV_ERR_INVALID_ARG;
+  if (n_tokens == 0) return Q4KV_OK;
+  const size_t tables = static_cast<size_t>((n_tokens + 15) / 16 * 16 + (8 * (n_tokens + 1) + 15) / 16 * 16);
+  if (card == nullptr || !aligned(card, 16) || card_bytes < least + tables || k_out == nullptr ||
+      v_out == nullptr || !aligned(k_out, 16) || !aligned(v_out, 16))
+    return Q4KV_ERR_INVALID_ARG;
+  return from_cuda(launch_card_decode(head_dim, n_kv_heads, static_cast<const uint8_t*>(card),
+                                      static_cast<int64_t>(card_bytes), n_tokens, k_out, v_out, out_dtype,
+                                      error_word, as_stream(stream)));
+}
+
 q4kv_status q4kv_selftest_bounded_wait(uint32_t* error_word, int32_t tries, void* stream) {
   if (error_word == nullptr || !aligned(error_word, 4) || tries < 1 || tries > (1 << 21))
     return Q4KV_ERR_INVALID_ARG;

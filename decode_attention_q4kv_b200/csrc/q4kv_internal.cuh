@@ -116,6 +116,13 @@ cudaError_t launch_append(const PoolView& pool, const void* k, const void* v, in
                           int64_t token_stride, const int32_t* tables, int32_t max_blocks,
                           const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_selftest_wait(uint32_t* error_word, unsigned tries, cudaStream_t stream);
+// Per-token mixed-width cards (quantize.cu).
+int64_t card_max_bytes(int d, int hkv, int64_t n);
+cudaError_t launch_card_encode(int d, int hkv, int k_rotated, const void* k, const void* v, int in_dtype,
+                               int64_t n, int64_t stride, const uint8_t* widths, uint8_t* card,
+                               uint32_t* error_word, cudaStream_t stream);
+cudaError_t launch_card_decode(int d, int hkv, const uint8_t* card, int64_t card_bytes, int64_t n, void* k_out,
+                               void* v_out, int out_dtype, uint32_t* error_word, cudaStream_t stream);
 // Block images (paging.cu): stride of one image for this pool, and one
 // launch moving n blocks' images between the pool and host memory.
 int64_t image_stride_bytes(const PoolView& pool);

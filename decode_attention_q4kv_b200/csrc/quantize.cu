@@ -167,8 +167,8 @@ struct GroupParams {
 template <int BITS>
 __device__ __forceinline__ GroupParams group_params(const float2 (&x)[8], float xs) {
   constexpr int L = (1 << BITS) - 1;
-  // RN(1/L); 15 and 255 have 11-bit significands
-  constexpr float kRecipL = BITS == 4 ? 0x1.111112p-4f : 0x1.010102p-8f;
+  // RN(1/L); 3, 15 and 255 have significands of at most 11 bits
+  constexpr float kRecipL = BITS == 2 ? 0x1.555556p-2f : BITS == 4 ? 0x1.111112p-4f : 0x1.010102p-8f;
   float mn = min3(min3(min3(x[0].x, x[0].y, x[1].x), min3(x[1].y, x[2].x, x[2].y),
                        min3(x[3].x, x[3].y, x[4].x)),
                   min3(x[4].y, x[5].x, x[5].y), min3(x[6].x, x[6].y, min(x[7].x, x[7].y)));
@@ -244,7 +244,17 @@ template <int BITS>
 __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupParams& g, int j,
                                             uint8_t* __restrict__ code_dst,
                                             __half2* __restrict__ param_dst) {
-  if (BITS == 4) {
+  if (BITS == 2) {
+    // element e (pair e % 8, half e / 8) at bits 2e of the lane's word: four
+    // codes per byte, element 4i + m at bits 2m of byte i
+    uint32_t w = 0;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      w |= (__float_as_uint(c[p].x) & 3u) << (2 * p);
+      w |= (__float_as_uint(c[p].y) & 3u) << (2 * (p + 8));
+    }
+    *reinterpret_cast<uint32_t*>(code_dst + j * 4) = w;
+  } else if (BITS == 4) {
     // byte b holds elements 2b (low nibble) and 2b+1 (high nibble); the sums
     // are exact (integers below 2^24)
     uint32_t b[8];
@@ -634,7 +644,11 @@ __device__ __forceinline__ void decode_lane(const uint8_t* __restrict__ codes,
   const float s = __low2float(p);
   const float z = __high2float(p);
   uint32_t w[4];
-  if (BITS == 4) {
+  if (BITS == 2) {
+    w[0] = *reinterpret_cast<const uint32_t*>(codes + j * 4);
+#pragma unroll
+    for (int i = 0; i < kEPL; ++i) x[i] = __fmaf_rn(static_cast<float>((w[0] >> (2 * i)) & 3u), s, z);
+  } else if (BITS == 4) {
     const uint2 u = *reinterpret_cast<const uint2*>(codes + j * 8);
     w[0] = u.x;
     w[1] = u.y;
@@ -755,6 +769,260 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Per-token widths {2, 4, 8, FP16} in one cache: the card.  QKVShare
+// (gist.science summary of arXiv 2605.03884), "Méthodologie": every token
+// gets a width from {2, 4, 8, FP16}; the cache travels as a compact artifact
+// of quantised groups, per-token widths and metadata, and the receiver
+// rebuilds FP16 keys and values from it.  Layout (bytes): a 64-byte header,
+// the widths (one byte per token, padded to 16), the int64 offset of every
+// token's record from the payload start plus the total (padded to 16), then
+// the records.  Record of (token, KV head h) at width w: K codes (D w / 8
+// bytes), V codes, K (s, z) pairs, V (s, z) pairs -- the pool's group coding
+// with L = 2^w - 1 -- or, at w = 16, the raw K row and V row.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kCardMagic = 0x43564B51u;   // bytes 'Q', 'K', 'V', 'C'
+constexpr int kCardHeader = 64;
+constexpr int kCardScanThreads = 1024;
+constexpr int kCardScanPer = 8;                // tokens per thread per round of the scan
+
+__host__ __device__ inline int64_t card_record_bytes(int d, int w) {
+  if (w == 16) return 4 * d;
+  if (w == 2 || w == 4 || w == 8) return 2 * (d * w / 8 + (d / kGroup) * 4);
+  return 0;
+}
+__host__ __device__ inline int64_t round16(int64_t x) { return (x + 15) / 16 * 16; }
+
+// One CTA: copies the widths into the card, writes every token's record
+// offset (an exclusive scan of Hkv * record bytes, in rounds of 8192 tokens)
+// and the header.  A width outside {2, 4, 8, 16} takes no bytes and raises
+// Q4KV_DEVERR_WIDTH.
+__global__ void __launch_bounds__(kCardScanThreads) card_layout_kernel(const uint8_t* __restrict__ widths,
+                                                                       int64_t n, int d, int hkv, int k_rotated,
+                                                                       int raw_dtype, uint8_t* card,
+                                                                       uint32_t* error_word) {
+  __shared__ int64_t warp_sums[kCardScanThreads / 32];
+  __shared__ int64_t carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint8_t* wdst = card + kCardHeader;
+  int64_t* offs = reinterpret_cast<int64_t*>(card + kCardHeader + round16(n));
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < n; base += static_cast<int64_t>(kCardScanThreads) * kCardScanPer) {
+    const int64_t t0 = base + static_cast<int64_t>(threadIdx.x) * kCardScanPer;
+    int64_t sz[kCardScanPer], sum = 0;
+#pragma unroll
+    for (int i = 0; i < kCardScanPer; ++i) {
+      sz[i] = 0;
+      if (t0 + i < n) {
+        const int w = widths[t0 + i];
+        wdst[t0 + i] = static_cast<uint8_t>(w);
+        sz[i] = hkv * card_record_bytes(d, w);
+        if (sz[i] == 0) raise_error(error_word, Q4KV_DEVERR_WIDTH);
+      }
+      sum += sz[i];
+    }
+    int64_t incl = sum;   // inclusive scan of the thread sums: warp, then across warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int64_t ws = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += y;
+      }
+      warp_sums[lane] = ws;   // inclusive over warps
+    }
+    __syncthreads();
+    int64_t run = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - sum;
+#pragma unroll
+    for (int i = 0; i < kCardScanPer; ++i) {
+      if (t0 + i < n) offs[t0 + i] = run;
+      run += sz[i];
+    }
+    __syncthreads();
+    if (threadIdx.x == kCardScanThreads - 1) carry = run;   // the last thread ends the round
+    __syncthreads();
+  }
+  // padding after the widths and after the offsets is zero, so a card's bytes
+  // depend on its contents only
+  if (threadIdx.x < 16 && n + threadIdx.x < round16(n)) wdst[n + threadIdx.x] = 0;
+  if (threadIdx.x < 16 && 8 * (n + 1) + threadIdx.x < round16(8 * (n + 1)))
+    reinterpret_cast<uint8_t*>(offs)[8 * (n + 1) + threadIdx.x] = 0;
+  if (threadIdx.x == 0) {
+    offs[n] = carry;
+    uint32_t* h = reinterpret_cast<uint32_t*>(card);
+    h[0] = kCardMagic;
+    h[1] = 1;   // version
+    h[2] = static_cast<uint32_t>(d);
+    h[3] = static_cast<uint32_t>(hkv);
+    h[4] = static_cast<uint32_t>(n & 0xFFFFFFFF);
+    h[5] = static_cast<uint32_t>(n >> 32);
+    h[6] = static_cast<uint32_t>(k_rotated);
+    h[7] = static_cast<uint32_t>(raw_dtype);
+    *reinterpret_cast<int64_t*>(card + 32) = carry;
+    for (int i = 40; i < kCardHeader; i += 4) *reinterpret_cast<uint32_t*>(card + i) = 0;
+  }
+}
+
+__host__ __device__ inline int64_t card_payload_at(int64_t n) {
+  return kCardHeader + round16(n) + round16(8 * (n + 1));
+}
+
+// Warp item = (token, VPW KV heads): every lane of a warp works on one token,
+// so its width is warp-uniform; the lane layout, rotation and coding are the
+// append kernel's.
+template <int D, typename InT>
+__global__ void __launch_bounds__(256) card_encode_kernel(const InT* __restrict__ k, const InT* __restrict__ v,
+                                                          int64_t n, int64_t stride, int hkv, int k_rotated,
+                                                          uint8_t* card) {
+  using S = Shape<D>;
+  const int lane = threadIdx.x & 31;
+  const int r = lane / S::LPV, j = lane % S::LPV;
+  const int hgroups = (hkv + S::VPW - 1) / S::VPW;
+  const int64_t* offs = reinterpret_cast<const int64_t*>(card + kCardHeader + round16(n));
+  uint8_t* payload = card + card_payload_at(n);
+  const int64_t n_items = n * hgroups;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; item < n_items;
+       item += n_warps) {
+    const int64_t t = item / hgroups;
+    const int hg = static_cast<int>(item % hgroups);
+    const int w = card[kCardHeader + t];
+    const int64_t rec = card_record_bytes(D, w);
+    if (rec == 0) continue;   // warp-uniform; reported by the layout kernel
+    const int h = hg * S::VPW + r;
+    const bool valid = h < hkv;
+    const int hs = valid ? h : hkv - 1;   // lanes past the last head read a real row, store nothing
+    const int64_t src = t * stride + static_cast<int64_t>(hs) * D + j * kEPL;
+    const uint4 k0 = __ldg(reinterpret_cast<const uint4*>(k + src));
+    const uint4 k1 = __ldg(reinterpret_cast<const uint4*>(k + src) + 1);
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(v + src));
+    const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(v + src) + 1);
+    uint8_t* dst = payload + offs[t] + static_cast<int64_t>(hs) * rec;
+    if (w == 16) {   // raw 16-bit rows
+      if (valid) {
+        uint4* kd = reinterpret_cast<uint4*>(dst + j * 32);
+        uint4* vd = reinterpret_cast<uint4*>(dst + 2 * D + j * 32);
+        kd[0] = k0;
+        kd[1] = k1;
+        vd[0] = v0;
+        vd[1] = v1;
+      }
+      continue;
+    }
+    float2 xk[8], xv[8];
+    unpack16<InT>(k0, k1, xk);
+    unpack16<InT>(v0, v1, xv);
+    float ks = 1.0f;
+    if (k_rotated) {   // warp-uniform
+      rotate_pairs<D>(xk, j);
+      ks = kRotScale<D>;
+    }
+    const int64_t cb = D * w / 8;
+    __half2* kp = reinterpret_cast<__half2*>(dst + 2 * cb);
+    __half2* vp = kp + S::NG;
+    if (w == 2) encode_kv<2>(xk, ks, xv, j, valid, dst, kp, dst + cb, vp);
+    else if (w == 4) encode_kv<4>(xk, ks, xv, j, valid, dst, kp, dst + cb, vp);
+    else encode_kv<8>(xk, ks, xv, j, valid, dst, kp, dst + cb, vp);
+  }
+}
+
+// Card -> K_hat, V_hat [n][Hkv][D]: x_hat = fl(code s + z), K un-rotated when
+// the card stores it rotated; FP16 tokens convert exactly; a token of an
+// invalid width reads 0.  The header must describe (D, Hkv, n) and every
+// record must lie inside the card's `card_bytes`, else the rows read 0 and
+// Q4KV_DEVERR_IMAGE is raised: a damaged card is never read out of bounds.
+__device__ __forceinline__ float raw16_to_float(uint16_t b, bool bf16) {
+  return bf16 ? __uint_as_float(static_cast<uint32_t>(b) << 16) : __half2float(__ushort_as_half(b));
+}
+
+template <int D, typename OutT>
+__global__ void __launch_bounds__(256) card_decode_kernel(const uint8_t* card, int64_t card_bytes, int64_t n,
+                                                          int hkv, OutT* __restrict__ k_out,
+                                                          OutT* __restrict__ v_out, uint32_t* error_word) {
+  using S = Shape<D>;
+  const int lane = threadIdx.x & 31;
+  const int r = lane / S::LPV, j = lane % S::LPV;
+  const int hgroups = (hkv + S::VPW - 1) / S::VPW;
+  const uint32_t* hdr = reinterpret_cast<const uint32_t*>(card);
+  const bool header_ok = hdr[0] == kCardMagic && hdr[1] == 1u && hdr[2] == static_cast<uint32_t>(D) &&
+                         hdr[3] == static_cast<uint32_t>(hkv) &&
+                         (static_cast<int64_t>(hdr[5]) << 32 | hdr[4]) == n;
+  const bool k_rotated = hdr[6] != 0, raw_bf16 = hdr[7] != 0;
+  const uint8_t* widths = card + kCardHeader;
+  const int64_t* offs = reinterpret_cast<const int64_t*>(card + kCardHeader + round16(n));
+  const uint8_t* payload = card + card_payload_at(n);
+  const int64_t room = card_bytes - card_payload_at(n);
+  const int64_t n_items = n * hgroups;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; item < n_items;
+       item += n_warps) {
+    const int64_t t = item / hgroups;
+    const int hg = static_cast<int>(item % hgroups);
+    const int h = hg * S::VPW + r;
+    const bool valid = h < hkv;
+    const int hs = valid ? h : hkv - 1;
+    OutT* kd = k_out + (t * hkv + hs) * D + j * kEPL;
+    OutT* vd = v_out + (t * hkv + hs) * D + j * kEPL;
+    int w = 0;
+    int64_t rec = 0, off = 0;
+    if (header_ok) {
+      w = widths[t];
+      rec = card_record_bytes(D, w);
+      off = offs[t];
+      if (rec != 0 && (off < 0 || off + hkv * rec > room)) {   // warp-uniform
+        if (lane == 0) raise_error(error_word, Q4KV_DEVERR_IMAGE);
+        rec = 0;
+      }
+    } else if (item == 0 && lane == 0) {
+      raise_error(error_word, Q4KV_DEVERR_IMAGE);
+    }
+    const uint8_t* src = payload + off + static_cast<int64_t>(hs) * rec;
+    float xk[kEPL], xv[kEPL];
+    if (rec == 0) {
+#pragma unroll
+      for (int i = 0; i < kEPL; ++i) xk[i] = xv[i] = 0.0f;
+    } else if (w == 16) {
+      const uint4* rk = reinterpret_cast<const uint4*>(src + j * 32);
+      const uint4* rv = reinterpret_cast<const uint4*>(src + 2 * D + j * 32);
+      const uint4 a[2] = {rk[0], rk[1]}, b[2] = {rv[0], rv[1]};
+      const uint16_t* ka = reinterpret_cast<const uint16_t*>(a);
+      const uint16_t* vb = reinterpret_cast<const uint16_t*>(b);
+#pragma unroll
+      for (int i = 0; i < kEPL; ++i) {
+        xk[i] = raw16_to_float(ka[i], raw_bf16);
+        xv[i] = raw16_to_float(vb[i], raw_bf16);
+      }
+    } else {
+      const int64_t cb = D * w / 8;
+      const __half2* kp = reinterpret_cast<const __half2*>(src + 2 * cb);
+      const __half2* vp = kp + S::NG;
+      if (w == 2) {
+        decode_lane<2>(src, kp, j, xk);
+        decode_lane<2>(src + cb, vp, j, xv);
+      } else if (w == 4) {
+        decode_lane<4>(src, kp, j, xk);
+        decode_lane<4>(src + cb, vp, j, xv);
+      } else {
+        decode_lane<8>(src, kp, j, xk);
+        decode_lane<8>(src + cb, vp, j, xv);
+      }
+      if (k_rotated) rotate_vector<D>(xk, j);   // warp-uniform
+    }
+    if (valid) {
+      store16<OutT>(kd, xk);
+      store16<OutT>(vd, xv);
+    }
+  }
+}
+
 inline int grid_for(int64_t n_items) {
   const int64_t warps_per_cta = 8;
   int64_t g = (n_items + warps_per_cta - 1) / warps_per_cta;
@@ -852,6 +1120,47 @@ cudaError_t launch_append(const PoolView& pool, const void* k, const void* v, in
   Q4KV_LAUNCH_AR(256, __nv_bfloat16)
 #undef Q4KV_LAUNCH_AR
 #undef Q4KV_LAUNCH_A
+}
+
+int64_t card_max_bytes(int d, int hkv, int64_t n) { return card_payload_at(n) + n * hkv * 4 * d; }
+
+cudaError_t launch_card_encode(int d, int hkv, int k_rotated, const void* k, const void* v, int in_dtype,
+                               int64_t n, int64_t stride, const uint8_t* widths, uint8_t* card,
+                               uint32_t* error_word, cudaStream_t stream) {
+  card_layout_kernel<<<1, kCardScanThreads, 0, stream>>>(widths, n, d, hkv, k_rotated, in_dtype == Q4KV_BF16,
+                                                         card, error_word);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || n == 0) return e;
+  const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;
+  const int64_t items = n * ((hkv + vpw - 1) / vpw);
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+  int64_t g = (items + 7) / 8;
+  if (g > static_cast<int64_t>(sms) * 8) g = static_cast<int64_t>(sms) * 8;
+#define Q4KV_CARD_E(DD, T)                                                                            \
+  card_encode_kernel<DD, T><<<static_cast<unsigned>(g), 256, 0, stream>>>(                          \
+      static_cast<const T*>(k), static_cast<const T*>(v), n, stride, hkv, k_rotated, card)
+  if (d == 128 && in_dtype == Q4KV_F16) Q4KV_CARD_E(128, __half);
+  else if (d == 128) Q4KV_CARD_E(128, __nv_bfloat16);
+  else if (in_dtype == Q4KV_F16) Q4KV_CARD_E(256, __half);
+  else Q4KV_CARD_E(256, __nv_bfloat16);
+#undef Q4KV_CARD_E
+  return cudaGetLastError();
+}
+
+cudaError_t launch_card_decode(int d, int hkv, const uint8_t* card, int64_t card_bytes, int64_t n, void* k_out,
+                               void* v_out, int out_dtype, uint32_t* error_word, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;
+  const dim3 grid(grid_for(n * ((hkv + vpw - 1) / vpw))), block(256);
+#define Q4KV_CARD_D(DD, T)                                                                            \
+  card_decode_kernel<DD, T><<<grid, block, 0, stream>>>(card, card_bytes, n, hkv, static_cast<T*>(k_out), \
+                                                        static_cast<T*>(v_out), error_word)
+  if (d == 128 && out_dtype == Q4KV_F32) Q4KV_CARD_D(128, float);
+  else if (d == 128) Q4KV_CARD_D(128, __half);
+  else if (out_dtype == Q4KV_F32) Q4KV_CARD_D(256, float);
+  else Q4KV_CARD_D(256, __half);
+#undef Q4KV_CARD_D
+  return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const PoolView& pool, const int32_t* block_ids, int32_t n_blocks,

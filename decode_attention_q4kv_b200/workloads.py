@@ -36,6 +36,12 @@ STREAM_Q = 2
 STREAM_OUTLIER = 3
 STREAM_EVICT = 4
 STREAM_PERM = 5
+STREAM_WIDTH = 6
+
+# Share of tokens at each width {2, 4, 8, 16} for a mixed-width card.  QKVShare
+# assigns widths per token from {2, 4, 8, FP16} with a learned controller and
+# reports no distribution; this fixed synthetic mix stands in for it.
+CARD_WIDTH_MIX = ((2, 0.25), (4, 0.45), (8, 0.20), (16, 0.10))
 
 _MASK64 = (1 << 64) - 1
 
@@ -266,3 +272,14 @@ def random_small(n_tokens: int, n_kv_heads: int, head_dim: int, dtype: str,
     v = normal(shape, seed, layer, STREAM_V, device) * scale
     dt = torch_dtype(dtype)
     return k.to(dt).contiguous(), v.to(dt).contiguous()
+
+
+def token_widths(n_tokens: int, seed: int, layer: int = 0, device="cpu",
+                 mix=CARD_WIDTH_MIX) -> torch.Tensor:
+    """uint8 [n_tokens] widths drawn independently from `mix` (seeded)."""
+    g = generator(seed, layer, STREAM_WIDTH, "cpu")
+    values = torch.tensor([w for w, _ in mix], dtype=torch.uint8)
+    probs = torch.tensor([p for _, p in mix], dtype=torch.float64)
+    idx = torch.multinomial(probs, n_tokens, replacement=True, generator=g) if n_tokens else \
+        torch.zeros(0, dtype=torch.int64)
+    return values[idx].to(device)

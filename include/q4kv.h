@@ -88,7 +88,8 @@ typedef enum {
 #define Q4KV_DEVERR_SEQ_LEN 2u   /* seq_len < 0 or > max_blocks_per_seq * 256 */
 #define Q4KV_DEVERR_SLOT_ID 4u   /* a slot id outside [0, 256 * (n_q4_blocks + n_q8_blocks)) */
 #define Q4KV_DEVERR_TIMEOUT 8u   /* a bounded device-side wait gave up */
-#define Q4KV_DEVERR_IMAGE 16u    /* a block image whose header does not fit its target block */
+#define Q4KV_DEVERR_IMAGE 16u    /* a block image or card whose header or layout does not fit */
+#define Q4KV_DEVERR_WIDTH 32u    /* a card token width outside {2, 4, 8, 16} */
 
 typedef enum { Q4KV_F16 = 0, Q4KV_BF16 = 1, Q4KV_F32 = 2 } q4kv_dtype;
 
@@ -342,6 +343,64 @@ q4kv_status q4kv_decode_attention_static_scratch(const q4kv_pool *pool,
  * context stays usable; tests use it to check that waits end.
  */
 q4kv_status q4kv_selftest_bounded_wait(uint32_t *error_word, int32_t tries, void *stream);
+
+/*
+ * Per-token widths {2, 4, 8, FP16} in one cache: the card ([QKVS]
+ * "Méthodologie": each token gets a width from {2, 4, 8, FP16}; the cache
+ * travels as a compact artifact of quantised groups, per-token widths and
+ * metadata; the receiver rebuilds FP16 keys and values from it).
+ *
+ * Card layout (device memory, 16-byte aligned, little-endian):
+ *   header 64 B: uint32 magic 0x43564B51 ("QKVC"), uint32 version 1,
+ *     uint32 head_dim, uint32 n_kv_heads, uint64 n_tokens, uint32 k_rotated,
+ *     uint32 raw dtype of FP16 tokens (0 fp16, 1 bf16), int64 payload bytes,
+ *     zeros to 64
+ *   widths: one byte per token, padded to a multiple of 16
+ *   offsets: int64 [n_tokens + 1], byte offset of each token's record from
+ *     the payload start, then the payload size; padded to 16
+ *   payload: token records in order.  The record of token t is, for every KV
+ *     head in order: K codes (D*w/8 bytes), V codes, K (s, z) half2 pairs
+ *     (D/64), V pairs -- the pool's group coding with L = 2^w - 1 (w = 2: four
+ *     codes per byte, element 4i+m at bits 2m of byte i; w = 4: the nibble
+ *     order; w = 8: one per byte), K rotated when k_rotated -- or, for
+ *     w = 16, the raw K row then the raw V row (2*D bytes each, the input's
+ *     own 16-bit values).  Per (token, head): 80 / 144 / 272 / 512 bytes at
+ *     D = 128 for w = 2 / 4 / 8 / 16.
+ *
+ * q4kv_card_max_bytes: the card size when every token is FP16 (host-only);
+ * a card of that size always fits.
+ */
+q4kv_status q4kv_card_max_bytes(int32_t head_dim, int32_t n_kv_heads, int64_t n_tokens, size_t *bytes);
+
+/*
+ * Encode n_tokens tokens into a card.
+ *   k, v        as in q4kv_quantize_blocks (fp16 or bf16, token stride rules)
+ *   widths      device uint8 [n_tokens], each 2, 4, 8 or 16; any other value
+ *               gives the token no record and raises Q4KV_DEVERR_WIDTH
+ *   card        device, 16-byte aligned, card_bytes >= q4kv_card_max_bytes
+ *   k_rotated   1 = code keys after the Walsh-Hadamard rotation (as the pool
+ *               does); FP16 tokens are always stored raw
+ * Codes, scales and zeros are bit-identical to the pool's coding of the same
+ * row at that width.  The payload size is written into the header.
+ */
+q4kv_status q4kv_card_encode(int32_t head_dim, int32_t n_kv_heads, int32_t k_rotated, const void *k,
+                             const void *v, int32_t in_dtype, int64_t n_tokens, int64_t token_stride,
+                             const uint8_t *widths, void *card, size_t card_bytes, uint32_t *error_word,
+                             void *stream);
+
+/*
+ * Rebuild K and V from a card (the receiver's injection path of [QKVS]).
+ *   k_out, v_out  device [n_tokens][Hkv][D] of out_dtype (Q4KV_F32 or
+ *                 Q4KV_F16), 16-byte aligned.  x_hat = fl(code*s + z); keys
+ *                 coded rotated are un-rotated (c*H, bit-exact); FP16 tokens
+ *                 are their raw values; a token with an invalid width reads 0.
+ * The header must hold (head_dim, n_kv_heads, n_tokens) and every record must
+ * lie inside card_bytes; otherwise the affected rows read 0 and
+ * Q4KV_DEVERR_IMAGE is raised (a damaged card is never read out of bounds).
+ */
+q4kv_status q4kv_card_decode(const void *card, size_t card_bytes, int32_t head_dim, int32_t n_kv_heads,
+                             int64_t n_tokens, void *k_out, void *v_out, int32_t out_dtype,
+                             uint32_t *error_word, void *stream);
 
 /*
  * Block images: paging blocks between device and host memory ([AMBP] sec.

@@ -24,7 +24,7 @@ def _pool(**kw):
 
 def test_exports_every_declared_function():
     names = _lib.header_functions()
-    assert len(names) == 19
+    assert len(names) == 22
     for n in names:
         assert hasattr(L, n), n
     # the binding declares a signature for each of them
@@ -238,3 +238,39 @@ def test_paging_rejects_bad_arguments_without_launching():
         assert call(FAKE, 2, addr + 8) == _lib.ERR_INVALID_ARG          # misaligned images
         assert call(FAKE, 2, addr) == _lib.ERR_INVALID_ARG              # not page-locked
         assert call(FAKE, 0, None) == 0                                 # nothing to move
+
+
+@pytest.mark.parametrize("d,hkv,n", [(128, 8, 0), (128, 3, 301), (256, 2, 8195)])
+def test_card_max_bytes_is_the_all_fp16_card(d, hkv, n):
+    from oracle import q4kv_oracle as O
+    out = ctypes.c_size_t(0)
+    assert L.q4kv_card_max_bytes(d, hkv, n, ctypes.byref(out)) == 0
+    assert out.value == O.card_layout(d, hkv, [16] * n)[4]
+
+
+def test_card_calls_reject_bad_arguments_without_launching():
+    out = ctypes.c_size_t(0)
+    assert L.q4kv_card_max_bytes(64, 8, 10, ctypes.byref(out)) == _lib.ERR_UNSUPPORTED
+    assert L.q4kv_card_max_bytes(128, 0, 10, ctypes.byref(out)) == _lib.ERR_INVALID_ARG
+    assert L.q4kv_card_max_bytes(128, 8, -1, ctypes.byref(out)) == _lib.ERR_INVALID_ARG
+    L.q4kv_card_max_bytes(128, 8, 10, ctypes.byref(out))
+    big = out.value
+    enc = lambda **kw: L.q4kv_card_encode(*[dict(dict(d=128, h=8, rot=1, k=FAKE, v=FAKE, dt=0, n=10, ts=1024,
+                                                      w=FAKE, card=FAKE, cb=big, err=None, s=None), **kw)[x]
+                                            for x in ("d", "h", "rot", "k", "v", "dt", "n", "ts", "w", "card",
+                                                      "cb", "err", "s")])
+    assert enc(cb=big - 1) == _lib.ERR_INVALID_ARG            # card too small for the worst case
+    assert enc(card=FAKE + 8) == _lib.ERR_INVALID_ARG
+    assert enc(w=None) == _lib.ERR_INVALID_ARG
+    assert enc(rot=2) == _lib.ERR_INVALID_ARG
+    assert enc(dt=2) == _lib.ERR_INVALID_ARG
+    assert enc(ts=1000) == _lib.ERR_INVALID_ARG
+    assert enc(d=96) == _lib.ERR_UNSUPPORTED
+    assert enc(err=FAKE + 2) == _lib.ERR_INVALID_ARG
+    dec = L.q4kv_card_decode
+    assert dec(FAKE, big, 128, 8, 10, FAKE, FAKE, 1, None, None) == _lib.ERR_INVALID_ARG   # bf16 output
+    assert dec(FAKE, 100, 128, 8, 10, FAKE, FAKE, 2, None, None) == _lib.ERR_INVALID_ARG   # no room for tables
+    assert dec(FAKE + 4, big, 128, 8, 10, FAKE, FAKE, 2, None, None) == _lib.ERR_INVALID_ARG
+    assert dec(FAKE, big, 128, 8, 10, FAKE + 4, FAKE, 2, None, None) == _lib.ERR_INVALID_ARG
+    assert dec(FAKE, big, 128, 8, -1, FAKE, FAKE, 2, None, None) == _lib.ERR_INVALID_ARG
+    assert dec(None, 0, 128, 8, 0, None, None, 2, None, None) == 0                       # nothing to rebuild
