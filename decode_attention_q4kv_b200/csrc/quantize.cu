@@ -128,7 +128,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 constexpr float kRoundMagic = 12582912.0f;
 
 // Correctly rounded quotient RN(u / s) for a divisor s whose significand
-// has at most 11 bits (every fp16 value, and the constants 15 and 255), from
+// has at most 11 bits (every fp16 value, and the constants 3, 15 and 255), from
 // r = RN(1/s): q0 = RN(u r), the residual u - q0 s is exact under an FMA, and
 // one correction q1 = RN(q0 + (u - q0 s) r) gives RN(u / s).  This is
 // Markstein's correction step (P. Markstein, "Computation of elementary

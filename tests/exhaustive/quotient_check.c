@@ -1,5 +1,5 @@
 /* Exhaustive check of the encoder's quotient: for a divisor s whose
- * significand has at most 11 bits (every fp16 value; also 15 and 255) and any
+ * significand has at most 11 bits (every fp16 value; also 3, 15 and 255) and any
  * binary32 dividend u, Markstein's correction step
  *     r = RN(1/s), q0 = RN(u r), q1 = RN(q0 + RN(u - q0 s) r)   (FMAs)
  * gives q1 = RN(u / s).  All steps scale exactly with the exponents of u and
