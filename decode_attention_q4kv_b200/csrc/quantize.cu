@@ -783,8 +783,6 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
 // ---------------------------------------------------------------------------
 constexpr uint32_t kCardMagic = 0x43564B51u;   // bytes 'Q', 'K', 'V', 'C'
 constexpr int kCardHeader = 64;
-constexpr int kCardScanThreads = 1024;
-constexpr int kCardScanPer = 8;                // tokens per thread per round of the scan
 
 __host__ __device__ inline int64_t card_record_bytes(int d, int w) {
   if (w == 16) return 4 * d;
@@ -793,70 +791,94 @@ __host__ __device__ inline int64_t card_record_bytes(int d, int w) {
 }
 __host__ __device__ inline int64_t round16(int64_t x) { return (x + 15) / 16 * 16; }
 
-// One CTA: copies the widths into the card, writes every token's record
-// offset (an exclusive scan of Hkv * record bytes, in rounds of 8192 tokens)
-// and the header.  A width outside {2, 4, 8, 16} takes no bytes and raises
-// Q4KV_DEVERR_WIDTH.
-__global__ void __launch_bounds__(kCardScanThreads) card_layout_kernel(const uint8_t* __restrict__ widths,
-                                                                       int64_t n, int d, int hkv, int k_rotated,
-                                                                       int raw_dtype, uint8_t* card,
-                                                                       uint32_t* error_word) {
-  __shared__ int64_t warp_sums[kCardScanThreads / 32];
-  __shared__ int64_t carry;
+__host__ __device__ inline int64_t card_payload_at(int64_t n) {
+  return kCardHeader + round16(n) + round16(8 * (n + 1));
+}
+
+// The record offsets are an exclusive scan of Hkv * record bytes over the
+// tokens, done in three launches with no waiting between CTAs: per-chunk
+// sums (4096 tokens per CTA), one CTA scanning the chunk sums (which also
+// writes the header and the table's last entry and zeroes the padding),
+// then per-chunk scans from those bases, staged in shared memory so the
+// table is written with coalesced stores.  The chunk sums live in the card's
+// payload, which the encoder overwrites afterwards.  A width outside
+// {2, 4, 8, 16} takes no bytes and raises Q4KV_DEVERR_WIDTH.
+constexpr int kScanThreads = 256;
+constexpr int kScanPer = 16;                              // tokens per thread
+constexpr int kScanChunk = kScanThreads * kScanPer;       // tokens per CTA
+
+__device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* warp_sums, int64_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint8_t* wdst = card + kCardHeader;
-  int64_t* offs = reinterpret_cast<int64_t*>(card + kCardHeader + round16(n));
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int64_t base = 0; base < n; base += static_cast<int64_t>(kCardScanThreads) * kCardScanPer) {
-    const int64_t t0 = base + static_cast<int64_t>(threadIdx.x) * kCardScanPer;
-    int64_t sz[kCardScanPer], sum = 0;
+  int64_t incl = x;
 #pragma unroll
-    for (int i = 0; i < kCardScanPer; ++i) {
-      sz[i] = 0;
-      if (t0 + i < n) {
-        const int w = widths[t0 + i];
-        wdst[t0 + i] = static_cast<uint8_t>(w);
-        sz[i] = hkv * card_record_bytes(d, w);
-        if (sz[i] == 0) raise_error(error_word, Q4KV_DEVERR_WIDTH);
-      }
-      sum += sz[i];
-    }
-    int64_t incl = sum;   // inclusive scan of the thread sums: warp, then across warps
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int64_t w = lane < static_cast<int>(blockDim.x >> 5) ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+      const int64_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
     }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      int64_t ws = warp_sums[lane];
+    warp_sums[lane] = w;   // inclusive over warps
+  }
+  __syncthreads();
+  const int64_t ex = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - x;
+  if (total != nullptr) *total = warp_sums[(blockDim.x >> 5) - 1];
+  __syncthreads();   // warp_sums may be reused right after
+  return ex;
+}
+
+__device__ __forceinline__ int64_t token_bytes(int w, int d, int hkv, uint32_t* error_word) {
+  const int64_t b = hkv * card_record_bytes(d, w);
+  if (b == 0) raise_error(error_word, Q4KV_DEVERR_WIDTH);
+  return b;
+}
+
+__global__ void __launch_bounds__(kScanThreads) card_chunk_sums_kernel(const uint8_t* __restrict__ widths, int64_t n,
+                                                                       int d, int hkv, int64_t* sums,
+                                                                       uint32_t* error_word) {
+  __shared__ int64_t warp_sums[32];
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kScanChunk + threadIdx.x * kScanPer;
+  int64_t sum = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int64_t y = __shfl_up_sync(0xffffffffu, ws, o);
-        if (lane >= o) ws += y;
-      }
-      warp_sums[lane] = ws;   // inclusive over warps
-    }
+  for (int i = 0; i < kScanPer; ++i)
+    if (t0 + i < n) sum += token_bytes(widths[t0 + i], d, hkv, error_word);
+  int64_t total;
+  block_exclusive_scan(sum, warp_sums, &total);
+  if (threadIdx.x == 0) sums[blockIdx.x] = total;
+}
+
+// One CTA: chunk sums -> exclusive chunk bases (in place), then the header,
+// the table's last entry (the payload size) and the zero padding.
+__global__ void __launch_bounds__(1024) card_chunk_scan_kernel(int64_t* sums, int64_t n_chunks, int64_t n, int d,
+                                                               int hkv, int k_rotated, int raw_dtype, uint8_t* card) {
+  __shared__ int64_t warp_sums[32];
+  __shared__ int64_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < n_chunks; base += blockDim.x) {
+    const int64_t c = base + threadIdx.x;
+    const int64_t x = c < n_chunks ? sums[c] : 0;
+    int64_t total;
+    const int64_t ex = block_exclusive_scan(x, warp_sums, &total);
+    if (c < n_chunks) sums[c] = carry + ex;
     __syncthreads();
-    int64_t run = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - sum;
-#pragma unroll
-    for (int i = 0; i < kCardScanPer; ++i) {
-      if (t0 + i < n) offs[t0 + i] = run;
-      run += sz[i];
-    }
-    __syncthreads();
-    if (threadIdx.x == kCardScanThreads - 1) carry = run;   // the last thread ends the round
+    if (threadIdx.x == 0) carry += total;
     __syncthreads();
   }
+  uint8_t* wdst = card + kCardHeader;
+  uint8_t* otab = card + kCardHeader + round16(n);
   // padding after the widths and after the offsets is zero, so a card's bytes
   // depend on its contents only
   if (threadIdx.x < 16 && n + threadIdx.x < round16(n)) wdst[n + threadIdx.x] = 0;
-  if (threadIdx.x < 16 && 8 * (n + 1) + threadIdx.x < round16(8 * (n + 1)))
-    reinterpret_cast<uint8_t*>(offs)[8 * (n + 1) + threadIdx.x] = 0;
+  if (threadIdx.x < 16 && 8 * (n + 1) + threadIdx.x < round16(8 * (n + 1))) otab[8 * (n + 1) + threadIdx.x] = 0;
   if (threadIdx.x == 0) {
-    offs[n] = carry;
+    reinterpret_cast<int64_t*>(otab)[n] = carry;
     uint32_t* h = reinterpret_cast<uint32_t*>(card);
     h[0] = kCardMagic;
     h[1] = 1;   // version
@@ -871,9 +893,43 @@ __global__ void __launch_bounds__(kCardScanThreads) card_layout_kernel(const uin
   }
 }
 
-__host__ __device__ inline int64_t card_payload_at(int64_t n) {
-  return kCardHeader + round16(n) + round16(8 * (n + 1));
+// Per chunk: the widths copied into the card and the record offsets, from
+// the chunk's base.
+__global__ void __launch_bounds__(kScanThreads) card_offsets_kernel(const uint8_t* __restrict__ widths, int64_t n,
+                                                                    int d, int hkv, const int64_t* bases,
+                                                                    uint8_t* card) {
+  __shared__ int64_t warp_sums[32];
+  __shared__ int64_t stage[kScanChunk];
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kScanChunk;
+  const int64_t t0 = c0 + threadIdx.x * kScanPer;
+  int w[kScanPer];
+  int64_t sum = 0;
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) {
+    w[i] = t0 + i < n ? widths[t0 + i] : 0;
+    sum += hkv * card_record_bytes(d, w[i]);
+  }
+  int64_t run = bases[blockIdx.x] + block_exclusive_scan(sum, warp_sums, nullptr);
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) {
+    stage[threadIdx.x * kScanPer + i] = run;
+    run += hkv * card_record_bytes(d, w[i]);
+  }
+  uint8_t* wdst = card + kCardHeader;
+  if (t0 + kScanPer <= n) {   // 16 widths as one aligned 16-byte store
+    uint32_t q[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) q[i / 4] |= static_cast<uint32_t>(w[i]) << (8 * (i % 4));
+    *reinterpret_cast<uint4*>(wdst + t0) = make_uint4(q[0], q[1], q[2], q[3]);
+  } else {
+    for (int i = 0; i < kScanPer && t0 + i < n; ++i) wdst[t0 + i] = static_cast<uint8_t>(w[i]);
+  }
+  __syncthreads();
+  int64_t* otab = reinterpret_cast<int64_t*>(card + kCardHeader + round16(n));
+  const int64_t cnt = min(static_cast<int64_t>(kScanChunk), n - c0);
+  for (int64_t i = threadIdx.x; i < cnt; i += kScanThreads) otab[c0 + i] = stage[i];
 }
+
 
 // Warp item = (token, VPW KV heads): every lane of a warp works on one token,
 // so its width is warp-uniform; the lane layout, rotation and coding are the
@@ -1127,8 +1183,15 @@ int64_t card_max_bytes(int d, int hkv, int64_t n) { return card_payload_at(n) + 
 cudaError_t launch_card_encode(int d, int hkv, int k_rotated, const void* k, const void* v, int in_dtype,
                                int64_t n, int64_t stride, const uint8_t* widths, uint8_t* card,
                                uint32_t* error_word, cudaStream_t stream) {
-  card_layout_kernel<<<1, kCardScanThreads, 0, stream>>>(widths, n, d, hkv, k_rotated, in_dtype == Q4KV_BF16,
-                                                         card, error_word);
+  // record offsets: chunk sums, their scan (with the header), then the table
+  const int64_t n_chunks = (n + kScanChunk - 1) / kScanChunk;
+  int64_t* sums = reinterpret_cast<int64_t*>(card + card_payload_at(n));   // scratch in the payload
+  if (n_chunks > 0)
+    card_chunk_sums_kernel<<<static_cast<unsigned>(n_chunks), kScanThreads, 0, stream>>>(widths, n, d, hkv, sums,
+                                                                                          error_word);
+  card_chunk_scan_kernel<<<1, 1024, 0, stream>>>(sums, n_chunks, n, d, hkv, k_rotated, in_dtype == Q4KV_BF16, card);
+  if (n_chunks > 0)
+    card_offsets_kernel<<<static_cast<unsigned>(n_chunks), kScanThreads, 0, stream>>>(widths, n, d, hkv, sums, card);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || n == 0) return e;
   const int vpw = d == 128 ? Shape<128>::VPW : Shape<256>::VPW;

@@ -28,7 +28,8 @@ def _dirty(n_bytes):
 
 
 @pytest.mark.parametrize("k_rotated", [True, False])
-@pytest.mark.parametrize("d,dtype,hkv,n", [(128, "fp16", 3, 301), (256, "bf16", 2, 97), (128, "bf16", 8, 8195)])
+@pytest.mark.parametrize("d,dtype,hkv,n", [(128, "fp16", 3, 301), (256, "bf16", 2, 97), (128, "bf16", 8, 8195),
+                                          (128, "fp16", 1, 4096)])
 def test_card_bytes_equal_the_oracle(d, dtype, hkv, n, k_rotated):
     k, v = W.random_small(n, hkv, d, dtype, seed=d + n, scale=2.0)
     widths = W.token_widths(n, seed=n)
