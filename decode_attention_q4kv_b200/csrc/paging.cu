@@ -89,36 +89,34 @@ __global__ void __launch_bounds__(kPageThreads) page_kernel(const __grid_constan
     uint4* img = host + i * stride_words;
     const uint4 hdr = make_uint4(kImageMagic, class_tag(is4, fp8) | static_cast<uint32_t>(d) << 16,
                                  static_cast<uint32_t>(hkv), static_cast<uint32_t>(blk));
-    {
-      uint4 val[kPageUnroll];
-      if constexpr (EXPORT) {
+    uint4 val[kPageUnroll];
+    if constexpr (EXPORT) {
 #pragma unroll
-        for (int u = 0; u < kPageUnroll; ++u) {
-          const int64_t w = w0 + u * kPageThreads;
-          if (w > 0 && w < total) val[u] = __ldg(pool_word(pool, blk, is4, iw, w));
-        }
+      for (int u = 0; u < kPageUnroll; ++u) {
+        const int64_t w = w0 + u * kPageThreads;
+        if (w > 0 && w < total) val[u] = __ldg(pool_word(pool, blk, is4, iw, w));
+      }
 #pragma unroll
-        for (int u = 0; u < kPageUnroll; ++u) {
-          const int64_t w = w0 + u * kPageThreads;
-          if (w < total) img[w] = w == 0 ? hdr : val[u];
-        }
-      } else {
-        const uint4 got = img[0];   // the header, loaded beside the data
+      for (int u = 0; u < kPageUnroll; ++u) {
+        const int64_t w = w0 + u * kPageThreads;
+        if (w < total) img[w] = w == 0 ? hdr : val[u];
+      }
+    } else {
+      const uint4 got = img[0];   // the header, loaded beside the data
 #pragma unroll
-        for (int u = 0; u < kPageUnroll; ++u) {
-          const int64_t w = w0 + u * kPageThreads;
-          if (w > 0 && w < total) val[u] = img[w];
-        }
-        // magic, class, head_dim and Hkv must fit the block; the source id is informational
-        if (got.x != hdr.x || got.y != hdr.y || got.z != hdr.z) {
-          if (w0 == 0) raise_error(pool.error_word, Q4KV_DEVERR_IMAGE);
-          continue;
-        }
+      for (int u = 0; u < kPageUnroll; ++u) {
+        const int64_t w = w0 + u * kPageThreads;
+        if (w > 0 && w < total) val[u] = img[w];
+      }
+      // magic, class, head_dim and Hkv must fit the block; the source id is informational
+      if (got.x != hdr.x || got.y != hdr.y || got.z != hdr.z) {
+        if (w0 == 0) raise_error(pool.error_word, Q4KV_DEVERR_IMAGE);
+        continue;
+      }
 #pragma unroll
-        for (int u = 0; u < kPageUnroll; ++u) {
-          const int64_t w = w0 + u * kPageThreads;
-          if (w > 0 && w < total) *pool_word(pool, blk, is4, iw, w) = val[u];
-        }
+      for (int u = 0; u < kPageUnroll; ++u) {
+        const int64_t w = w0 + u * kPageThreads;
+        if (w > 0 && w < total) *pool_word(pool, blk, is4, iw, w) = val[u];
       }
     }
   }
