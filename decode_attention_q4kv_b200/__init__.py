@@ -248,8 +248,11 @@ def card_max_bytes(head_dim: int, n_kv_heads: int, n_tokens: int) -> int:
 
 
 def card_encode(k: torch.Tensor, v: torch.Tensor, widths: torch.Tensor, k_rotated: bool = True,
-                error_word: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Card (device uint8) of K/V [n][Hkv][D] at per-token widths {2, 4, 8, 16}."""
+                error_word: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Card (device uint8) of K/V [n][Hkv][D] at per-token widths {2, 4, 8, 16}.
+
+    `out` (device uint8, at least card_max_bytes) is reused when given; the
+    card's own size is in its header (payload bytes) and its offset table."""
     dev = _require_cuda(k, v, widths)
     if k.dtype != v.dtype or k.dtype not in _IN_DTYPES or k.shape != v.shape or k.dim() != 3:
         raise ValueError("k and v must be [n][Hkv][D] of one dtype, float16 or bfloat16")
@@ -257,7 +260,13 @@ def card_encode(k: torch.Tensor, v: torch.Tensor, widths: torch.Tensor, k_rotate
         raise ValueError("each token's [Hkv][D] row must be contiguous, with equal strides for k and v")
     n, hkv, d = k.shape
     w = widths.to(torch.uint8).contiguous()
-    card = torch.empty(card_max_bytes(d, hkv, n), dtype=torch.uint8, device=dev)
+    need = card_max_bytes(d, hkv, n)
+    if out is None:
+        card = torch.empty(need, dtype=torch.uint8, device=dev)
+    elif out.dtype != torch.uint8 or not out.is_contiguous() or out.numel() < need or out.device != dev:
+        raise ValueError(f"out must be contiguous uint8 on {dev} with at least {need} bytes")
+    else:
+        card = out
     check(lib().q4kv_card_encode(d, hkv, int(k_rotated), _ptr(k), _ptr(v), _IN_DTYPES[k.dtype], n, k.stride(0),
                                  _ptr(w), _ptr(card), card.numel(), _ptr(error_word), _stream(dev)),
           "q4kv_card_encode")
