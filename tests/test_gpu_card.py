@@ -46,6 +46,10 @@ def test_card_bytes_equal_the_oracle(d, dtype, hkv, n, k_rotated):
     ref = O.card_encode(kh, vh, dt, widths.numpy(), k_rotated=k_rotated)
     got = card.cpu().numpy()
     np.testing.assert_array_equal(got[:ref.size], ref)
+    # a caller's buffer is reused and gets the same bytes
+    again = torch.full_like(card, 0x5A)
+    assert q4.card_encode(k.to(cuda()), v.to(cuda()), widths.to(cuda()), k_rotated=k_rotated, out=again) is again
+    np.testing.assert_array_equal(again.cpu().numpy()[:ref.size], ref)
     # decode: the oracle's rebuilt rows exactly (fp32) and their fp16 rounding
     k_hat, v_hat = O.card_decode(ref)
     kd, vd = q4.card_decode(card, n, hkv, d, error_word=err)
