@@ -285,17 +285,31 @@ def job_throughput(world: int, bytes_per_step: float, steps: int, elapsed_s: flo
     return world * bytes_per_step * steps / elapsed_s / 1e9
 
 
-def sources_digest():
+# Files whose contents decide a kernel's DRAM traffic per launch: its own
+# source, the shared device headers and the ABI header; for decode also the
+# host code that picks the split count (the partials it writes depend on it).
+_CSRC = os.path.join("decode_attention_q4kv_b200", "csrc")
+KERNEL_SOURCES = {
+    "quantize": ("quantize.cu", "async_copy.cuh", "q4kv_internal.cuh"),
+    "decode": ("decode_tc.cu", "decode.cu", "api.cu", "async_copy.cuh", "q4kv_internal.cuh"),
+}
+
+
+def sources_digest(kernel=None):
+    """Digest of one kernel's sources (KERNEL_SOURCES), or of every file under csrc/."""
+    names = KERNEL_SOURCES[kernel] if kernel else sorted(os.listdir(os.path.join(ROOT, _CSRC)))
+    paths = [os.path.join(ROOT, _CSRC, n) for n in names]
+    if kernel:
+        paths.append(os.path.join(ROOT, "include", "q4kv.h"))
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "decode_attention_q4kv_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel_key, launches_scale=1.0):
-    """DRAM bytes per launch from the committed ncu summary, if the sources still match."""
+    """DRAM bytes per launch from the committed ncu summary, if that kernel's sources still match."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -303,7 +317,7 @@ def traffic_for(kernel_key, launches_scale=1.0):
     except OSError:
         return None
     ent = t.get(kernel_key)
-    if not ent or ent.get("sources") != sources_digest():
+    if not ent or ent.get("sources") != sources_digest(kernel_key.split(":")[0]):
         return None
     return ent["dram_bytes_per_launch"] * launches_scale
 

@@ -321,7 +321,11 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
   int64_t s = n_splits;
   if (s == 0) {
     // persistent CTAs (one per SM) take items (sequence, KV head, split) in
-    // waves; cost = waves * (blocks per item + per-item overhead)
+    // waves; cost = waves * (blocks per item + per-item overhead).  The
+    // overhead (query preparation, cross-warp merge, partial write) is 3.2
+    // block-times, fitted to decode times measured with forced split counts
+    // on the Gemma-, Llama- and Qwen-shaped layers and the batch/context
+    // sweep; with it the choice was the fastest measured split on each.
     const int64_t pairs = static_cast<int64_t>(batch > 0 ? batch : 1) * n_kv_heads;
     double best = 1e300;
     s = 1;
@@ -330,7 +334,7 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
       if ((nb + bps - 1) / bps != cand) continue;         // each distinct split only once
       const int64_t items = pairs * cand;
       const int64_t waves = (items + num_sms - 1) / num_sms;
-      const double cost = static_cast<double>(waves) * (static_cast<double>(bps) + 0.75);
+      const double cost = static_cast<double>(waves) * (static_cast<double>(bps) + 3.2);
       if (cost < best - 1e-9) {
         best = cost;
         s = cand;
