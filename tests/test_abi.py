@@ -274,3 +274,16 @@ def test_card_calls_reject_bad_arguments_without_launching():
     assert dec(FAKE, big, 128, 8, 10, FAKE + 4, FAKE, 2, None, None) == _lib.ERR_INVALID_ARG
     assert dec(FAKE, big, 128, 8, -1, FAKE, FAKE, 2, None, None) == _lib.ERR_INVALID_ARG
     assert dec(None, 0, 128, 8, 0, None, None, 2, None, None) == 0                       # nothing to rebuild
+
+
+@pytest.mark.parametrize("shape,splits", [((5, 16, 8, 256, 32), 3),       # Gemma-3-12B shape, 5 x 8192
+                                          ((10, 32, 8, 128, 128), 5),     # Llama-3.1-8B, 10 x 32768
+                                          ((32, 40, 8, 128, 64), 1),      # Qwen2.5-14B, 32 x 16384
+                                          ((16, 32, 8, 128, 128), 1),     # sweep 16 x 32K
+                                          ((64, 32, 8, 128, 16), 1),      # sweep 64 x 4K
+                                          ((1, 32, 8, 128, 512), 18)])    # sweep 1 x 128K
+def test_default_split_counts_are_the_fastest_measured(shape, splits):
+    """The cost model's choice on the workload shapes equals the split count
+    that measured fastest among forced-split runs on a B200 (148 SMs)."""
+    st, p = _plan(*shape, 0, 148)
+    assert st == 0 and p.n_splits == splits
