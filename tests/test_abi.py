@@ -283,7 +283,9 @@ def test_card_calls_reject_bad_arguments_without_launching():
                                           ((64, 32, 8, 128, 16), 1),      # sweep 64 x 4K
                                           ((1, 32, 8, 128, 512), 18)])    # sweep 1 x 128K
 def test_default_split_counts_are_the_fastest_measured(shape, splits):
-    """The cost model's choice on the workload shapes equals the split count
-    that measured fastest among forced-split runs on a B200 (148 SMs)."""
+    """The cost model's choice on the workload shapes is the split count that
+    measured fastest among the forced-split runs made on a B200 (148 SMs):
+    Gemma 2/3/4/5/6/7/8/11/16/32, Llama 1/2/3/4/5/6/8/11, Qwen 1/2/3/4/6/8,
+    and the old and new choice on the sweep points."""
     st, p = _plan(*shape, 0, 148)
     assert st == 0 and p.n_splits == splits
