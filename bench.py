@@ -6,14 +6,18 @@ One step is one pass of the whole path over one batch of synthetic input:
 for every layer, quantise all K/V tokens into the paged 4-bit pool (K
 Walsh-Hadamard rotated), apply the workload's eviction / mixed-width steps,
 then run split-K paged GQA decode attention for the batch.  The default
-workload is the Gemma-3-12B-shaped 5-agent cache (48 layers, 16 query / 8
-KV heads, head_dim 256, 5 x 8192 tokens, bf16 input).
+workload is the largest single-GPU configuration: the Qwen2.5-14B-shaped
+eviction-masked cache (48 layers, 40 query / 8 KV heads, head_dim 128,
+32 sessions x 16384 tokens, fp16 input, 60 % of slots remapped to the
+sentinel), all 48 layers resident in HBM (~132 GB).
 
 Printed (rank 0, one JSON line): value = algorithmic HBM bytes of the whole
 step (quantise: read K/V, write codes + scale/zero; decode: read codes +
 scale/zero + mask of every live block) / step time, in GB/s, summed over
-ranks; per-kernel CUDA-event times; the roofline of the dominant kernel; an
-end-to-end number through host buffers; the CPU oracle on a bounded sample.
+ranks; the metric's parts (decode GB/s, its fraction of HBM and KV tokens/s;
+quantise GB/s); per-kernel CUDA-event times; the roofline of the dominant
+kernel and of both kernels; an end-to-end number through host buffers; the
+CPU oracle on a bounded sample, on one thread and on all host cores.
 """
 from __future__ import annotations
 
@@ -31,6 +35,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "Q4 paged decode-attn HBM GB/s (% of ~8 TB/s), KV tokens/s; quantize GB/s"
+
+# The arithmetic the path computes in: the encoder is binary32 (rotation,
+# group statistics, correctly rounded quotients) producing 4/8-bit codes with
+# fp16 scale/zero; decode runs keys as u4/u8 codes x s8 query digits on int8
+# MMAs (exact int32), values as fp16 MMAs with fp16 weights, both
+# accumulating in fp32; softmax and merge in fp32.
+DTYPE_LABEL = "int8 MMA (u4/u8 codes x s8 query digits, s32 acc) + fp16 MMA (f32 acc); encoder f32"
 
 
 # ---------------------------------------------------------------------------
@@ -138,7 +149,7 @@ class ClockSampler:
 class Job:
     """All layers of one workload resident on one GPU, ready to step."""
 
-    def __init__(self, w, device, rank=0, layers=None, fp8=False):
+    def __init__(self, w, device, rank=0, layers=None, fp8=False, decode_kernel=1):
         import torch
 
         import decode_attention_q4kv_b200 as q4
@@ -176,6 +187,7 @@ class Job:
         self.lens = W.seq_lens(w).to(device)
         self.evict = W.evicted_slot_ids(w, W.identity_tables(w)).to(device) if w.evict_fraction else None
         self.plan = q4.DecodePlan(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.blocks_per_seq)
+        self.plan.c.kernel = decode_kernel
         self.ws = self.plan.workspace(device)
         if w.permuted_pool:
             # fill the whole pool once by tiling the quantised prefill (setup, not timed)
@@ -280,6 +292,14 @@ def reduce_max(value: float, device) -> float:
     return float(t.item())
 
 
+def check_world(gpus: int, world: int) -> None:
+    """--gpus N must match the launch: one process per GPU (torchrun for N > 1)."""
+    if gpus != world:
+        sys.stderr.write(f"bench.py: --gpus {gpus} but WORLD_SIZE is {world}; launch N > 1 ranks with "
+                         f"python -m torch.distributed.run --nproc-per-node {gpus} bench.py --gpus {gpus}\n")
+        sys.exit(2)
+
+
 def job_throughput(world: int, bytes_per_step: float, steps: int, elapsed_s: float) -> float:
     """Whole-job GB/s: every rank moved bytes_per_step per step; time = slowest rank."""
     return world * bytes_per_step * steps / elapsed_s / 1e9
@@ -340,6 +360,7 @@ def run_gpu(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    check_world(args.gpus, world)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -348,7 +369,7 @@ def run_gpu(args):
                                 device_id=dev)
 
     w = workload_by_name(args.workload)
-    job = Job(w, dev, rank, args.layers, fp8=args.fp8)
+    job = Job(w, dev, rank, args.layers, fp8=args.fp8, decode_kernel=args.decode_kernel)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -418,31 +439,41 @@ def run_gpu(args):
         d_cold_gbps = job.decode_bytes / (d_cold_ms * 1e-3) / 1e9
         kv_tok = w.batch * w.ctx * w.n_kv_heads
         dominant = "quantize" if q_ms >= d_ms else "decode"
-        if dominant == "quantize":
-            roof = dict(bound="hbm", achieved=round(q_gbps, 1), peak=peak, unit="GB/s",
-                        frac=round(q_gbps / peak, 4),
-                        traffic=traffic_for(f"quantize:{w.name}"),
-                        kernel="quantize_kernel", algorithmic_bytes_per_launch=job.quant_bytes,
-                        us_per_launch=round(q_ms * 1e3, 2), peak_source=f"{peak_src} hbm_gbs (burst copy)")
-        else:
-            roof = dict(bound="hbm", achieved=round(d_cold_gbps, 1), peak=peak, unit="GB/s",
-                        frac=round(d_cold_gbps / peak, 4),
-                        traffic=traffic_for(f"decode:{w.name}"),
-                        kernel="decode", algorithmic_bytes_per_launch=job.decode_bytes,
-                        us_per_launch=round(d_cold_ms * 1e3, 2), peak_source=f"{peak_src} hbm_gbs (burst copy)")
+        roofs = {
+            "quantize": dict(bound="hbm", achieved=round(q_gbps, 1), peak=peak, unit="GB/s",
+                             frac=round(q_gbps / peak, 4),
+                             traffic=traffic_for(f"quantize:{w.name}"),
+                             kernel="quantize_kernel", algorithmic_bytes_per_launch=job.quant_bytes,
+                             us_per_launch=round(q_ms * 1e3, 2),
+                             peak_source=f"{peak_src} hbm_gbs (burst copy)"),
+            "decode": dict(bound="hbm", achieved=round(d_cold_gbps, 1), peak=peak, unit="GB/s",
+                           frac=round(d_cold_gbps / peak, 4),
+                           traffic=traffic_for(f"decode:{w.name}"),
+                           kernel="decode_tc_kernel + merge_kernel",
+                           algorithmic_bytes_per_launch=job.decode_bytes,
+                           us_per_launch=round(d_cold_ms * 1e3, 2),
+                           peak_source=f"{peak_src} hbm_gbs (burst copy)"),
+        }
+        roof = roofs[dominant]
         value = job_throughput(world, job.bytes_per_step, args.steps, elapsed)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_LABEL, "data": "synthetic",
+            "metric_parts": {"decode_gbps": round(d_cold_gbps, 1),
+                             "decode_frac_of_hbm": round(d_cold_gbps / peak, 4),
+                             "kv_tokens_per_s": round(kv_tok / (d_cold_ms * 1e-3), 1),
+                             "quantize_gbps": round(q_gbps, 1),
+                             "quantize_frac_of_hbm": round(q_gbps / peak, 4),
+                             "hbm_peak_gbps": peak, "hbm_peak_source": peak_src},
             "config": {"workload": w.name, "layers": job.n_layers, "batch": w.batch, "ctx": w.ctx,
                        "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                        "input_dtype": w.dtype, "storage": ("fp8 e4m3 codes (the comparison cache), no scale, 256-token blocks" if args.fp8 else
                                    "int4 codes, group 64, fp16 scale+zero, 256-token blocks"),
                        "q8_fraction": 0.0 if args.fp8 else w.q8_fraction, "evict_fraction": w.evict_fraction,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "decode_splits": job.plan.n_splits,
+                       "decode_splits": job.plan.n_splits, "decode_kernel": args.decode_kernel,
                        "l2": "step inputs larger than L2 (%.1f GB)" % (job.bytes_per_step / 1e9)},
             "kernels": {
                 "quantize": {"gbps": round(q_gbps, 1), "us_per_launch": round(q_ms * 1e3, 2),
@@ -460,6 +491,7 @@ def run_gpu(args):
                 "card": card,
             },
             "roofline": roof,
+            "roofline_kernels": roofs,
             "gpu_launches": job.launches_per_layer * job.n_layers * args.steps,
             "clocks": clk.result(),
         }
@@ -631,12 +663,29 @@ def run_e2e(job, args, dev, world):
 # CPU oracle (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(w, kv_heads=1, layer=0):
-    """One bounded sample: one layer, `kv_heads` KV heads, all sessions, on the host.
+_LAYER_CACHE = {}
+
+
+def _layer_inputs(w, layer):
+    """Host K/V/q of one layer (drawing them is slower than the sample; the
+    last layer drawn is kept, so successive KV-head slices reuse it)."""
+    from decode_attention_q4kv_b200 import workloads as W
+    key = (w.name, layer)
+    if key not in _LAYER_CACHE:
+        _LAYER_CACHE.clear()
+        n_tok = w.prefill_tokens or w.n_tokens
+        k, v = W.kv_tokens(w, layer, n_tok, "cpu")
+        _LAYER_CACHE[key] = (k, v, W.query(w, layer, "cpu"))
+    return _LAYER_CACHE[key]
+
+
+def oracle_sample(w, kv_heads=1, layer=0, head=0):
+    """One bounded sample: one layer, KV heads [head, head + kv_heads), all
+    sessions, on the host.
 
     Quantises every token of those heads and decodes every query head that
     reads them, with the oracle as it stands.  Returns (seconds, algorithmic
-    bytes of the sample).
+    bytes of the sample); drawing the inputs is not timed.
     """
     import numpy as np
     import torch
@@ -645,11 +694,10 @@ def oracle_sample(w, kv_heads=1, layer=0):
     from oracle import q4kv_oracle as O
 
     n_tok = w.prefill_tokens or w.n_tokens
-    k, v = W.kv_tokens(w, layer, n_tok, "cpu")
-    q = W.query(w, layer, "cpu")
-    k, v = k[:, :kv_heads].contiguous(), v[:, :kv_heads].contiguous()
+    k, v, q = _layer_inputs(w, layer)
+    k, v = k[:, head:head + kv_heads].contiguous(), v[:, head:head + kv_heads].contiguous()
     g = w.gqa
-    q = q[:, : kv_heads * g].contiguous()
+    q = q[:, head * g:(head + kv_heads) * g].contiguous()
 
     def host(t):
         if t.dtype == torch.float16:
@@ -681,22 +729,100 @@ def oracle_sample(w, kv_heads=1, layer=0):
     return secs, (qb + db) * frac
 
 
-def cpu_baseline(w, target_s=15.0):
-    """The oracle on a bounded sample: one-KV-head slices of successive layers until ~target_s."""
+def host_cores() -> int:
+    """Cores this process may run on (its affinity mask), else the machine's count."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def _oracle_samples_1t(w, slices):
+    """oracle_sample of each (layer, head) slice in turn on one thread (a
+    worker of the all-cores leg)."""
+    from threadpoolctl import threadpool_limits
+    secs = nbytes = 0.0
+    with threadpool_limits(limits=1):
+        for layer, head in slices:
+            s, b = oracle_sample(w, kv_heads=1, layer=layer, head=head)
+            secs += s
+            nbytes += b
+    return secs, nbytes
+
+
+def _worker_ready(w, layer):
+    """Imports and the worker's input layer, paid before the timed region."""
+    from oracle import q4kv_oracle  # noqa: F401
+    _layer_inputs(w, layer)
+    return True
+
+
+def cpu_baseline_all_cores(w, workers, per_worker=1):
+    """The oracle, unchanged, on `workers` processes at once: each quantises and
+    decodes its own one-KV-head slice of a different layer on one thread.
+    Value = the slices' algorithmic bytes / wall time from submission to the
+    last result (the pool is started and warmed first).  Workers are spawned,
+    not forked, because this process has initialised CUDA."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=ctx) as ex:
+        # every worker draws the same layer; each then takes other KV heads
+        for f in [ex.submit(_worker_ready, w, 0) for _ in range(workers)]:
+            f.result()
+        t0 = time.perf_counter()
+        futs = [ex.submit(_oracle_samples_1t, w, [(0, (per_worker * i + j) % w.n_kv_heads)
+                                                   for j in range(per_worker)])
+                for i in range(workers)]
+        nbytes = sum(f.result()[1] for f in futs)
+        wall = time.perf_counter() - t0
+    return nbytes / wall / 1e9, wall
+
+
+def all_cores_workers(w, cores):
+    """Worker count for the all-cores leg: every core, bounded by host memory
+    (each worker draws one layer's K/V in fp32 before slicing one head)."""
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = 16 << 30
+    n_tok = w.prefill_tokens or w.n_tokens
+    per_worker = 8 * n_tok * w.n_kv_heads * w.head_dim + (1 << 30)
+    return max(1, min(cores, int(0.6 * avail // per_worker)))
+
+
+def cpu_baseline(w, target_s=15.0, all_cores=True):
+    """The oracle on a bounded sample: one-KV-head slices of successive layers
+    until ~target_s on one thread; then the same slices on all host cores."""
     from threadpoolctl import threadpool_limits
 
     with threadpool_limits(limits=1):
         total_s, total_b, n = 0.0, 0.0, 0
         while total_s < target_s and n < 4 * w.n_kv_heads:
-            s2, b2 = oracle_sample(w, kv_heads=1, layer=n)
+            s2, b2 = oracle_sample(w, kv_heads=1, layer=n // w.n_kv_heads, head=n % w.n_kv_heads)
             total_s += s2
             total_b += b2
             n += 1
-    return {"value": round(total_b / total_s / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} x (one layer, one KV head of {w.n_kv_heads}: quantise all "
-                      f"{w.prefill_tokens or w.n_tokens} tokens + decode the {w.gqa} query heads "
-                      f"of all {w.batch} sessions); numpy/BLAS limited to 1 thread",
-            "seconds": round(total_s, 2)}
+    cores = host_cores()
+    out = {"value": round(total_b / total_s / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "host_cores": cores,
+           "sample": f"{n} x (one KV head of {w.n_kv_heads} of a layer: quantise all "
+                     f"{w.prefill_tokens or w.n_tokens} tokens + decode the {w.gqa} query heads "
+                     f"of all {w.batch} sessions); numpy/BLAS limited to 1 thread",
+           "seconds": round(total_s, 2)}
+    if all_cores and cores > 1:
+        workers = all_cores_workers(w, cores)
+        per_worker = max(1, min(16, round(5.0 / max(total_s / n, 1e-3))))   # ~5 s per worker
+        try:
+            v, wall = cpu_baseline_all_cores(w, workers, per_worker)
+            out["all_cores"] = {"value": round(v, 5), "unit": "GB/s", "cores": workers,
+                                "sample": f"{workers} processes (spawned) at once, each {per_worker} "
+                                          f"slice(s) as above on one thread",
+                                "seconds": round(wall, 2)}
+        except Exception as e:          # reported, not fatal: the GPU line stands without it
+            out["all_cores"] = {"error": repr(e)[:200]}
+    return out
 
 
 def run_reference(args):
@@ -707,11 +833,12 @@ def run_reference(args):
 
     w = workload_by_name(args.workload)
     with threadpool_limits(limits=1):
+        hkv = w.n_kv_heads
         for i in range(args.warmup):
-            oracle_sample(w, kv_heads=1, layer=i)
+            oracle_sample(w, kv_heads=1, layer=i // hkv, head=i % hkv)
         secs, nbytes = 0.0, 0.0
-        for i in range(args.steps):
-            s, b = oracle_sample(w, kv_heads=1, layer=args.warmup + i)
+        for i in range(args.warmup, args.warmup + args.steps):
+            s, b = oracle_sample(w, kv_heads=1, layer=i // hkv, head=i % hkv)
             secs += s
             nbytes += b
     value = nbytes / secs / 1e9
@@ -724,7 +851,8 @@ def run_reference(args):
                        "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                        "input_dtype": w.dtype},
             "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": "each step: one layer, one KV head (all tokens quantised, "
+                             "host_cores": host_cores(),
+                             "sample": "each step: one KV head of a layer (all tokens quantised, "
                                        "its query heads decoded), numpy/BLAS limited to 1 thread"},
             "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -737,7 +865,11 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="q4kv", choices=["q4kv", "reference"])
-    ap.add_argument("--workload", default="gemma")
+    ap.add_argument("--workload", default="evict",
+                    help="evict (default: Qwen2.5-14B shape, 32 x 16384, 60%% evicted), gemma, mixed, tiny, "
+                         "or sweep:B:C")
+    ap.add_argument("--decode-kernel", type=int, default=1, choices=[0, 1],
+                    help="decode variant: 1 tensor-core pipeline (default), 0 CUDA-core kernel")
     ap.add_argument("--fp8", action="store_true",
                     help="run the same workload on the FP8 (E4M3) comparison cache instead of Q4")
     ap.add_argument("--layers", type=int, default=None)

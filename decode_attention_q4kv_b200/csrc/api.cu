@@ -378,7 +378,7 @@ q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan*
   if (st != Q4KV_OK) return st;
   if (plan->head_dim != pool->head_dim || plan->n_kv_heads != pool->n_kv_heads ||
       ref.n_splits != plan->n_splits || ref.tokens_per_split != plan->tokens_per_split ||
-      ref.workspace_bytes != plan->workspace_bytes)
+      ref.workspace_bytes != plan->workspace_bytes || (plan->kernel != 0 && plan->kernel != 1))
     return Q4KV_ERR_INVALID_ARG;
   if ((q_dtype != Q4KV_F16 && q_dtype != Q4KV_BF16) ||
       (out_dtype != Q4KV_F32 && out_dtype != Q4KV_F16 && out_dtype != Q4KV_BF16) ||

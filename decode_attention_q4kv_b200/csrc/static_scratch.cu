@@ -1,36 +1,25 @@
 // Allocation-free decode entry point: the split partials of
 // q4kv_decode_attention live in a file-scope device array instead of a
 // caller-provided workspace, for callers that cannot allocate device memory.
-#include <mutex>
-
 #include "q4kv_internal.cuh"
 
 namespace {
 
 constexpr size_t kScratchBytes = Q4KV_STATIC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 128;
 
 // One copy per device that loads this library, held until process exit.
 __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices];   // device address of g_decode_scratch, per device
-
 // In host code `g_decode_scratch` names a host-side stand-in, not device
-// memory, so the device address is looked up once per device (with that
-// device current) and cached.
+// memory.  The device address is looked up on every call for the device and
+// context current at that moment: a cached address would dangle after a
+// cudaDeviceReset or under another context that loaded the module anew.
+// The lookup allocates nothing; the first one on a device loads the module.
 q4kv_status scratch_address(void** addr) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return Q4KV_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return Q4KV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr) return Q4KV_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *addr = g_scratch_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr) return Q4KV_ERR_CUDA;
+  *addr = p;
   return Q4KV_OK;
 }
 

@@ -266,7 +266,10 @@ typedef struct {
   int32_t max_blocks_per_seq;  /* width of the block table */
   int32_t n_splits;
   int32_t tokens_per_split;    /* multiple of 64 */
-  int32_t kernel;              /* kernel variant chosen for this shape (informational) */
+  int32_t kernel;              /* kernel variant: 1 = tensor-core pipeline (what
+                                  q4kv_decode_plan_make picks), 0 = the CUDA-core
+                                  kernel (4/8-bit pools only; one CTA per item);
+                                  any other value is rejected */
   size_t workspace_bytes;      /* device scratch the call needs (0 when n_splits == 1) */
 } q4kv_decode_plan;
 
@@ -317,9 +320,11 @@ q4kv_status q4kv_decode_attention(const q4kv_pool *pool, const q4kv_decode_plan 
  *   - A plan whose workspace_bytes exceeds Q4KV_STATIC_SCRATCH_BYTES is
  *     rejected with Q4KV_ERR_WORKSPACE before anything runs; force fewer
  *     splits (q4kv_decode_plan_make n_splits) or use q4kv_decode_attention.
- *   - The first call on a device looks up the array's device address once
- *     (with that device current); make that first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address for the device current
+ *     at that moment (cudaGetSymbolAddress, which allocates nothing), so the
+ *     address stays right after a device reset.  The first call on a device
+ *     also loads the library's device code there; make that first call
+ *     before any stream capture.
  *   - All calls share the array and it keeps the last call's contents; the
  *     kernels overwrite every partial they later read, so nothing needs to
  *     start at zero.  Calls that overlap on the GPU (other streams, other

@@ -176,6 +176,10 @@ def test_decode_rejects_bad_arguments_without_launching():
     bad = _lib.DecodePlan.from_buffer_copy(plan)
     bad.tokens_per_split += 64
     assert call(pl=bad) == _lib.ERR_INVALID_ARG                          # not a plan the library made
+    for k in (2, -1):                                                    # only variants 0 and 1 exist
+        bad = _lib.DecodePlan.from_buffer_copy(plan)
+        bad.kernel = k
+        assert call(pl=bad) == _lib.ERR_INVALID_ARG
     st, empty = _plan(0, 32, 8, 128, 4, 0, 148)
     assert st == 0
     assert call(pl=empty, ws=0, wsb=0) == 0                              # batch 0: nothing to do

@@ -18,7 +18,7 @@ def test_reference_arm_prints_one_contract_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] >= 3
     assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["value"] > 0
-    assert d["config"]["workload"] == "gemma3_12b_5x8192_d256"
+    assert d["config"]["workload"] == "qwen25_14b_32x16384_evict60"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

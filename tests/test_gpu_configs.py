@@ -130,8 +130,12 @@ def test_mixed_workload():
         _check_attention(job, li, [(0, 0), (9, 7), (4, 3)], q8_chunks=q8)
 
 
-@pytest.mark.parametrize("batch,ctx", [(1, 4096), (16, 32768), (256, 32768), (64, 131072)])
+@pytest.mark.parametrize("ctx", W.SWEEP_CONTEXTS)
+@pytest.mark.parametrize("batch", W.SWEEP_BATCHES)
 def test_sweep_point(batch, ctx):
+    """Every point of the batch {1, 16, 64, 256} x context {4K, 32K, 128K}
+    sweep, up to 256 x 128K (a 37.7 GB pool): sampled encoder rows bit-exact,
+    three (sequence, KV head) rows against the oracle."""
     job = _run(f"sweep:{batch}:{ctx}", [0])
     _check_encoder_rows(job, 0)
     _check_attention(job, 0, [(0, 0), (batch - 1, 7), (batch // 2, 3)])

@@ -221,3 +221,24 @@ def test_long_sequences_with_mixed_widths_and_eviction(kernel):
     for s in (0, 1):
         out, _ = c.run(s, kernel=kernel)
         assert_close(out, want, what=f"long, splits {s}")
+
+
+@pytest.mark.parametrize("rotated", [True, False])
+@pytest.mark.parametrize("big", [300.0, 3000.0, 30000.0])
+def test_wide_dynamic_range_query(rotated, big):
+    """Queries with one outlier channel per head (300, 3000 or 30000) and the
+    rest N(0, 1e-2), fp16, over rotated and raw keys.  The decode kernel turns
+    the (rotated) query into fixed point with one power-of-two scale per head,
+    so the small channels keep only the precision the digits leave them; the
+    outlier makes the softmax sharp, so near-ties between the top keys show
+    any error of those small channels.  Element by element against the
+    oracle's fp64 attention (max-abs 2e-3, relative L2 1e-2)."""
+    c = Case([1200, 333, 2048], hq=32, hkv=8, d=128, seed=15, rotated=rotated)
+    g = torch.Generator().manual_seed(16 + int(big))
+    q = torch.randn(c.q.shape, generator=g) * 1e-2
+    ch = torch.randint(0, q.shape[2], q.shape[:2], generator=g)
+    q.scatter_(2, ch[..., None], big)
+    c.q = q.to(torch.float16)
+    for s in (0, 3):
+        out, _ = c.run(s)
+        assert_close(out, c.oracle(), what=f"outlier {big}, {'rotated' if rotated else 'raw'} keys, splits {s}")
