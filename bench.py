@@ -427,6 +427,7 @@ def run_gpu(args):
 
     paging = measure_paging(job, dev, reps, d_cold_ms)
     card = measure_card(job, dev, reps) if not args.fp8 else None
+    q2mix = measure_q2mix(job, dev, reps) if not args.fp8 else None
 
     e2e = run_e2e(job, args, dev, world) if not args.no_e2e else None
     if world > 1:
@@ -489,6 +490,7 @@ def run_gpu(args):
                            "note": "one new token per sequence written over its last slot, then decode"},
                 "paging": paging,
                 "card": card,
+                "q2mix": q2mix,
             },
             "roofline": roof,
             "roofline_kernels": roofs,
@@ -503,6 +505,61 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_q2mix(job, dev, reps):
+    """Three code widths in one paged pool: the first layer's blocks coded
+    8-bit (the quarter with the highest mean |K|), 2-bit (the quarter with
+    the lowest) and 4-bit (the rest) -- a fixed synthetic policy standing in
+    for QKVShare's learned width controller, which gives no distribution.
+    Times the encoder over the whole layer and decode over the mixed pool
+    with the bench's own plan; algorithmic bytes count each block at its width."""
+    import torch
+    import decode_attention_q4kv_b200 as q4
+    w = job.w
+    if w.permuted_pool:
+        return None
+    L = job.layers[0]
+    k, v = L["k"], L["v"]
+    nb, hkv, d = w.n_blocks, w.n_kv_heads, w.head_dim
+    am = q4.block_absmean(k)
+    order = torch.argsort(am, descending=True, stable=True)
+    ranks = torch.empty_like(order)
+    ranks[order] = torch.arange(nb, device=dev)
+    n8, n2 = nb // 4, nb // 4
+    n4 = nb - n8 - n2
+    ids = torch.where(ranks < n8, n4 + ranks,
+                      torch.where(ranks >= nb - n2, n4 + n8 + ranks - (nb - n2), ranks - n8)).to(torch.int32)
+    pool = q4.Q4KVPool(hkv, d, n4, n8, device=dev, n_q2_blocks=n2)
+    tables = ids.view(w.batch, w.blocks_per_seq)
+    ng = d // 64
+    row = {4: d // 2 + 4 * ng, 8: d + 4 * ng, 2: d // 4 + 4 * ng}
+    code_bytes = 256 * hkv * 2 * (n4 * row[4] + n8 * row[8] + n2 * row[2])
+    q_bytes = w.n_tokens * hkv * 2 * d * 2 + code_bytes
+    d_bytes = code_bytes + nb * 32 + w.batch * w.blocks_per_seq * 4 + w.batch * w.n_q_heads * d * (2 + 4)
+
+    def timed(fn):
+        out = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            out.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in out)
+
+    q_ms = timed(lambda: pool.quantize(k, v, ids))
+    dec = lambda: q4.decode_attention(pool, L["q"], tables, job.lens, plan=job.plan, workspace=job.ws, out=L["out"])
+    dec()
+    d_ms = timed(dec)
+    assert pool.read_device_error() == 0
+    return {"blocks": {"8": n8, "4": n4, "2": n2}, "bits_per_value": round(8 * code_bytes / (2 * nb * 256 * hkv * d), 3),
+            "quantize_us": round(q_ms * 1e3, 1), "quantize_gbps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+            "decode_us": round(d_ms * 1e3, 2), "decode_gbps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1),
+            "decode_bytes": d_bytes,
+            "note": "first layer, blocks 8-bit (top quarter by mean |K|), 2-bit (bottom quarter), 4-bit (rest); "
+                    "decode repeated on one layer (L2 may hold part of it)"}
 
 
 def measure_card(job, dev, reps):

@@ -60,25 +60,29 @@ class Q4KVPool:
     """Device storage of the paged cache plus its C descriptor.
 
     Unified block ids [0, n_q4_blocks) are 4-bit, [n_q4_blocks,
-    n_q4_blocks + n_q8_blocks) are 8-bit.  Tensors (row-major):
+    n_q4_blocks + n_q8_blocks) are 8-bit, the next n_q2_blocks ids 2-bit.
+    Tensors (row-major):
       k_codes4/v_codes4   uint8 [n_q4][Hkv][256][D/2]
       k_params4/v_params4 fp16  [n_q4][Hkv][256][D/64][2]   (scale, zero)
       k_codes8/v_codes8   uint8 [n_q8][Hkv][256][D]
       k_params8/v_params8 fp16  [n_q8][Hkv][256][D/64][2]
-      mask                int32 [n_q4+n_q8][8] (bit set = slot remapped)
+      k_codes2/v_codes2   uint8 [n_q2][Hkv][256][D/4]
+      k_params2/v_params2 fp16  [n_q2][Hkv][256][D/64][2]
+      mask                int32 [n_q4+n_q8+n_q2][8] (bit set = slot remapped)
       error_word          int32 [4] (word 0 holds device error bits)
     """
 
     def __init__(self, n_kv_heads: int, head_dim: int, n_q4_blocks: int, n_q8_blocks: int = 0,
-                 k_rotated: bool = True, device="cuda", fp8: bool = False):
+                 k_rotated: bool = True, device="cuda", fp8: bool = False, n_q2_blocks: int = 0):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("Q4KVPool lives on a CUDA device")
-        if fp8 and (n_q4_blocks or k_rotated):
-            raise ValueError("an FP8 pool has only 8-bit blocks (n_q4_blocks = 0) and raw keys (k_rotated = False)")
+        if fp8 and (n_q4_blocks or n_q2_blocks or k_rotated):
+            raise ValueError("an FP8 pool has only 8-bit blocks (n_q4_blocks = n_q2_blocks = 0) and raw keys "
+                             "(k_rotated = False)")
         self.fp8 = bool(fp8)
         self.n_kv_heads, self.head_dim = n_kv_heads, head_dim
-        self.n_q4_blocks, self.n_q8_blocks = n_q4_blocks, n_q8_blocks
+        self.n_q4_blocks, self.n_q8_blocks, self.n_q2_blocks = n_q4_blocks, n_q8_blocks, n_q2_blocks
         self.k_rotated = bool(k_rotated)
         ng = head_dim // GROUP
         T = BLOCK_TOKENS
@@ -94,7 +98,10 @@ class Q4KVPool:
         self.k_codes8, self.v_codes8 = codes(n_q8_blocks, head_dim), codes(n_q8_blocks, head_dim)
         n_par8 = 0 if self.fp8 else n_q8_blocks                 # FP8 blocks carry no params
         self.k_params8, self.v_params8 = params(n_par8), params(n_par8)
-        self.mask = torch.zeros((n_q4_blocks + n_q8_blocks, 8), dtype=torch.int32, device=self.device)
+        self.k_codes2, self.v_codes2 = codes(n_q2_blocks, head_dim // 4), codes(n_q2_blocks, head_dim // 4)
+        self.k_params2, self.v_params2 = params(n_q2_blocks), params(n_q2_blocks)
+        self.mask = torch.zeros((n_q4_blocks + n_q8_blocks + n_q2_blocks, 8), dtype=torch.int32,
+                                device=self.device)
         self.error_word = torch.zeros(4, dtype=torch.int32, device=self.device)
         self.desc = _lib.PoolDesc(
             head_dim, n_kv_heads, int(self.k_rotated), n_q4_blocks, n_q8_blocks, int(self.fp8),
@@ -104,15 +111,21 @@ class Q4KVPool:
             self.v_codes8.data_ptr() if n_q8_blocks else 0,
             self.k_params8.data_ptr() if n_q8_blocks else 0,
             self.v_params8.data_ptr() if n_q8_blocks else 0,
-            self.mask.data_ptr(), self.error_word.data_ptr())
+            self.mask.data_ptr(), self.error_word.data_ptr(),
+            n_q2_blocks, 0,
+            self.k_codes2.data_ptr() if n_q2_blocks else 0,
+            self.v_codes2.data_ptr() if n_q2_blocks else 0,
+            self.k_params2.data_ptr() if n_q2_blocks else 0,
+            self.v_params2.data_ptr() if n_q2_blocks else 0)
 
     @property
     def n_blocks(self) -> int:
-        return self.n_q4_blocks + self.n_q8_blocks
+        return self.n_q4_blocks + self.n_q8_blocks + self.n_q2_blocks
 
     def nbytes(self) -> int:
         ts = (self.k_codes4, self.v_codes4, self.k_params4, self.v_params4, self.k_codes8,
-              self.v_codes8, self.k_params8, self.v_params8, self.mask)
+              self.v_codes8, self.k_params8, self.v_params8, self.k_codes2, self.v_codes2,
+              self.k_params2, self.v_params2, self.mask)
         return sum(t.numel() * t.element_size() for t in ts)
 
     # -- writes -------------------------------------------------------------

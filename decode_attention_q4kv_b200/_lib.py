@@ -29,7 +29,10 @@ class PoolDesc(ctypes.Structure):
                 ("k_params4", c_void_p), ("v_params4", c_void_p),
                 ("k_codes8", c_void_p), ("v_codes8", c_void_p),
                 ("k_params8", c_void_p), ("v_params8", c_void_p),
-                ("remap_mask", c_void_p), ("error_word", c_void_p)]
+                ("remap_mask", c_void_p), ("error_word", c_void_p),
+                ("n_q2_blocks", c_int32), ("reserved", c_int32),
+                ("k_codes2", c_void_p), ("v_codes2", c_void_p),
+                ("k_params2", c_void_p), ("v_params2", c_void_p)]
 
 
 class DecodePlan(ctypes.Structure):

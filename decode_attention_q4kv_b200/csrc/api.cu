@@ -15,12 +15,13 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 q4kv_status check_pool(const q4kv_pool* p) {
   if (p == nullptr) return Q4KV_ERR_INVALID_ARG;
   if ((p->value_format != Q4KV_FORMAT_INT && p->value_format != Q4KV_FORMAT_FP8) || p->n_kv_heads < 1 ||
-      p->n_q4_blocks < 0 || p->n_q8_blocks < 0 || (p->k_rotated != 0 && p->k_rotated != 1))
+      p->n_q4_blocks < 0 || p->n_q8_blocks < 0 || p->n_q2_blocks < 0 || p->reserved != 0 ||
+      (p->k_rotated != 0 && p->k_rotated != 1))
     return Q4KV_ERR_INVALID_ARG;
   const bool fp8 = p->value_format == Q4KV_FORMAT_FP8;
-  if (fp8 && (p->n_q4_blocks != 0 || p->k_rotated != 0)) return Q4KV_ERR_INVALID_ARG;
+  if (fp8 && (p->n_q4_blocks != 0 || p->n_q2_blocks != 0 || p->k_rotated != 0)) return Q4KV_ERR_INVALID_ARG;
   if (p->head_dim != 128 && p->head_dim != 256) return Q4KV_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(p->n_q4_blocks) + p->n_q8_blocks > (int64_t{1} << 31) / kBlockTokens)
+  if (static_cast<int64_t>(p->n_q4_blocks) + p->n_q8_blocks + p->n_q2_blocks > (int64_t{1} << 31) / kBlockTokens)
     return Q4KV_ERR_INVALID_ARG;
   if (p->n_q4_blocks > 0) {
     const void* a[4] = {p->k_codes4, p->v_codes4, p->k_params4, p->v_params4};
@@ -32,7 +33,12 @@ q4kv_status check_pool(const q4kv_pool* p) {
     for (int i = 0; i < (fp8 ? 2 : 4); ++i)   // an FP8 pool has no params
       if (a[i] == nullptr || !aligned(a[i], 16)) return Q4KV_ERR_INVALID_ARG;
   }
-  if (p->n_q4_blocks + p->n_q8_blocks > 0 &&
+  if (p->n_q2_blocks > 0) {
+    const void* a[4] = {p->k_codes2, p->v_codes2, p->k_params2, p->v_params2};
+    for (const void* x : a)
+      if (x == nullptr || !aligned(x, 16)) return Q4KV_ERR_INVALID_ARG;
+  }
+  if (p->n_q4_blocks + p->n_q8_blocks + p->n_q2_blocks > 0 &&
       (p->remap_mask == nullptr || !aligned(p->remap_mask, 16)))
     return Q4KV_ERR_INVALID_ARG;
   if (p->error_word != nullptr && !aligned(p->error_word, 4)) return Q4KV_ERR_INVALID_ARG;
@@ -93,7 +99,7 @@ int32_t q4kv_abi_version(void) { return Q4KV_ABI_VERSION; }
 q4kv_status q4kv_pool_array_bytes(int32_t head_dim, int32_t n_kv_heads, int64_t n_blocks,
                                   int32_t bits, size_t* codes_bytes, size_t* params_bytes) {
   if (codes_bytes == nullptr || params_bytes == nullptr || n_kv_heads < 1 || n_blocks < 0 ||
-      (bits != 4 && bits != 8))
+      (bits != 2 && bits != 4 && bits != 8))
     return Q4KV_ERR_INVALID_ARG;
   if (head_dim != 128 && head_dim != 256) return Q4KV_ERR_UNSUPPORTED;
   const size_t rows = static_cast<size_t>(n_blocks) * n_kv_heads * kBlockTokens;
@@ -171,7 +177,7 @@ q4kv_status q4kv_export_blocks_host_ids(const q4kv_pool* pool, const int32_t* bl
   if (st != Q4KV_OK || n_blocks == 0) return st;
   const PoolView v = view_of(*pool);
   for (int32_t i = 0; i < n_blocks; ++i)
-    if (block_ids[i] < 0 || block_ids[i] >= v.n_q4 + v.n_q8) return Q4KV_ERR_INVALID_ARG;
+    if (block_ids[i] < 0 || block_ids[i] >= v.n_blocks()) return Q4KV_ERR_INVALID_ARG;
   host_headers(v, block_ids, n_blocks, static_cast<uint8_t*>(host_images), true);
   return from_cuda(copy_pages(v, block_ids, n_blocks, static_cast<uint8_t*>(host_images), true, as_stream(stream)));
 }
@@ -183,7 +189,7 @@ q4kv_status q4kv_import_blocks_host_ids(const q4kv_pool* pool, const void* host_
   if (st != Q4KV_OK || n_blocks == 0) return st;
   const PoolView v = view_of(*pool);
   for (int32_t i = 0; i < n_blocks; ++i)
-    if (block_ids[i] < 0 || block_ids[i] >= v.n_q4 + v.n_q8) return Q4KV_ERR_INVALID_ARG;
+    if (block_ids[i] < 0 || block_ids[i] >= v.n_blocks()) return Q4KV_ERR_INVALID_ARG;
   uint8_t* img = static_cast<uint8_t*>(const_cast<void*>(host_images));
   if (!host_headers(v, block_ids, n_blocks, img, false)) return Q4KV_ERR_INVALID_ARG;
   return from_cuda(copy_pages(v, block_ids, n_blocks, img, false, as_stream(stream)));
@@ -321,11 +327,12 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
   int64_t s = n_splits;
   if (s == 0) {
     // persistent CTAs (one per SM) take items (sequence, KV head, split) in
-    // waves; cost = waves * (blocks per item + per-item overhead).  The
-    // overhead (query preparation, cross-warp merge, partial write) is 3.2
-    // block-times, fitted to decode times measured with forced split counts
-    // on the Gemma-, Llama- and Qwen-shaped layers and the batch/context
-    // sweep; with it the choice was the fastest measured split on each.
+    // waves; cost = waves * (blocks per item + per-item cost).  The per-item
+    // cost (what an item boundary costs the consumer warps: loading the next
+    // item's query operands, handing the state to the aux warp that merges
+    // it) is 0.9 block-time, fitted to decode times measured with forced
+    // split counts on the Gemma-, Llama- and Qwen-shaped layers and the
+    // batch/context sweep.
     const int64_t pairs = static_cast<int64_t>(batch > 0 ? batch : 1) * n_kv_heads;
     double best = 1e300;
     s = 1;
@@ -334,7 +341,7 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
       if ((nb + bps - 1) / bps != cand) continue;         // each distinct split only once
       const int64_t items = pairs * cand;
       const int64_t waves = (items + num_sms - 1) / num_sms;
-      const double cost = static_cast<double>(waves) * (static_cast<double>(bps) + 3.2);
+      const double cost = static_cast<double>(waves) * (static_cast<double>(bps) + 0.9);
       if (cost < best - 1e-9) {
         best = cost;
         s = cand;
@@ -388,11 +395,13 @@ q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan*
   if (q == nullptr || block_tables == nullptr || seq_lens == nullptr || out == nullptr ||
       !aligned(q, 16) || !aligned(block_tables, 16) || !aligned(seq_lens, 4) || !aligned(out, 16))
     return Q4KV_ERR_INVALID_ARG;
-  if (pool->n_q4_blocks + pool->n_q8_blocks == 0) return Q4KV_ERR_INVALID_ARG;
+  if (pool->n_q4_blocks + pool->n_q8_blocks + pool->n_q2_blocks == 0) return Q4KV_ERR_INVALID_ARG;
+  // the CUDA-core variant reads 4- and 8-bit blocks only
+  if (plan->kernel == 0 && pool->n_q2_blocks > 0) return Q4KV_ERR_UNSUPPORTED;
   // TMA row coordinates are int32: (blocks of one width) x heads x 256 < 2^31
-  const int64_t code_rows =
-      static_cast<int64_t>(pool->n_q4_blocks > pool->n_q8_blocks ? pool->n_q4_blocks : pool->n_q8_blocks) *
-      pool->n_kv_heads * kBlockTokens;
+  int64_t widest = pool->n_q4_blocks > pool->n_q8_blocks ? pool->n_q4_blocks : pool->n_q8_blocks;
+  if (pool->n_q2_blocks > widest) widest = pool->n_q2_blocks;
+  const int64_t code_rows = widest * pool->n_kv_heads * kBlockTokens;
   if (code_rows >= (int64_t{1} << 31)) return Q4KV_ERR_UNSUPPORTED;
   // the FP8 comparison cache is read by the tensor-core kernel only
   if (pool->value_format == Q4KV_FORMAT_FP8 && plan->kernel != 1) return Q4KV_ERR_UNSUPPORTED;

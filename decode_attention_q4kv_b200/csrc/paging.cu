@@ -8,7 +8,8 @@
 // storage tier behind it is the caller's).  A block travels as an image: a
 // 16-byte header and then the block's sections byte for byte as the pool
 // holds them -- K codes, V codes, K params, V params (not for FP8 pools), the
-// 32-byte remap mask.
+// 32-byte remap mask; its class tag is the block's code width (2, 4 or 8) or
+// 0x108 for an FP8 block.
 //
 // Two ways to move them.  With the block ids on the device, one kernel moves
 // any number of blocks in either direction, reading or writing the host side
@@ -37,27 +38,40 @@ struct ImageWords {
   __host__ __device__ int64_t total() const { return 1 + 2 * codes + 2 * params + 2; }
 };
 
-__host__ __device__ inline ImageWords image_words(int d, int hkv, bool is4, bool fp8) {
+// bits: the block's code width (2, 4 or 8; FP8 blocks are 8 bits wide)
+__host__ __device__ inline ImageWords image_words(int d, int hkv, int bits, bool fp8) {
   ImageWords w;
-  w.codes = static_cast<int64_t>(hkv) * kBlockTokens * (is4 ? d / 2 : d) / 16;
+  w.codes = static_cast<int64_t>(hkv) * kBlockTokens * (d * bits / 8) / 16;
   w.params = fp8 ? 0 : static_cast<int64_t>(hkv) * kBlockTokens * (d / kGroup) * 4 / 16;
   return w;
 }
 
-__device__ __forceinline__ uint32_t class_tag(bool is4, bool fp8) { return fp8 ? 0x108u : (is4 ? 4u : 8u); }
+__host__ __device__ inline uint32_t class_tag(int bits, bool fp8) { return fp8 ? 0x108u : static_cast<uint32_t>(bits); }
+
+// The arrays and array index of a block of the pool's class `bits`.
+struct ClassArrays {
+  uint8_t *kc, *vc;
+  void *kp, *vp;
+  int64_t phys;
+};
+__host__ __device__ inline ClassArrays class_arrays(const PoolView& p, int32_t blk, int bits) {
+  if (bits == 4) return {p.k_codes4, p.v_codes4, p.k_params4, p.v_params4, blk};
+  if (bits == 8) return {p.k_codes8, p.v_codes8, p.k_params8, p.v_params8, static_cast<int64_t>(blk) - p.n_q4};
+  return {p.k_codes2, p.v_codes2, p.k_params2, p.v_params2, static_cast<int64_t>(blk) - p.n_q4 - p.n_q8};
+}
 
 // Word w (1 <= w < total) of block blk's image, as a pointer into the pool.
-__device__ __forceinline__ uint4* pool_word(const PoolView& p, int32_t blk, bool is4, const ImageWords& iw,
+__device__ __forceinline__ uint4* pool_word(const PoolView& p, int32_t blk, int bits, const ImageWords& iw,
                                             int64_t w) {
-  const int64_t phys = is4 ? blk : blk - p.n_q4;
+  const ClassArrays a = class_arrays(p, blk, bits);
   w -= 1;
-  if (w < iw.codes) return reinterpret_cast<uint4*>(is4 ? p.k_codes4 : p.k_codes8) + phys * iw.codes + w;
+  if (w < iw.codes) return reinterpret_cast<uint4*>(a.kc) + a.phys * iw.codes + w;
   w -= iw.codes;
-  if (w < iw.codes) return reinterpret_cast<uint4*>(is4 ? p.v_codes4 : p.v_codes8) + phys * iw.codes + w;
+  if (w < iw.codes) return reinterpret_cast<uint4*>(a.vc) + a.phys * iw.codes + w;
   w -= iw.codes;
-  if (w < iw.params) return reinterpret_cast<uint4*>(is4 ? p.k_params4 : p.k_params8) + phys * iw.params + w;
+  if (w < iw.params) return reinterpret_cast<uint4*>(a.kp) + a.phys * iw.params + w;
   w -= iw.params;
-  if (w < iw.params) return reinterpret_cast<uint4*>(is4 ? p.v_params4 : p.v_params8) + phys * iw.params + w;
+  if (w < iw.params) return reinterpret_cast<uint4*>(a.vp) + a.phys * iw.params + w;
   w -= iw.params;
   return reinterpret_cast<uint4*>(p.mask + static_cast<int64_t>(blk) * kMaskWords) + w;
 }
@@ -79,22 +93,22 @@ __global__ void __launch_bounds__(kPageThreads) page_kernel(const __grid_constan
     const int64_t i = ch / chunks_per_image;
     const int64_t w0 = (ch - i * chunks_per_image) * kChunk + threadIdx.x;
     const int32_t blk = __ldg(ids + i);
-    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+    if (blk < 0 || blk >= pool.n_blocks()) {
       if (w0 == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
       continue;
     }
-    const bool is4 = !fp8 && blk < pool.n_q4;
-    const ImageWords iw = image_words(d, hkv, is4, fp8);
+    const int bits = pool.bits_of(blk);
+    const ImageWords iw = image_words(d, hkv, bits, fp8);
     const int64_t total = iw.total();
     uint4* img = host + i * stride_words;
-    const uint4 hdr = make_uint4(kImageMagic, class_tag(is4, fp8) | static_cast<uint32_t>(d) << 16,
+    const uint4 hdr = make_uint4(kImageMagic, class_tag(bits, fp8) | static_cast<uint32_t>(d) << 16,
                                  static_cast<uint32_t>(hkv), static_cast<uint32_t>(blk));
     uint4 val[kPageUnroll];
     if constexpr (EXPORT) {
 #pragma unroll
       for (int u = 0; u < kPageUnroll; ++u) {
         const int64_t w = w0 + u * kPageThreads;
-        if (w > 0 && w < total) val[u] = __ldg(pool_word(pool, blk, is4, iw, w));
+        if (w > 0 && w < total) val[u] = __ldg(pool_word(pool, blk, bits, iw, w));
       }
 #pragma unroll
       for (int u = 0; u < kPageUnroll; ++u) {
@@ -116,7 +130,7 @@ __global__ void __launch_bounds__(kPageThreads) page_kernel(const __grid_constan
 #pragma unroll
       for (int u = 0; u < kPageUnroll; ++u) {
         const int64_t w = w0 + u * kPageThreads;
-        if (w > 0 && w < total) *pool_word(pool, blk, is4, iw, w) = val[u];
+        if (w > 0 && w < total) *pool_word(pool, blk, bits, iw, w) = val[u];
       }
     }
   }
@@ -134,22 +148,20 @@ __global__ void __launch_bounds__(kPageThreads) page_kernel(const __grid_constan
 namespace {
 
 struct HostClass {
-  bool is4;
-  int64_t phys;
+  int bits;
   ImageWords iw;
 };
 
 HostClass host_class(const PoolView& p, int32_t blk) {
   HostClass c;
-  c.is4 = !p.fp8 && blk < p.n_q4;
-  c.phys = c.is4 ? blk : blk - p.n_q4;
-  c.iw = image_words(p.head_dim, p.n_kv_heads, c.is4, p.fp8 != 0);
+  c.bits = p.bits_of(blk);
+  c.iw = image_words(p.head_dim, p.n_kv_heads, c.bits, p.fp8 != 0);
   return c;
 }
 
 void host_header(const PoolView& p, int32_t blk, const HostClass& c, uint32_t out[4]) {
   out[0] = kImageMagic;
-  out[1] = (p.fp8 ? 0x108u : (c.is4 ? 4u : 8u)) | static_cast<uint32_t>(p.head_dim) << 16;
+  out[1] = class_tag(c.bits, p.fp8 != 0) | static_cast<uint32_t>(p.head_dim) << 16;
   out[2] = static_cast<uint32_t>(p.n_kv_heads);
   out[3] = static_cast<uint32_t>(blk);
 }
@@ -163,18 +175,17 @@ cudaError_t copy_pages(const PoolView& p, const int32_t* ids, int32_t n, uint8_t
   while (i < n) {
     const HostClass c = host_class(p, ids[i]);
     int32_t len = 1;   // the run: ids[i] + r for r < len, all of the same class
-    while (i + len < n && ids[i + len] == ids[i] + len && host_class(p, ids[i + len]).is4 == c.is4) ++len;
+    while (i + len < n && ids[i + len] == ids[i] + len && host_class(p, ids[i + len]).bits == c.bits) ++len;
     const int64_t cb = c.iw.codes * 16, pb = c.iw.params * 16;
+    const ClassArrays a = class_arrays(p, ids[i], c.bits);
     struct Sec {
       void* pool;
       int64_t bytes, image_off;
     } secs[5] = {
-        {(c.is4 ? p.k_codes4 : p.k_codes8) + c.phys * cb, cb, 16},
-        {(c.is4 ? p.v_codes4 : p.v_codes8) + c.phys * cb, cb, 16 + cb},
-        {static_cast<uint8_t*>(static_cast<void*>(c.is4 ? p.k_params4 : p.k_params8)) + c.phys * pb, pb,
-         16 + 2 * cb},
-        {static_cast<uint8_t*>(static_cast<void*>(c.is4 ? p.v_params4 : p.v_params8)) + c.phys * pb, pb,
-         16 + 2 * cb + pb},
+        {a.kc + a.phys * cb, cb, 16},
+        {a.vc + a.phys * cb, cb, 16 + cb},
+        {static_cast<uint8_t*>(a.kp) + a.phys * pb, pb, 16 + 2 * cb},
+        {static_cast<uint8_t*>(a.vp) + a.phys * pb, pb, 16 + 2 * cb + pb},
         {p.mask + static_cast<int64_t>(ids[i]) * kMaskWords, kMaskWords * 4, 16 + 2 * cb + 2 * pb},
     };
     for (const Sec& sec : secs) {
@@ -210,8 +221,9 @@ bool host_headers(const PoolView& p, const int32_t* ids, int32_t n, uint8_t* hos
 
 int64_t image_stride_bytes(const PoolView& pool) {
   const bool fp8 = pool.fp8 != 0;
-  const bool is4 = !fp8 && pool.n_q8 == 0;   // the largest class present
-  return image_words(pool.head_dim, pool.n_kv_heads, is4, fp8).total() * 16;
+  // the widest class present (a pool with no blocks: as if 4-bit)
+  const int bits = (fp8 || pool.n_q8 > 0) ? 8 : (pool.n_q4 > 0 || pool.n_q2 == 0 ? 4 : 2);
+  return image_words(pool.head_dim, pool.n_kv_heads, bits, fp8).total() * 16;
 }
 
 cudaError_t launch_page(const PoolView& pool, const int32_t* ids, int32_t n, void* host, bool to_host,

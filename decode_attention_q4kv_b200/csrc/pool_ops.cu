@@ -15,7 +15,7 @@ namespace q4kv {
 namespace {
 
 __global__ void invalidate_kernel(PoolView pool, const int64_t* __restrict__ slot_ids, int64_t n) {
-  const int64_t n_slots = static_cast<int64_t>(pool.n_q4 + pool.n_q8) * kBlockTokens;
+  const int64_t n_slots = static_cast<int64_t>(pool.n_blocks()) * kBlockTokens;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t s = slot_ids[i];

@@ -34,6 +34,16 @@ struct PoolView {
   __half2* v_params8;
   uint32_t* mask;
   uint32_t* error_word;
+  int32_t n_q2;       // 2-bit blocks: unified ids [n_q4 + n_q8, n_q4 + n_q8 + n_q2)
+  uint8_t* k_codes2;
+  uint8_t* v_codes2;
+  __half2* k_params2;
+  __half2* v_params2;
+  __host__ __device__ __forceinline__ int n_blocks() const { return n_q4 + n_q8 + n_q2; }
+  // code bits of a valid unified block id
+  __host__ __device__ __forceinline__ int bits_of(int blk) const {
+    return blk < n_q4 ? 4 : (blk < n_q4 + n_q8 ? 8 : 2);
+  }
 };
 
 inline PoolView view_of(const q4kv_pool& p) {
@@ -54,6 +64,11 @@ inline PoolView view_of(const q4kv_pool& p) {
   v.v_params8 = reinterpret_cast<__half2*>(p.v_params8);
   v.mask = p.remap_mask;
   v.error_word = p.error_word;
+  v.n_q2 = p.n_q2_blocks;
+  v.k_codes2 = p.k_codes2;
+  v.v_codes2 = p.v_codes2;
+  v.k_params2 = reinterpret_cast<__half2*>(p.k_params2);
+  v.v_params2 = reinterpret_cast<__half2*>(p.v_params2);
   return v;
 }
 

@@ -475,12 +475,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const uint4 k0 = lds16(src), k1 = lds16(src + 16);
       const uint4 v0 = lds16(src + kQHalf), v1 = lds16(src + kQHalf + 16);
       const int h = h0 + hh;
-      if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+      if (blk < 0 || blk >= pool.n_blocks()) {
         if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
       } else {
         const int slot = static_cast<int>(t % kBlockTokens);
-        const bool is8 = MIXED && blk >= pool.n_q4;   // a pool without 8-bit blocks drops that path
-        const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+        // a pool with only 4-bit blocks drops the other widths' paths
+        const int bits = MIXED ? pool.bits_of(blk) : 4;
+        const bool is8 = bits == 8;
+        const int64_t phys = bits == 4 ? blk : (is8 ? blk - pool.n_q4 : blk - pool.n_q4 - pool.n_q8);
         const int64_t row = (phys * hkv + h) * kBlockTokens + slot;   // (block, head, slot)
         float2 xk[8], xv[8];
         unpack16<InT>(k0, k1, xk);
@@ -496,6 +498,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
           if (is8)
             encode_kv<8>(xk, ks, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
                          pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+          else if (MIXED && bits == 2)
+            encode_kv<2>(xk, ks, xv, j, valid, pool.k_codes2 + row * (D / 4), pool.k_params2 + row * S::NG,
+                         pool.v_codes2 + row * (D / 4), pool.v_params2 + row * S::NG);
           else
             encode_kv<4>(xk, ks, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
                          pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
@@ -557,7 +562,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ Poo
       continue;
     }
     const int32_t blk = __ldg(tables + static_cast<int64_t>(b) * max_blocks + p / kBlockTokens);
-    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+    if (blk < 0 || blk >= pool.n_blocks()) {
       if (lane == 0 && hg == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
       continue;
     }
@@ -571,8 +576,9 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ Poo
     const uint4 k1 = __ldg(reinterpret_cast<const uint4*>(k + src) + 1);
     const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(v + src));
     const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(v + src) + 1);
-    const bool is8 = blk >= pool.n_q4;
-    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+    const int bits = pool.bits_of(blk);
+    const bool is8 = bits == 8;
+    const int64_t phys = bits == 4 ? blk : (is8 ? blk - pool.n_q4 : blk - pool.n_q4 - pool.n_q8);
     const int64_t row = (phys * hkv + hs) * kBlockTokens + slot;   // (block, head, slot)
     float2 xk[8], xv[8];
     unpack16<InT>(k0, k1, xk);
@@ -591,6 +597,9 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ Poo
     if (is8)
       encode_kv<8>(xk, ks, xv, j, valid, pool.k_codes8 + row * D, pool.k_params8 + row * S::NG,
                    pool.v_codes8 + row * D, pool.v_params8 + row * S::NG);
+    else if (bits == 2)
+      encode_kv<2>(xk, ks, xv, j, valid, pool.k_codes2 + row * (D / 4), pool.k_params2 + row * S::NG,
+                   pool.v_codes2 + row * (D / 4), pool.v_params2 + row * S::NG);
     else
       encode_kv<4>(xk, ks, xv, j, valid, pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG,
                    pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG);
@@ -728,7 +737,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
     OutT* vd = v_out + out_row * D + j * kEPL;
     const int32_t blk = __ldg(block_ids + li);
     float x[kEPL];
-    if (blk < 0 || blk >= pool.n_q4 + pool.n_q8) {
+    if (blk < 0 || blk >= pool.n_blocks()) {
       if (lane == 0) raise_error(pool.error_word, Q4KV_DEVERR_BLOCK_ID);
 #pragma unroll
       for (int i = 0; i < kEPL; ++i) x[i] = 0.0f;
@@ -736,8 +745,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
       store16<OutT>(vd, x);
       continue;
     }
-    const bool is8 = blk >= pool.n_q4;
-    const int64_t phys = is8 ? blk - pool.n_q4 : blk;
+    const int bits = pool.bits_of(blk);
+    const bool is8 = bits == 8, is2 = bits == 2;
+    const int64_t phys = bits == 4 ? blk : (is8 ? blk - pool.n_q4 : blk - pool.n_q4 - pool.n_q8);
     const int64_t row = (phys * hkv + h) * kBlockTokens + slot;
     const bool masked =
         (pool.mask[static_cast<int64_t>(blk) * kMaskWords + slot / 32] >> (slot % 32)) & 1u;
@@ -746,6 +756,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
       decode_fp8_lane(pool.k_codes8 + row * D, j, x);
     else if (is8)
       decode_lane<8>(pool.k_codes8 + row * D, pool.k_params8 + row * S::NG, j, x);
+    else if (is2)
+      decode_lane<2>(pool.k_codes2 + row * (D / 4), pool.k_params2 + row * S::NG, j, x);
     else
       decode_lane<4>(pool.k_codes4 + row * (D / 2), pool.k_params4 + row * S::NG, j, x);
     if (unrotate_k && pool.k_rotated) rotate_vector<D>(x, j);
@@ -759,6 +771,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView pool,
       decode_fp8_lane(pool.v_codes8 + row * D, j, x);
     else if (is8)
       decode_lane<8>(pool.v_codes8 + row * D, pool.v_params8 + row * S::NG, j, x);
+    else if (is2)
+      decode_lane<2>(pool.v_codes2 + row * (D / 4), pool.v_params2 + row * S::NG, j, x);
     else
       decode_lane<4>(pool.v_codes4 + row * (D / 2), pool.v_params4 + row * S::NG, j, x);
     if (masked) {
@@ -1125,7 +1139,7 @@ cudaError_t launch_quantize(const PoolView& pool, const void* k, const void* v, 
   } while (0)
 #define Q4KV_LAUNCH_QR(DD, T)                                   \
   do {                                                          \
-    const bool mixed = pool.n_q8 > 0;                           \
+    const bool mixed = pool.n_q8 > 0 || pool.n_q2 > 0;          \
     if (pool.k_rotated && mixed) Q4KV_LAUNCH_Q(DD, T, true, true);        \
     else if (pool.k_rotated) Q4KV_LAUNCH_Q(DD, T, true, false);           \
     else if (mixed) Q4KV_LAUNCH_Q(DD, T, false, true);                    \

@@ -68,7 +68,7 @@
 extern "C" {
 #endif
 
-#define Q4KV_ABI_VERSION 3
+#define Q4KV_ABI_VERSION 4
 #define Q4KV_BLOCK_TOKENS 256
 #define Q4KV_GROUP 64
 #define Q4KV_MASK_WORDS 8            /* uint32 words of remap mask per block */
@@ -84,9 +84,9 @@ typedef enum {
 } q4kv_status;
 
 /* Bits of pool->error_word. */
-#define Q4KV_DEVERR_BLOCK_ID 1u  /* a block id outside [0, n_q4_blocks + n_q8_blocks) */
+#define Q4KV_DEVERR_BLOCK_ID 1u  /* a block id outside [0, n_q4_blocks + n_q8_blocks + n_q2_blocks) */
 #define Q4KV_DEVERR_SEQ_LEN 2u   /* seq_len < 0 or > max_blocks_per_seq * 256 */
-#define Q4KV_DEVERR_SLOT_ID 4u   /* a slot id outside [0, 256 * (n_q4_blocks + n_q8_blocks)) */
+#define Q4KV_DEVERR_SLOT_ID 4u   /* a slot id outside [0, 256 * (n_q4 + n_q8 + n_q2 blocks)) */
 #define Q4KV_DEVERR_TIMEOUT 8u   /* a bounded device-side wait gave up */
 #define Q4KV_DEVERR_IMAGE 16u    /* a block image or card whose header or layout does not fit */
 #define Q4KV_DEVERR_WIDTH 32u    /* a card token width outside {2, 4, 8, 16} */
@@ -95,16 +95,16 @@ typedef enum { Q4KV_F16 = 0, Q4KV_BF16 = 1, Q4KV_F32 = 2 } q4kv_dtype;
 
 /*
  * Value formats of a pool (q4kv_pool.value_format).
- *   Q4KV_FORMAT_INT  4-bit (and optional 8-bit) integer codes with a scale and
- *                    a zero per group of 64, as described above.
+ *   Q4KV_FORMAT_INT  4-bit (and optional 8- and 2-bit) integer codes with a
+ *                    scale and a zero per group of 64, as described above.
  *   Q4KV_FORMAT_FP8  the FP8 cache the 4-bit cache is compared against ([UQ]
  *                    "技術/ビジネス面": TTFT and throughput are reported against
  *                    an FP8 KV cache).  Every value is one OCP E4M3 byte
  *                    (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
  *                    no infinities; largest finite 448) holding the input value
  *                    rounded to nearest, ties to even, saturated to +-448; no
- *                    scale and no rotation.  Such a pool has n_q4_blocks = 0 and
- *                    k_rotated = 0, keeps its codes in k_codes8 / v_codes8
+ *                    scale and no rotation.  Such a pool has n_q4_blocks = 0,
+ *                    n_q2_blocks = 0 and k_rotated = 0, keeps its codes in k_codes8 / v_codes8
  *                    [n_q8][Hkv][256][D], and has no params (their pointers are
  *                    ignored).  Quantise, append, dequantise, invalidate and
  *                    decode all accept it.
@@ -113,16 +113,23 @@ typedef enum { Q4KV_F16 = 0, Q4KV_BF16 = 1, Q4KV_F32 = 2 } q4kv_dtype;
 #define Q4KV_FORMAT_FP8 1
 
 /*
- * The paged pool ([AMBP] sec. 2.1 items 1-2; 8-bit blocks: [QKVS]).
+ * The paged pool ([AMBP] sec. 2.1 items 1-2; 8- and 2-bit blocks: [QKVS]
+ * "Méthodologie", widths from {2, 4, 8, FP16} in one cache, here per block).
  * Unified block ids: [0, n_q4_blocks) are 4-bit blocks, stored at index id
  * of the *4 arrays; [n_q4_blocks, n_q4_blocks + n_q8_blocks) are 8-bit blocks,
- * stored at index id - n_q4_blocks of the *8 arrays.
+ * stored at index id - n_q4_blocks of the *8 arrays; the next n_q2_blocks ids
+ * are 2-bit blocks, stored at index id - n_q4_blocks - n_q8_blocks of the *2
+ * arrays.  Every class codes a group of 64 values with the same steps and
+ * L = 2^bits - 1 levels.
  * Every array pointer must be 16-byte aligned.  Layouts (row-major):
- *   k_codes4, v_codes4   uint8 [n_q4][Hkv][256][D/2]
+ *   k_codes4, v_codes4   uint8 [n_q4][Hkv][256][D/2]    (element 2i in the low nibble of byte i)
  *   k_params4, v_params4 half2 [n_q4][Hkv][256][D/64]   (.x = scale, .y = zero)
  *   k_codes8, v_codes8   uint8 [n_q8][Hkv][256][D]      (may be NULL if n_q8 == 0)
  *   k_params8, v_params8 half2 [n_q8][Hkv][256][D/64]
- *   remap_mask           uint32 [n_q4 + n_q8][8]; bit (s % 32) of word s / 32
+ *   k_codes2, v_codes2   uint8 [n_q2][Hkv][256][D/4]    (element 4i + m at bits 2m of byte i;
+ *                                                        may be NULL if n_q2 == 0)
+ *   k_params2, v_params2 half2 [n_q2][Hkv][256][D/64]
+ *   remap_mask           uint32 [n_q4 + n_q8 + n_q2][8]; bit (s % 32) of word s / 32
  *                        set = slot s of that block is remapped to the sentinel
  *   error_word           optional uint32 (NULL = do not report)
  * The descriptor itself is read on the host during each call and may be
@@ -141,6 +148,10 @@ typedef struct {
   void *k_params8, *v_params8;
   uint32_t *remap_mask;
   uint32_t *error_word;
+  int32_t n_q2_blocks;  /* >= 0; 0 for an FP8 pool */
+  int32_t reserved;     /* must be 0 */
+  uint8_t *k_codes2, *v_codes2;
+  void *k_params2, *v_params2;
 } q4kv_pool;
 
 /* Human-readable name of a status code (static storage). */
@@ -151,7 +162,7 @@ int32_t q4kv_abi_version(void);
 
 /*
  * Bytes of one codes array and of one params array for `n_blocks` blocks of
- * width `bits` (4 or 8), so a caller can size the pool ([AMBP] sec. 2.1
+ * width `bits` (2, 4 or 8), so a caller can size the pool ([AMBP] sec. 2.1
  * item 2: 144 bytes per token and KV head at D = 128, 4 bits, i.e. 71.875 %
  * below fp16).  Host-only; touches no device.
  */

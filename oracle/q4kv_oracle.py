@@ -48,6 +48,9 @@ design notes):
     stay where they are; one 256-bit mask per physical block, shared by
     all KV heads; writing a token into a slot makes the slot live again;
   * 8-bit blocks use the same steps with 255 levels, one code per byte;
+    2-bit blocks ([QKVS] widths from {2, 4, 8, FP16}, here a third block
+    class) the same steps with 3 levels, four codes per byte, element
+    4i + m at bits 2m of byte i (the nibble order, generalised);
   * the FP8 comparison cache stores each raw value as one OCP E4M3 byte
     (bias 7, 3 mantissa bits, no infinities, largest finite 448), rounded
     to nearest with ties to even and saturated to +-448; no scale, no
@@ -267,15 +270,18 @@ class OraclePool:
     """Host model of the paged cache.
 
     Unified block ids: [0, n_q4) are 4-bit blocks, [n_q4, n_q4 + n_q8) are
-    8-bit blocks.  Per block and KV head: codes [256][D/2] (4-bit) or
-    [256][D] (8-bit) and params [256][D/64][2] fp16 as (scale, zero).
-    mask[block][8] uint32: bit (slot mod 32) of word (slot / 32) set means
-    the slot has been remapped to the sentinel.
+    8-bit blocks, [n_q4 + n_q8, n_q4 + n_q8 + n_q2) are 2-bit blocks
+    ([QKVS] "Methodologie": widths from {2, 4, 8, FP16} in one cache; here
+    per block).  Per block and KV head: codes [256][D/2] (4-bit), [256][D]
+    (8-bit) or [256][D/4] (2-bit, element 4i + m at bits 2m of byte i) and
+    params [256][D/64][2] fp16 as (scale, zero).  mask[block][8] uint32:
+    bit (slot mod 32) of word (slot / 32) set means the slot has been
+    remapped to the sentinel.
     """
 
     def __init__(self, n_kv_heads: int, head_dim: int, n_q4: int, n_q8: int = 0,
-                 k_rotated: bool = True, fp8: bool = False):
-        if fp8 and (n_q4 or k_rotated):
+                 k_rotated: bool = True, fp8: bool = False, n_q2: int = 0):
+        if fp8 and (n_q4 or n_q2 or k_rotated):
             raise ValueError("an FP8 pool has only 8-bit blocks and raw keys")
         self.fp8 = fp8
         self.hkv = n_kv_heads
@@ -289,16 +295,37 @@ class OraclePool:
         self.params4 = {s: np.zeros((n_q4, n_kv_heads, T, ng, 2), np.float16) for s in "kv"}
         self.codes8 = {s: np.zeros((n_q8, n_kv_heads, T, head_dim), np.uint8) for s in "kv"}
         self.params8 = {s: np.zeros((n_q8, n_kv_heads, T, ng, 2), np.float16) for s in "kv"}
-        self.mask = np.zeros((n_q4 + n_q8, MASK_WORDS), np.uint32)
+        self.n_q2 = n_q2
+        self.codes2 = {s: np.zeros((n_q2, n_kv_heads, T, head_dim // 4), np.uint8) for s in "kv"}
+        self.params2 = {s: np.zeros((n_q2, n_kv_heads, T, ng, 2), np.float16) for s in "kv"}
+        self.mask = np.zeros((n_q4 + n_q8 + n_q2, MASK_WORDS), np.uint32)
 
     @property
     def n_blocks(self) -> int:
-        return self.n_q4 + self.n_q8
+        return self.n_q4 + self.n_q8 + self.n_q2
 
     def bits(self, blk: int) -> int:
         if not 0 <= blk < self.n_blocks:
             raise IndexError(f"block id {blk} outside [0, {self.n_blocks})")
-        return 4 if blk < self.n_q4 else 8
+        if blk < self.n_q4:
+            return 4
+        return 8 if blk < self.n_q4 + self.n_q8 else 2
+
+    def _store(self, name: str, blk: int, slots, codes: np.ndarray, par: np.ndarray) -> None:
+        """Write codes [Hkv][n][D] (unpacked) and params [Hkv][n][ng][2] of
+        `slots` of block `blk` in the block's width."""
+        bits = self.bits(blk)
+        if bits == 4:
+            self.codes4[name][blk, :, slots] = pack_nibbles(codes)
+            self.params4[name][blk, :, slots] = par
+        elif bits == 8:
+            i8 = blk - self.n_q4
+            self.codes8[name][i8, :, slots] = codes
+            self.params8[name][i8, :, slots] = par
+        else:
+            i2 = blk - self.n_q4 - self.n_q8
+            self.codes2[name][i2, :, slots] = pack_codes(codes, 2)
+            self.params2[name][i2, :, slots] = par
 
     # -- writes ------------------------------------------------------------
     def quantize_blocks(self, k: np.ndarray, v: np.ndarray, dtype: str,
@@ -326,13 +353,7 @@ class OraclePool:
                 codes, s_h, z_h = quantize_groups(x, bits)       # [cnt][Hkv][D]
                 codes = codes.transpose(1, 0, 2)                  # [Hkv][cnt][D]
                 par = np.stack([s_h, z_h], axis=-1).transpose(1, 0, 2, 3)
-                if bits == 4:
-                    self.codes4[name][blk, :, : t1 - t0] = pack_nibbles(codes)
-                    self.params4[name][blk, :, : t1 - t0] = par
-                else:
-                    i8 = blk - self.n_q4
-                    self.codes8[name][i8, :, : t1 - t0] = codes
-                    self.params8[name][i8, :, : t1 - t0] = par
+                self._store(name, blk, slice(0, t1 - t0), codes, par)
             for slot in range(t1 - t0):
                 self.mask[blk, slot // 32] &= np.uint32(~(1 << (slot % 32)) & 0xFFFFFFFF)
 
@@ -363,13 +384,7 @@ class OraclePool:
                         continue
                     codes, s_h, z_h = quantize_groups(x, bits)
                     par = np.stack([s_h[0], z_h[0]], axis=-1)  # [Hkv][D/64][2]
-                    if bits == 4:
-                        self.codes4[name][blk, :, slot] = pack_nibbles(codes[0])
-                        self.params4[name][blk, :, slot] = par
-                    else:
-                        i8 = blk - self.n_q4
-                        self.codes8[name][i8, :, slot] = codes[0]
-                        self.params8[name][i8, :, slot] = par
+                    self._store(name, blk, slice(slot, slot + 1), codes[0][:, None], par[:, None])
                 self.mask[blk, slot // 32] &= np.uint32(~(1 << (slot % 32)) & 0xFFFFFFFF)
 
     def invalidate_slots(self, slot_ids: Sequence[int]) -> None:
@@ -382,13 +397,13 @@ class OraclePool:
 
     # -- block images: paging between device and host [AMBP 2.1 items 1, 3; 5] --
     def block_class(self, blk: int) -> int:
-        """Class tag of a block's image: 4 (4-bit), 8 (8-bit) or 0x108 (FP8)."""
+        """Class tag of a block's image: 2, 4 or 8 (code width) or 0x108 (FP8)."""
         bits = self.bits(blk)
         return 0x108 if self.fp8 else bits
 
     def image_sections(self, cls: int):
         """(name, bytes) of the sections of an image of class `cls`, in order."""
-        row = self.d // 2 if cls == 4 else self.d
+        row = {2: self.d // 4, 4: self.d // 2}.get(cls, self.d)
         codes = self.hkv * BLOCK_TOKENS * row
         params = 0 if cls == 0x108 else self.hkv * BLOCK_TOKENS * (self.d // GROUP) * 4
         secs = [("header", IMAGE_HEADER_BYTES), ("k_codes", codes), ("v_codes", codes)]
@@ -398,7 +413,8 @@ class OraclePool:
 
     def image_stride(self) -> int:
         """Bytes between consecutive images: the largest class of the pool."""
-        classes = [0x108] if self.fp8 else ([4] if self.n_q4 else []) + ([8] if self.n_q8 else [])
+        classes = [0x108] if self.fp8 else (([4] if self.n_q4 else []) + ([8] if self.n_q8 else [])
+                                             + ([2] if self.n_q2 else []))
         return max(sum(b for _, b in self.image_sections(c)) for c in classes or [4])
 
     def _block_arrays(self, blk: int):
@@ -406,6 +422,10 @@ class OraclePool:
         if self.bits(blk) == 4:
             arrs = [self.codes4["k"][blk], self.codes4["v"][blk],
                     self.params4["k"][blk], self.params4["v"][blk]]
+        elif self.bits(blk) == 2:
+            i2 = blk - self.n_q4 - self.n_q8
+            arrs = [self.codes2["k"][i2], self.codes2["v"][i2],
+                    self.params2["k"][i2], self.params2["v"][i2]]
         else:
             i8 = blk - self.n_q4
             arrs = [self.codes8["k"][i8], self.codes8["v"][i8]]
@@ -461,6 +481,10 @@ class OraclePool:
         if self.bits(blk) == 4:
             codes = unpack_nibbles(self.codes4[name][blk])
             par = self.params4[name][blk]
+        elif self.bits(blk) == 2:
+            i2 = blk - self.n_q4 - self.n_q8
+            codes = unpack_codes(self.codes2[name][i2], 2)
+            par = self.params2[name][i2]
         else:
             codes = self.codes8[name][blk - self.n_q4]
             par = self.params8[name][blk - self.n_q4]

@@ -25,10 +25,10 @@ def host(t: torch.Tensor):
 
 
 def oracle_pool(k: torch.Tensor, v: torch.Tensor, ids, n_q4: int, n_q8: int = 0,
-                rotated: bool = True) -> O.OraclePool:
+                rotated: bool = True, n_q2: int = 0) -> O.OraclePool:
     kh, dt = host(k)
     vh, _ = host(v)
-    pool = O.OraclePool(k.shape[1], k.shape[2], n_q4, n_q8, k_rotated=rotated)
+    pool = O.OraclePool(k.shape[1], k.shape[2], n_q4, n_q8, k_rotated=rotated, n_q2=n_q2)
     pool.quantize_blocks(kh, vh, dt, [int(i) for i in ids])
     return pool
 
@@ -44,6 +44,12 @@ def assert_pool_equal(gpu, ref: O.OraclePool, blocks=None):
                 g_par = getattr(gpu, f"{name}_params4")[blk].cpu().numpy()
                 r_codes = ref.codes4[name][blk]
                 r_par = ref.params4[name][blk]
+            elif blk >= ref.n_q4 + ref.n_q8:
+                i = blk - ref.n_q4 - ref.n_q8
+                g_codes = getattr(gpu, f"{name}_codes2")[i].cpu().numpy()
+                g_par = getattr(gpu, f"{name}_params2")[i].cpu().numpy()
+                r_codes = ref.codes2[name][i]
+                r_par = ref.params2[name][i]
             else:
                 i = blk - ref.n_q4
                 g_codes = getattr(gpu, f"{name}_codes8")[i].cpu().numpy()

@@ -726,3 +726,124 @@ def test_card_round_trip_bounds(dtype):
         sk = (kr.max(-1) - kr.min(-1)) / L
         lim = np.sqrt(64 * ((0.5 * sk + L * sk * 2.0 ** -10 + np.abs(kr.min(-1)) * 2.0 ** -10) ** 2).sum(-1))
         assert (np.linalg.norm(k_hat[t] - x_k[t], axis=-1) <= lim * 1.001 + 1e-4).all()
+
+
+# ---------------------------------------------------------------------------
+# 2-bit blocks in the paged pool (QKVShare, "Methodologie": widths {2, 4, 8,
+# FP16} in one cache; a third block class after the 4- and 8-bit ones)
+# ---------------------------------------------------------------------------
+
+def _pool3(seed, d=128, hkv=2, n=700, rotated=True):
+    """4-, 8- and 2-bit blocks in one pool: ids 0-1 4-bit, 2 8-bit, 3-4 2-bit."""
+    k, v = _rand_kv(n, hkv, d, seed)
+    pool = O.OraclePool(hkv, d, 2, 1, k_rotated=rotated, n_q2=2)
+    pool.quantize_blocks(k, v, "fp16", [3, 1, 4])                # 2-bit, 4-bit, 2-bit
+    return pool, k, v
+
+
+def test_2bit_ids_follow_the_8bit_ones():
+    pool = O.OraclePool(2, 128, 3, 2, n_q2=4)
+    assert pool.n_blocks == 9
+    assert [pool.bits(b) for b in range(9)] == [4, 4, 4, 8, 8, 2, 2, 2, 2]
+    with pytest.raises(IndexError):
+        pool.bits(9)
+
+
+def test_2bit_ramp_codes_and_byte_layout():
+    """Values z + k s (k = 0..3, representable s and z) give codes k; the
+    stored byte i holds elements 4i .. 4i+3 at bits 0, 2, 4, 6."""
+    z, s = np.float32(-1.5), np.float32(0.5)
+    d, hkv = 128, 1
+    j = np.arange(d)
+    pattern = (j * 7 + j // 5) % 4                    # not a plain repeat: catches swapped elements
+    x = (z + pattern * s).astype(np.float16)
+    k = np.tile(x, (256, hkv, 1)).reshape(256, hkv, d)
+    pool = O.OraclePool(hkv, d, 0, 0, k_rotated=False, n_q2=1)
+    pool.quantize_blocks(k, k, "fp16", [0])
+    for name in "kv":
+        byte = pool.codes2[name][0, 0, 0]                # slot 0 of head 0
+        want = [int(pattern[4 * i]) | int(pattern[4 * i + 1]) << 2 | int(pattern[4 * i + 2]) << 4
+                | int(pattern[4 * i + 3]) << 6 for i in range(d // 4)]
+        assert list(byte) == want
+        par = pool.params2[name][0, 0, 0]
+        assert np.all(par[:, 0] == np.float16(s)) and np.all(par[:, 1] == np.float16(z))
+
+
+def test_2bit_codes_are_the_nearest_level():
+    """Brute force: each code is the level k in {0..3} nearest to x in exact
+    arithmetic, z_h + k s_h (elements within 1e-6 s of a midpoint skipped)."""
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((400, 128)) * rng.choice([0.05, 1, 20], size=(400, 1))).astype(np.float32)
+    codes, s_h, z_h = O.quantize_groups(x, 2)
+    xs = x.reshape(400, 2, 64).astype(np.float64)
+    s = s_h.astype(np.float64)[..., None]
+    z = z_h.astype(np.float64)[..., None]
+    lv = z[..., None] + s[..., None] * np.arange(4)          # [400][2][1][4]
+    dist = np.abs(xs[..., None] - lv)
+    near = np.argmin(dist, axis=-1)
+    srt = np.sort(dist, axis=-1)
+    clear = (srt[..., 1] - srt[..., 0]) > 1e-6 * s
+    got = codes.reshape(400, 2, 64)
+    assert np.all(got[clear & (s > 0)] == near[clear & (s > 0)])
+    assert clear.mean() > 0.99
+
+
+def test_2bit_blocks_dequantise_by_independent_unpacking():
+    """K_hat / V_hat of a 2-bit block rebuilt from the raw bytes with shifts
+    and masks written here, scale and zero read from the params."""
+    pool, _, _ = _pool3(22)
+    for blk in (3, 4):
+        kh, vh = pool.dequantize_block(blk)
+        i2 = blk - pool.n_q4 - pool.n_q8
+        for name, got in (("k", kh), ("v", vh)):
+            raw = pool.codes2[name][i2].astype(np.uint32)          # [Hkv][256][32]
+            c = np.stack([(raw >> (2 * m)) & 3 for m in range(4)], axis=-1).reshape(raw.shape[:-1] + (128,))
+            par = pool.params2[name][i2].astype(np.float32)         # [Hkv][256][2][2]
+            s = np.repeat(par[..., 0], 64, axis=-1)
+            z = np.repeat(par[..., 1], 64, axis=-1)
+            want = (c.astype(np.float32) * s + z).astype(np.float32)
+            live = ~pool.masked(blk)
+            assert np.array_equal(got[:, live], want[:, live])
+
+
+def test_mixed_2_4_8_pool_attention_matches_brute_force():
+    d, hkv, hq, n = 128, 2, 8, 700
+    pool, _, _ = _pool3(23, d, hkv, n)
+    pool.invalidate_slots([3 * 256 + 9, 1 * 256 + 40])
+    rng = np.random.default_rng(24)
+    q = rng.standard_normal((1, hq, d)).astype(np.float16)
+    tables = np.array([[3, 1, 4]], np.int32)
+    out = O.decode_attention(pool, q, "fp16", tables, [n])
+    H = scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d)
+    kh = np.concatenate([pool.dequantize_block(b)[0] for b in (3, 1, 4)], axis=1)[:, :n].astype(np.float64)
+    vh = np.concatenate([pool.dequantize_block(b)[1] for b in (3, 1, 4)], axis=1)[:, :n].astype(np.float64)
+    masked = np.concatenate([pool.masked(b) for b in (3, 1, 4)])[:n]
+    for h in range(hq):
+        kv = h // (hq // hkv)
+        logits = (kh[kv] @ (H @ q[0, h].astype(np.float64))) / math.sqrt(d)
+        logits[masked] = O.SENTINEL_LOGIT
+        want = scipy.special.softmax(logits) @ vh[kv]
+        assert np.allclose(out[0, h], want, rtol=0, atol=1e-12)
+
+
+def test_2bit_round_trip_bound():
+    rng = np.random.default_rng(25)
+    x = (rng.standard_normal((300, 128)) * rng.choice([0.01, 1, 30], size=(300, 1))).astype(np.float32)
+    codes, s_h, z_h = O.quantize_groups(x, 2)
+    assert codes.max() <= 3
+    err, bound = _roundtrip_bound(x, codes, s_h, z_h, 2)
+    assert np.all(err <= bound)
+
+
+def test_2bit_block_image_size_and_restore():
+    """A 2-bit block's image: header 16 B + mask 32 B + 80 B per (token, KV
+    head) at D = 128 (two 32-byte code rows, two 8-byte param rows); loading
+    it into another pool's 2-bit block restores the block exactly."""
+    pool, _, _ = _pool3(26)
+    img = pool.block_image(3)
+    assert pool.block_class(3) == 2
+    assert img.size == 48 + 80 * 256 * pool.hkv
+    other = O.OraclePool(pool.hkv, pool.d, 2, 1, n_q2=2)
+    assert other.load_block_image(4, img)
+    assert np.array_equal(other.block_image(4)[16:], img[16:])
+    assert not other.load_block_image(0, img)            # a 4-bit block refuses a 2-bit image
