@@ -638,8 +638,12 @@ def measure_paging(job, dev, reps, decode_ms):
     s_dec, s_copy = torch.cuda.Stream(), torch.cuda.Stream()
 
     def beside(import_ids):
+        # The GPU first spins ~50 us in a gate kernel while the host enqueues
+        # the decode and the import on their streams, so both start together
+        # and neither span includes the host's own launch time.
         spans = []
         for _ in range(reps):
+            torch.cuda._sleep(100000)
             go = torch.cuda.Event()
             go.record()
             s_dec.wait_event(go)

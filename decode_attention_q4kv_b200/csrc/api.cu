@@ -300,6 +300,9 @@ q4kv_status q4kv_mixed_block_ids(const double* absmean, int32_t n_chunks, int32_
                                     as_stream(stream)));
 }
 
+// Longest work item the split model chooses, in 256-token blocks.
+constexpr int64_t kMaxItemBlocks = 64;
+
 q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
                                   int32_t head_dim, int32_t max_blocks_per_seq, int32_t n_splits,
                                   int32_t num_sms, q4kv_decode_plan* plan) {
@@ -333,10 +336,18 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
     // it) is 0.9 block-time, fitted to decode times measured with forced
     // split counts on the Gemma-, Llama- and Qwen-shaped layers and the
     // batch/context sweep.
+    //
+    // Items are capped at kMaxItemBlocks blocks.  A warp's value sums are
+    // accumulated by the tensor cores in fp32 over every tile of its item,
+    // and the code-times-scale part nearly cancels the zero part, so their
+    // rounding grows with the item's length: with one item per 131072-token
+    // sequence the attention output was off by 2.2e-2 relative (L2), with
+    // 32768 tokens per item by 2.7e-3.
     const int64_t pairs = static_cast<int64_t>(batch > 0 ? batch : 1) * n_kv_heads;
+    const int64_t smin = (nb + kMaxItemBlocks - 1) / kMaxItemBlocks;
     double best = 1e300;
-    s = 1;
-    for (int64_t cand = 1; cand <= nb; ++cand) {
+    s = smin;
+    for (int64_t cand = smin; cand <= nb; ++cand) {
       const int64_t bps = (nb + cand - 1) / cand;
       if ((nb + bps - 1) / bps != cand) continue;         // each distinct split only once
       const int64_t items = pairs * cand;
