@@ -427,7 +427,8 @@ def run_gpu(args):
 
     paging = measure_paging(job, dev, reps, d_cold_ms)
     card = measure_card(job, dev, reps) if not args.fp8 else None
-    q2mix = measure_q2mix(job, dev, reps) if not args.fp8 else None
+    # 2-bit blocks are read by plan kernel 1 only
+    q2mix = measure_q2mix(job, dev, reps) if not args.fp8 and args.decode_kernel == 1 else None
 
     e2e = run_e2e(job, args, dev, world) if not args.no_e2e else None
     if world > 1:

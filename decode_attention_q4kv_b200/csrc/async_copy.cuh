@@ -49,6 +49,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   }
   return false;
 }
+// One test of the phase, never suspending the thread.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for a warp that has nothing else to do (a producer or a
+// helper warp): test, then sleep ns0 doubling up to ns1 between tests, so its
+// polling takes few issue slots from the warps sharing its scheduler.  A
+// try_wait with a suspend hint polls far more often while it waits.  The
+// limit (4 kSpinLimit tests, at least ~2 s when ns1 >= 64) is only a bound.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, unsigned ns0, unsigned ns1) {
+  unsigned ns = ns0;
+  for (unsigned i = 0; i < 4 * kSpinLimit; ++i) {
+    if (mbar_test(bar, parity)) return true;
+    __nanosleep(ns);
+    ns = ns < ns1 ? 2 * ns : ns1;
+  }
+  return false;
+}
 // bytes and both addresses must be multiples of 16
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

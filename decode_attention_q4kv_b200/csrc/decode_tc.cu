@@ -539,22 +539,29 @@ __device__ __forceinline__ void pair_tiles(PairState<D>& st, const TileAt (&ta)[
     }
   }
   // ---- online softmax ----
-  float mx = -INFINITY;
+  // The column max (a shuffle reduction) is needed only when some logit
+  // exceeds the running max by more than kLazy; a warp vote finds out.
+  bool grow = false;
 #pragma unroll
-  for (int i = 0; i < NTL; ++i) mx = fmaxf(mx, fmaxf(logit[i][0], logit[i][1]));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-  if (mx > st.m + kLazy) {          // also taken on the first live tile (m = -inf)
-    const float alpha = ex2(st.m - mx);
-    st.m = mx;
-    st.l *= alpha;
-    st.z[0] *= alpha;
-    st.z[1] *= alpha;
+  for (int i = 0; i < NTL; ++i) grow |= fmaxf(logit[i][0], logit[i][1]) > st.m + kLazy;
+  if (__any_sync(0xffffffffu, grow)) {
+    float mx = -INFINITY;
 #pragma unroll
-    for (int mv = 0; mv < D / 16; ++mv)
+    for (int i = 0; i < NTL; ++i) mx = fmaxf(mx, fmaxf(logit[i][0], logit[i][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (mx > st.m + kLazy) {          // also taken on the first live tile (m = -inf)
+      const float alpha = ex2(st.m - mx);
+      st.m = mx;
+      st.l *= alpha;
+      st.z[0] *= alpha;
+      st.z[1] *= alpha;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st.o[mv][e] *= alpha;
+      for (int mv = 0; mv < D / 16; ++mv)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.o[mv][e] *= alpha;
+    }
   }
   uint32_t wb[NTL][2];
 #pragma unroll
@@ -768,25 +775,33 @@ __device__ __forceinline__ void head_tiles(HeadState<D>& st, const TileAt (&ta)[
       }
     }
   }
-  // ---- online softmax per head column ----
+  // ---- online softmax per head column (max reduction only when a warp vote
+  // finds a logit above the running max + kLazy) ----
+  bool grow = false;
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    float mx = -INFINITY;
+  for (int c = 0; c < 2; ++c)
 #pragma unroll
-    for (int i = 0; i < NTL; ++i) mx = fmaxf(mx, fmaxf(logit[i][0][c], logit[i][1][c]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    if (mx > st.m[c] + kLazy) {
-      const float alpha = ex2(st.m[c] - mx);
-      st.m[c] = mx;
-      st.l[c] *= alpha;
+    for (int i = 0; i < NTL; ++i) grow |= fmaxf(logit[i][0][c], logit[i][1][c]) > st.m[c] + kLazy;
+  if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-      for (int gr = 0; gr < NG; ++gr) st.z[c][gr] *= alpha;
+    for (int c = 0; c < 2; ++c) {
+      float mx = -INFINITY;
 #pragma unroll
-      for (int mv = 0; mv < D / 16; ++mv) {
-        st.o[mv][c] *= alpha;
-        st.o[mv][2 + c] *= alpha;
+      for (int i = 0; i < NTL; ++i) mx = fmaxf(mx, fmaxf(logit[i][0][c], logit[i][1][c]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      if (mx > st.m[c] + kLazy) {
+        const float alpha = ex2(st.m[c] - mx);
+        st.m[c] = mx;
+        st.l[c] *= alpha;
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr) st.z[c][gr] *= alpha;
+#pragma unroll
+        for (int mv = 0; mv < D / 16; ++mv) {
+          st.o[mv][c] *= alpha;
+          st.o[mv][2 + c] *= alpha;
+        }
       }
     }
   }
@@ -1329,10 +1344,22 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     if (lane != 0) return;
     uint32_t it = 0;
     bool gave_up = false;
+    // Global reads are issued ahead of the waits that follow them: the next
+    // item's sequence length one item ahead, and a stage's block-table entry
+    // before the wait for its free slot.  Read only after the slot frees,
+    // their latency (about a microsecond under load) would add to every
+    // stage's time in flight.
+    auto seq_of = [&](int item) {
+      int b, kvh, split;
+      item_coords(item, S, hkv, b, kvh, split);
+      return a.seq_lens[b];
+    };
+    int seq_next = blockIdx.x < n_items ? seq_of(blockIdx.x) : 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       int b, kvh, split;
       item_coords(item, S, hkv, b, kvh, split);
-      const int seq = a.seq_lens[b];
+      const int seq = seq_next;
+      if (item + static_cast<int>(gridDim.x) < n_items) seq_next = seq_of(item + gridDim.x);
       const bool bad_seq = seq < 0 || seq > mb * kBlockTokens;
       if (bad_seq && split == 0 && kvh == 0) raise_error(P.error_word, Q4KV_DEVERR_SEQ_LEN);
       const int t0 = split * tps;
@@ -1340,11 +1367,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       int tok = t0;
       do {
         const int s = it % kNS;
+        const int32_t blk_read = tok < t1 ? a.tables[static_cast<int64_t>(b) * mb + tok / kBlockTokens] : -1;
         // A stage that stays taken past the limit ends production: writing
         // the stage or arriving on its full barrier could then land in a
         // phase the consumers have not finished.  Their own bounded waits
         // run out in turn and they report the timeout.
-        if (!mbar_wait(&empty[s], ((it / kNS) & 1) ^ 1)) {
+        if (!mbar_wait_idle(&empty[s], ((it / kNS) & 1) ^ 1, 32, 128)) {
           gave_up = true;
           break;
         }
@@ -1359,7 +1387,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         int step = Geo<D, 4>::TS;
         if (tok < t1) {
           // a stage never crosses a block boundary, whatever the split length
-          const int32_t blk = a.tables[static_cast<int64_t>(b) * mb + tok / kBlockTokens];
+          const int32_t blk = blk_read;
           if (blk < 0 || blk >= P.n_blocks()) {
             raise_error(P.error_word, Q4KV_DEVERR_BLOCK_ID);
             meta.poison = 1;
@@ -1455,7 +1483,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     for (int item = i0; item < n_items; item += gridDim.x, ++k) {
       const int buf = k & 1;
       bool late = false;
-      if (!timed_out && !mbar_wait(&done[buf], (k >> 1) & 1)) {
+      if (!timed_out && !mbar_wait_idle(&done[buf], (k >> 1) & 1, 128, 1024)) {
         timed_out = late = true;
         if (lane == 0) raise_error(P.error_word, Q4KV_DEVERR_TIMEOUT);
       }
