@@ -26,6 +26,17 @@
 namespace q4kv {
 namespace {
 
+
+// Single-lane operations without a divergent branch: the instruction is
+// predicated on the lane.
+__device__ __forceinline__ void arrive_if(bool p, uint64_t* bar) {
+  asm volatile("{\n .reg .pred q;\n .reg .b64 st;\n setp.ne.u32 q, %1, 0;\n @q mbarrier.arrive.shared::cta.b64 st, [%0];\n}"
+               :: "r"(smem_u32(bar)), "r"(static_cast<uint32_t>(p)) : "memory");
+}
+__device__ __forceinline__ void red_and_if(bool p, uint32_t* addr, uint32_t v) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q red.global.and.b32 [%1], %2;\n}"
+               :: "r"(static_cast<uint32_t>(p)), "l"(addr), "r"(v) : "memory");
+}
 constexpr int kEPL = 16;  // channels held by one lane
 
 template <int D>
@@ -228,8 +239,9 @@ __device__ __forceinline__ void clamped_codes(const float2 (&x)[8], float xs, co
   const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    const int r0 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(__fmul_rn(x[p].x, xs), g.z), g.s)), 0), L);
-    const int r1 = min(max(__float2int_rn(__fdiv_rn(__fsub_rn(__fmul_rn(x[p].y, xs), g.z), g.s)), 0), L);
+    // s = 0 (a constant group) codes 0, as on the fast path
+    const int r0 = g.s == 0.0f ? 0 : min(max(__float2int_rn(__fdiv_rn(__fsub_rn(__fmul_rn(x[p].x, xs), g.z), g.s)), 0), L);
+    const int r1 = g.s == 0.0f ? 0 : min(max(__float2int_rn(__fdiv_rn(__fsub_rn(__fmul_rn(x[p].y, xs), g.z), g.s)), 0), L);
     const float2 k = make_float2(static_cast<float>(r0), static_cast<float>(r1));
     if (BITS == 4) {
       if (p % 2 == 0) c[p / 2] = __fadd2_rn(k, m2);
@@ -282,7 +294,9 @@ __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupPar
     w.w = __byte_perm(__byte_perm(q[12], q[13], 0x0040), __byte_perm(q[14], q[15], 0x0040), 0x5410);
     *reinterpret_cast<uint4*>(code_dst + j * 16) = w;
   }
-  if ((j & 3) == 0) param_dst[j >> 2] = __halves2half2(g.sh, g.zh);
+  // the four lanes of a group hold the same parameters and all store them:
+  // one branch fewer, and the stores merge in the same sector
+  param_dst[j >> 2] = __halves2half2(g.sh, g.zh);
 }
 
 // FP8 comparison cache: the lane's 16 values as OCP E4M3 bytes (round to
@@ -507,16 +521,17 @@ __global__ void __launch_bounds__(kQThreads, 1)
         }
         // freshly written slots are live: one word update for the item's tokens
         const uint32_t tf = t0 + ti;
-        if (h == 0 && lane == 0 && tf < geo.n_tokens) {
-          const int nv = static_cast<int>(umin(static_cast<uint32_t>(S::VPW), geo.n_tokens - tf));
+        if (h == 0) {
+          const bool doit = lane == 0 && tf < geo.n_tokens;
+          const int nv = doit ? static_cast<int>(umin(static_cast<uint32_t>(S::VPW), geo.n_tokens - tf)) : 0;
           const int sf = static_cast<int>(tf % kBlockTokens);
-          atomicAnd(pool.mask + static_cast<int64_t>(blk) * kMaskWords + sf / 32,
-                    ~(((1u << nv) - 1u) << (sf % 32)));
+          red_and_if(doit, pool.mask + static_cast<int64_t>(blk) * kMaskWords + sf / 32,
+                     ~(((1u << nv) - 1u) << (sf % 32)));
         }
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    arrive_if(lane == 0, &empty[s]);
     pos = nxt;
     blk = blk_next;
   }

@@ -198,6 +198,24 @@ def test_large_block_ids_and_many_tokens():
     assert_pool_equal(pool, ref, blocks=[0, 1, 31, 62, 63])
 
 
+def test_constant_group_beside_a_clamped_group():
+    # One warp item (4 tokens of one head at D = 128) whose groups take both
+    # encoder paths: token 1's values are beyond the fp16 range (zero = inf,
+    # the exact path), token 0 is a constant group whose value is not
+    # fp16-exact (s = 0 with x - z > 0; the oracle codes it 0, and so must
+    # either path).
+    rng = np.random.default_rng(12)
+    hkv, d = 1, 128
+    base = rng.standard_normal((256, hkv, d)).astype(np.float32)
+    base[0] = 1.1e-6                            # bf16 value above its fp16 rounding
+    base[1] = 70000.0 + rng.standard_normal((hkv, d)) * 1000.0
+    x = torch.from_numpy(base).to(torch.bfloat16)
+    assert float(x[0, 0, 0]) > float(x[0, 0, 0].to(torch.float16))
+    for rotated in (False, True):
+        pool, ref = _quantize_both(x, x, [0], 1, rotated=rotated)
+        assert_pool_equal(pool, ref)
+
+
 def test_near_tie_values_take_the_exact_path():
     # V is stored unrotated, so its quotients can be placed on and next to
     # half-integers exactly: z = -1, s = 1/16 (all fp16-exact), values
