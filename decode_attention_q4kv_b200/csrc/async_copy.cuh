@@ -20,6 +20,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(smem_u32(bar))
                : "memory");
 }
+// An arrival by the threads where p holds, as one predicated instruction
+// (no divergent branch around a single-lane arrival).
+__device__ __forceinline__ void arrive_if(bool p, uint64_t* bar) {
+  asm volatile("{\n .reg .pred q;\n .reg .b64 st;\n setp.ne.u32 q, %1, 0;\n @q mbarrier.arrive.shared::cta.b64 st, [%0];\n}"
+               :: "r"(smem_u32(bar)), "r"(static_cast<uint32_t>(p)) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}" ::"r"(
                    smem_u32(bar)),

@@ -29,10 +29,6 @@ namespace {
 
 // Single-lane operations without a divergent branch: the instruction is
 // predicated on the lane.
-__device__ __forceinline__ void arrive_if(bool p, uint64_t* bar) {
-  asm volatile("{\n .reg .pred q;\n .reg .b64 st;\n setp.ne.u32 q, %1, 0;\n @q mbarrier.arrive.shared::cta.b64 st, [%0];\n}"
-               :: "r"(smem_u32(bar)), "r"(static_cast<uint32_t>(p)) : "memory");
-}
 __device__ __forceinline__ void red_and_if(bool p, uint32_t* addr, uint32_t v) {
   asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q red.global.and.b32 [%1], %2;\n}"
                :: "r"(static_cast<uint32_t>(p)), "l"(addr), "r"(v) : "memory");
