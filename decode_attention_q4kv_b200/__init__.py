@@ -376,5 +376,50 @@ def decode_attention(pool: Q4KVPool, q: torch.Tensor, block_tables: torch.Tensor
     return out
 
 
-__all__ = ["Q4KVPool", "Q4KVError", "DecodePlan", "decode_attention", "block_absmean",
+def append_decode(pool: Q4KVPool, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                  block_tables: torch.Tensor, seq_lens: torch.Tensor, n_new: Optional[torch.Tensor] = None,
+                  softmax_scale: float = 0.0, out_dtype=torch.float16, plan: Optional[DecodePlan] = None,
+                  workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One generation step: append k_new/v_new [B][T][Hkv][D] at each
+    sequence's position seq_lens[b] (lengths before the append, not
+    modified), then decode q [B][Hq][D] over seq_lens[b] + n_new[b] tokens
+    (+ T when n_new is None).  Same result as pool.append then
+    decode_attention with the grown lengths; the decode overlaps the append."""
+    dev = _require_cuda(k_new, v_new, q, block_tables, seq_lens)
+    if k_new.dtype != v_new.dtype or k_new.dtype not in _IN_DTYPES:
+        raise ValueError("k_new and v_new must share dtype float16 or bfloat16")
+    if k_new.shape != v_new.shape or k_new.dim() != 4 or k_new.stride() != v_new.stride():
+        raise ValueError("k_new and v_new must be [B][T][Hkv][D] with equal strides")
+    if k_new.stride(3) != 1 or k_new.stride(2) != k_new.shape[3]:
+        raise ValueError("each token's [Hkv][D] row must be contiguous")
+    if q.dtype not in _IN_DTYPES or q.dim() != 3 or not q.is_contiguous():
+        raise ValueError("q must be contiguous fp16/bf16 [B][Hq][D]")
+    B, hq, d = q.shape
+    tables = block_tables.to(torch.int32).contiguous()
+    lens = seq_lens.to(torch.int32).contiguous()
+    if k_new.shape[0] != B or tables.dim() != 2 or tables.shape[0] != B or lens.shape != (B,):
+        raise ValueError("k_new, q, block_tables and seq_lens must share the batch")
+    nn = None
+    if n_new is not None:
+        if n_new.shape != (B,):
+            raise ValueError("n_new must be [B]")
+        _require_cuda(n_new)
+        nn = n_new.to(torch.int32).contiguous()
+    if plan is None:
+        plan = DecodePlan(B, hq, pool.n_kv_heads, d, tables.shape[1])
+    if workspace is None:
+        workspace = plan.workspace(dev)
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=out_dtype, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib().q4kv_append_decode(ctypes.byref(pool.desc), ctypes.byref(plan.c), _ptr(k_new), _ptr(v_new),
+                                   _IN_DTYPES[k_new.dtype], k_new.shape[1],
+                                   _ptr(nn) if nn is not None else None, k_new.stride(0), k_new.stride(1),
+                                   _ptr(q), _IN_DTYPES[q.dtype], _ptr(tables), _ptr(lens), float(softmax_scale),
+                                   _ptr(out), _OUT_DTYPES[out.dtype], _ptr(workspace), ws_bytes, _stream(dev)),
+          "q4kv_append_decode")
+    return out
+
+
+__all__ = ["Q4KVPool", "Q4KVError", "DecodePlan", "decode_attention", "append_decode", "block_absmean",
            "mixed_block_ids", "card_max_bytes", "card_encode", "card_decode", "BLOCK_TOKENS", "GROUP"]

@@ -73,6 +73,9 @@ _SIGNATURES = {
     "q4kv_decode_attention": (c_int32, [P(PoolDesc), P(DecodePlan), c_void_p, c_int32, c_void_p,
                                         c_void_p, c_float, c_void_p, c_int32, c_void_p, c_size_t,
                                         c_void_p]),
+    "q4kv_append_decode": (c_int32, [P(PoolDesc), P(DecodePlan), c_void_p, c_void_p, c_int32, c_int32,
+                                     c_void_p, c_int64, c_int64, c_void_p, c_int32, c_void_p, c_void_p,
+                                     c_float, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
     "q4kv_read_device_error": (c_int32, [P(PoolDesc), P(ctypes.c_uint32), c_int32, c_void_p]),
     "q4kv_decode_attention_static_scratch": (c_int32, [P(PoolDesc), P(DecodePlan), c_void_p, c_int32,
                                                        c_void_p, c_void_p, c_float, c_void_p,

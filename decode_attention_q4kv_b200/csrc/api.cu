@@ -123,24 +123,36 @@ q4kv_status q4kv_quantize_blocks(const q4kv_pool* pool, const void* k, const voi
                                    block_ids, as_stream(stream)));
 }
 
+// Arguments of an append; *rows = 0 when it writes nothing.
+static q4kv_status check_append(const q4kv_pool* pool, const void* k, const void* v, int32_t in_dtype,
+                                int32_t batch, int32_t max_new, const int32_t* n_new, int64_t seq_stride,
+                                int64_t token_stride, const int32_t* tables, int32_t max_blocks,
+                                const int32_t* seq_lens, int64_t* rows) {
+  q4kv_status st = check_pool(pool);
+  if (st != Q4KV_OK) return st;
+  if (batch < 0 || max_new < 0 || seq_stride < 0) return Q4KV_ERR_INVALID_ARG;
+  *rows = batch > 0 && max_new > 0 ? 1 : 0;
+  st = check_input(k, in_dtype, *rows, token_stride, pool->n_kv_heads, pool->head_dim);
+  if (st != Q4KV_OK) return st;
+  st = check_input(v, in_dtype, *rows, token_stride, pool->n_kv_heads, pool->head_dim);
+  if (st != Q4KV_OK) return st;
+  if ((seq_stride * 2) % 16 != 0) return Q4KV_ERR_INVALID_ARG;
+  if (*rows == 0) return Q4KV_OK;
+  if (tables == nullptr || !aligned(tables, 4) || max_blocks < 1 || seq_lens == nullptr ||
+      !aligned(seq_lens, 4) || (n_new != nullptr && !aligned(n_new, 4)))
+    return Q4KV_ERR_INVALID_ARG;
+  return Q4KV_OK;
+}
+
 q4kv_status q4kv_append_tokens(const q4kv_pool* pool, const void* k, const void* v,
                                int32_t in_dtype, int32_t batch, int32_t max_new,
                                const int32_t* n_new, int64_t seq_stride, int64_t token_stride,
                                const int32_t* tables, int32_t max_blocks, const int32_t* seq_lens,
                                void* stream) {
-  q4kv_status st = check_pool(pool);
-  if (st != Q4KV_OK) return st;
-  if (batch < 0 || max_new < 0 || seq_stride < 0) return Q4KV_ERR_INVALID_ARG;
-  const int64_t rows = batch > 0 && max_new > 0 ? 1 : 0;
-  st = check_input(k, in_dtype, rows, token_stride, pool->n_kv_heads, pool->head_dim);
-  if (st != Q4KV_OK) return st;
-  st = check_input(v, in_dtype, rows, token_stride, pool->n_kv_heads, pool->head_dim);
-  if (st != Q4KV_OK) return st;
-  if ((seq_stride * 2) % 16 != 0) return Q4KV_ERR_INVALID_ARG;
-  if (rows == 0) return Q4KV_OK;
-  if (tables == nullptr || !aligned(tables, 4) || max_blocks < 1 || seq_lens == nullptr ||
-      !aligned(seq_lens, 4) || (n_new != nullptr && !aligned(n_new, 4)))
-    return Q4KV_ERR_INVALID_ARG;
+  int64_t rows = 0;
+  const q4kv_status st = check_append(pool, k, v, in_dtype, batch, max_new, n_new, seq_stride, token_stride,
+                                      tables, max_blocks, seq_lens, &rows);
+  if (st != Q4KV_OK || rows == 0) return st;
   return from_cuda(launch_append(view_of(*pool), k, v, in_dtype, batch, max_new, n_new, seq_stride,
                                  token_stride, tables, max_blocks, seq_lens, as_stream(stream)));
 }
@@ -381,11 +393,12 @@ q4kv_status q4kv_decode_plan_make(int32_t batch, int32_t n_q_heads, int32_t n_kv
   return Q4KV_OK;
 }
 
-q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan* plan,
-                                  const void* q, int32_t q_dtype, const int32_t* block_tables,
-                                  const int32_t* seq_lens, float softmax_scale, void* out,
-                                  int32_t out_dtype, void* workspace, size_t workspace_bytes,
-                                  void* stream) {
+// Arguments of a decode, filled into *a; *empty = 1 when there is nothing to do.
+static q4kv_status prepare_decode(const q4kv_pool* pool, const q4kv_decode_plan* plan, const void* q,
+                                  int32_t q_dtype, const int32_t* block_tables, const int32_t* seq_lens,
+                                  float softmax_scale, void* out, int32_t out_dtype, void* workspace,
+                                  size_t workspace_bytes, DecodeArgs* a, int* empty) {
+  *empty = 1;
   q4kv_status st = check_pool(pool);
   if (st != Q4KV_OK) return st;
   if (plan == nullptr) return Q4KV_ERR_INVALID_ARG;
@@ -403,6 +416,7 @@ q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan*
       !isfinite(softmax_scale))
     return Q4KV_ERR_INVALID_ARG;
   if (plan->batch == 0) return Q4KV_OK;
+  *empty = 0;
   if (q == nullptr || block_tables == nullptr || seq_lens == nullptr || out == nullptr ||
       !aligned(q, 16) || !aligned(block_tables, 16) || !aligned(seq_lens, 4) || !aligned(out, 16))
     return Q4KV_ERR_INVALID_ARG;
@@ -419,23 +433,67 @@ q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan*
   if (plan->workspace_bytes > 0 &&
       (workspace == nullptr || workspace_bytes < plan->workspace_bytes || !aligned(workspace, 256)))
     return Q4KV_ERR_WORKSPACE;
-  DecodeArgs a;
-  a.pool = view_of(*pool);
-  a.plan = *plan;
-  a.q = q;
-  a.q_dtype = q_dtype;
-  a.tables = block_tables;
-  a.seq_lens = seq_lens;
-  a.scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(plan->head_dim));
-  a.out = out;
-  a.out_dtype = out_dtype;
+  a->pool = view_of(*pool);
+  a->plan = *plan;
+  a->q = q;
+  a->q_dtype = q_dtype;
+  a->tables = block_tables;
+  a->seq_lens = seq_lens;
+  a->add_lens = nullptr;
+  a->add_const = 0;
+  a->defer_wait = 0;
+  a->scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(plan->head_dim));
+  a->out = out;
+  a->out_dtype = out_dtype;
   const size_t rows = static_cast<size_t>(plan->batch) * plan->n_q_heads * plan->n_splits;
-  a.ws_o = static_cast<float*>(workspace);
-  a.ws_ml = plan->workspace_bytes > 0
-                ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                           round_up(rows * plan->head_dim * sizeof(float), 256))
-                : nullptr;
+  a->ws_o = static_cast<float*>(workspace);
+  a->ws_ml = plan->workspace_bytes > 0
+                 ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                            round_up(rows * plan->head_dim * sizeof(float), 256))
+                 : nullptr;
+  return Q4KV_OK;
+}
+
+q4kv_status q4kv_decode_attention(const q4kv_pool* pool, const q4kv_decode_plan* plan,
+                                  const void* q, int32_t q_dtype, const int32_t* block_tables,
+                                  const int32_t* seq_lens, float softmax_scale, void* out,
+                                  int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  DecodeArgs a;
+  int empty = 1;
+  const q4kv_status st = prepare_decode(pool, plan, q, q_dtype, block_tables, seq_lens, softmax_scale, out,
+                                        out_dtype, workspace, workspace_bytes, &a, &empty);
+  if (st != Q4KV_OK || empty) return st;
   return from_cuda(launch_decode(a, as_stream(stream)));
+}
+
+q4kv_status q4kv_append_decode(const q4kv_pool* pool, const q4kv_decode_plan* plan, const void* k_new,
+                               const void* v_new, int32_t in_dtype, int32_t max_new, const int32_t* n_new,
+                               int64_t seq_stride, int64_t token_stride, const void* q, int32_t q_dtype,
+                               const int32_t* block_tables, const int32_t* seq_lens, float softmax_scale,
+                               void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (plan == nullptr) return Q4KV_ERR_INVALID_ARG;
+  int64_t rows = 0;
+  q4kv_status st = check_append(pool, k_new, v_new, in_dtype, plan->batch, max_new, n_new, seq_stride,
+                                token_stride, block_tables, plan->max_blocks_per_seq, seq_lens, &rows);
+  if (st != Q4KV_OK) return st;
+  DecodeArgs a;
+  int empty = 1;
+  st = prepare_decode(pool, plan, q, q_dtype, block_tables, seq_lens, softmax_scale, out, out_dtype,
+                      workspace, workspace_bytes, &a, &empty);
+  if (st != Q4KV_OK || empty) return st;
+  cudaStream_t s = as_stream(stream);
+  if (rows > 0) {
+    const cudaError_t e = launch_append(view_of(*pool), k_new, v_new, in_dtype, plan->batch, max_new, n_new,
+                                        seq_stride, token_stride, block_tables, plan->max_blocks_per_seq,
+                                        seq_lens, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    a.add_lens = n_new;
+    a.add_const = max_new;
+    a.defer_wait = 1;
+  }
+  return from_cuda(launch_decode(a, s));
 }
 
 q4kv_status q4kv_read_device_error(const q4kv_pool* pool, uint32_t* bits, int32_t clear,

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kThreads) decode_simple_kernel(const DecodeArg
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int hq = a.plan.n_q_heads, g = hq / P.n_kv_heads;
   const int S = a.plan.n_splits, tps = a.plan.tokens_per_split, mb = a.plan.max_blocks_per_seq;
-  const int seq = a.seq_lens[b];
+  const int seq = seq_len_of(a, b);
   const bool bad_seq = seq < 0 || seq > mb * kBlockTokens;
   if (bad_seq && split == 0 && kvh == 0 && tid == 0) raise_error(P.error_word, Q4KV_DEVERR_SEQ_LEN);
 

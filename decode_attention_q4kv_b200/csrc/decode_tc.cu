@@ -992,7 +992,11 @@ __device__ __forceinline__ void fp8_tile(Fp8State<D>& st, const TileAt& ta, cons
 // ---------------------------------------------------------------------------
 // aux warp: query preparation and the per-item merge
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void item_coords(int item, int S, int hkv, int& b, int& kvh, int& split) {
+// Work item -> (sequence, KV head, split), splits varying fastest.  (After
+// an append, moving the last splits' items, which hold the blocks it
+// writes, to the end of the order was measured slower than this order.)
+__device__ __forceinline__ void item_coords(const DecodeArgs& a, int item, int& b, int& kvh, int& split) {
+  const int S = a.plan.n_splits, hkv = a.plan.n_kv_heads;
   split = item % S;
   kvh = (item / S) % hkv;
   b = item / (S * hkv);
@@ -1168,7 +1172,7 @@ __device__ void prep_q4(const DecodeArgs& a, int item, uint8_t* tab, int* qint, 
                         int lane) {
   const int hkv = a.pool.n_kv_heads, G = a.plan.n_q_heads / hkv;
   int b, kvh, split;
-  item_coords(item, a.plan.n_splits, hkv, b, kvh, split);
+  item_coords(a, item, b, kvh, split);
   for (int h = 0; h < G; ++h) prep_head<D>(a, b, kvh, h, qint, gsum, escale, lane);
   __syncwarp();
 #pragma unroll 1
@@ -1211,7 +1215,7 @@ template <int D>
 __device__ void prep_fp8(const DecodeArgs& a, int item, uint8_t* tab, int lane) {
   const int hkv = a.pool.n_kv_heads, G = a.plan.n_q_heads / hkv;
   int b, kvh, split;
-  item_coords(item, a.plan.n_splits, hkv, b, kvh, split);
+  item_coords(a, item, b, kvh, split);
   for (int h = 0; h < G; ++h) prep_fp8_head<D>(a, b, kvh, h, tab, lane);
 }
 
@@ -1223,7 +1227,7 @@ __device__ void merge_item(const DecodeArgs& a, int item, const float* mrg_o, co
   using C = Cfg<D>;
   const int hkv = a.pool.n_kv_heads, hq = a.plan.n_q_heads, G = hq / hkv, S = a.plan.n_splits;
   int b, kvh, split;
-  item_coords(item, S, hkv, b, kvh, split);
+  item_coords(a, item, b, kvh, split);
   int flag = 0;
 #pragma unroll
   for (int w = 0; w < C::CW; ++w) flag |= mrg_flag[w];
@@ -1312,7 +1316,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   float* aux_f = reinterpret_cast<float*>(smem + C::kOffAuxW);
   float* aux_den = aux_f + CW * 8;
 
-  griddep_wait();   // earlier kernels in the stream (the encoder) have finished
+  // Earlier kernels in the stream (the encoder) have finished -- unless the
+  // one before is an append, whose blocks only the producer waits for.
+  if (!a.defer_wait) griddep_wait();
   griddep_launch_dependents();
   const PoolView& P = a.pool;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1349,16 +1355,20 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     // before the wait for its free slot.  Read only after the slot frees,
     // their latency (about a microsecond under load) would add to every
     // stage's time in flight.
+    // (x = the length before an append, y = the length decoded)
     auto seq_of = [&](int item) {
       int b, kvh, split;
-      item_coords(item, S, hkv, b, kvh, split);
-      return a.seq_lens[b];
+      item_coords(a, item, b, kvh, split);
+      return make_int2(a.seq_lens[b], seq_len_of(a, b));
     };
-    int seq_next = blockIdx.x < n_items ? seq_of(blockIdx.x) : 0;
+    // An append just before: its writes land in blocks at or past the old
+    // length, which are read only after waiting for the append grid.
+    bool waited = !a.defer_wait;
+    int2 seq_next = blockIdx.x < n_items ? seq_of(blockIdx.x) : make_int2(0, 0);
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       int b, kvh, split;
-      item_coords(item, S, hkv, b, kvh, split);
-      const int seq = seq_next;
+      item_coords(a, item, b, kvh, split);
+      const int seq = seq_next.y, fresh_blk = seq_next.x / kBlockTokens;
       if (item + static_cast<int>(gridDim.x) < n_items) seq_next = seq_of(item + gridDim.x);
       const bool bad_seq = seq < 0 || seq > mb * kBlockTokens;
       if (bad_seq && split == 0 && kvh == 0) raise_error(P.error_word, Q4KV_DEVERR_SEQ_LEN);
@@ -1403,6 +1413,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         meta.last = (tok + step >= t1) ? 1 : 0;
         *reinterpret_cast<StageMeta*>(stg + kOffMeta) = meta;
         if (meta.blk >= 0) {
+          if (!waited && tok / kBlockTokens >= fresh_blk) {
+            griddep_wait();
+            waited = true;
+          }
           const int rows = (meta.ntok + 15) & ~15;   // whole 16-token tiles, inside the block
           const int bits = meta.bits;
           const int64_t phys = bits == 4 ? meta.blk : (bits == 8 ? meta.blk - P.n_q4 : meta.blk - P.n_q4 - P.n_q8);
@@ -1438,6 +1452,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     // last stages issued to complete
     for (uint32_t k = (it > kNS ? it - kNS : 0); k < it; ++k)
       if (!mbar_wait(&full[k % kNS], (k / kNS) & 1)) break;
+    if (!waited) griddep_wait();   // this grid never completes before the append
     return;
   }
 
@@ -1449,7 +1464,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     constexpr int NT = (CW + 1) * 32;
     const int wid = warp < CW ? warp : CW;
     int b0, kvh0, split0;
-    item_coords(blockIdx.x, S, hkv, b0, kvh0, split0);
+    item_coords(a, blockIdx.x, b0, kvh0, split0);
     for (int h = wid; h < G; h += CW + 1) {
       if (FP8) prep_fp8_head<D>(a, b0, kvh0, h, qtab0, lane);
       else prep_head<D>(a, b0, kvh0, h, qint, gsum, escale, lane);

@@ -164,12 +164,23 @@ struct DecodeArgs {
   int q_dtype;
   const int32_t* tables;
   const int32_t* seq_lens;
+  // Sequence b is seq_lens[b] + (add_lens ? add_lens[b] : add_const) tokens
+  // long (an append just before the decode adds the second term).
+  const int32_t* add_lens;
+  int add_const;
+  // 1: the kernel before this one in the stream is an append whose writes
+  // all land at positions >= seq_lens[b]; the tensor-core kernel then waits
+  // for it only before it reads those blocks (programmatic dependent launch).
+  int defer_wait;
   float scale;
   void* out;
   int out_dtype;
   float* ws_o;   // [B][Hq][S][D]
   float* ws_ml;  // [B][Hq][S][2] (running max, running sum)
 };
+__device__ __forceinline__ int seq_len_of(const DecodeArgs& a, int b) {
+  return a.seq_lens[b] + (a.add_lens != nullptr ? a.add_lens[b] : a.add_const);
+}
 // plan.kernel selects the decode kernel: 1 = tensor-core pipeline
 // (decode_tc.cu), 0 = CUDA-core kernel (decode.cu); both share the merge.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);

@@ -317,6 +317,35 @@ q4kv_status q4kv_decode_attention(const q4kv_pool *pool, const q4kv_decode_plan 
                                   void *stream);
 
 /*
+ * One generation step: append each sequence's new tokens, then decode over
+ * the grown cache ([AMBP] sec. 2.1 item 4: EXTEND grows the cache in place,
+ * then attention reads it).  Equal to q4kv_append_tokens followed by
+ * q4kv_decode_attention with lengths seq_lens[b] + n_new[b], but faster: the
+ * decode starts while the append runs (programmatic dependent launch) and
+ * waits for it only before it streams a block at or past position
+ * seq_lens[b], the only blocks an append writes.
+ *   plan         as for q4kv_decode_attention; plan->batch sequences and
+ *                plan->max_blocks_per_seq block-table columns for both steps
+ *   k_new, v_new, in_dtype, max_new, n_new, seq_stride, token_stride
+ *                the new tokens, as for q4kv_append_tokens (batch =
+ *                plan->batch); max_new == 0 decodes without appending
+ *   q, q_dtype, block_tables, softmax_scale, out, out_dtype, workspace,
+ *   workspace_bytes  as for q4kv_decode_attention
+ *   seq_lens     device int32 [batch], the lengths BEFORE the append (not
+ *                modified); sequence b is decoded over seq_lens[b] +
+ *                n_new[b] tokens (+ max_new when n_new is NULL)
+ * Errors as for the two calls; nothing is launched unless both sets of
+ * arguments are valid.  Device-side errors (Q4KV_DEVERR_*) of either step go
+ * to the pool's error word.
+ */
+q4kv_status q4kv_append_decode(const q4kv_pool *pool, const q4kv_decode_plan *plan, const void *k_new,
+                               const void *v_new, int32_t in_dtype, int32_t max_new, const int32_t *n_new,
+                               int64_t seq_stride, int64_t token_stride, const void *q, int32_t q_dtype,
+                               const int32_t *block_tables, const int32_t *seq_lens, float softmax_scale,
+                               void *out, int32_t out_dtype, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/*
  * Decode attention for callers that cannot allocate device memory.
  * (The source pages have no counterpart: this is an interface convenience.)
  *

@@ -24,7 +24,7 @@ def _pool(**kw):
 
 def test_exports_every_declared_function():
     names = _lib.header_functions()
-    assert len(names) == 22
+    assert len(names) == 23
     for n in names:
         assert hasattr(L, n), n
     # the binding declares a signature for each of them
@@ -185,6 +185,38 @@ def test_decode_rejects_bad_arguments_without_launching():
     st, empty = _plan(0, 32, 8, 128, 4, 0, 148)
     assert st == 0
     assert call(pl=empty, ws=0, wsb=0) == 0                              # batch 0: nothing to do
+
+
+def test_append_decode_rejects_bad_arguments_without_launching():
+    """The fused generation step validates both the append and the decode
+    arguments before it launches anything (a fake pointer would fault)."""
+    p = _pool()
+    st, plan = _plan(2, 32, 8, 128, 4, 4, 148)
+    assert st == 0
+    f = L.q4kv_append_decode
+
+    def call(pool=p, pl=plan, k=FAKE, dt=0, t=3, nn=None, ss=3 * 1024, ts=1024, q=FAKE, qd=0, tab=FAKE,
+             lens=FAKE, scale=0.0, out=FAKE, od=1, ws=FAKE, wsb=None):
+        wsb = (pl.workspace_bytes if pl is not None else 0) if wsb is None else wsb
+        return f(ctypes.byref(pool), None if pl is None else ctypes.byref(pl), k, k, dt, t, nn, ss, ts, q, qd,
+                 tab, lens, scale, out, od, ws, wsb, None)
+
+    assert call(pl=None) == _lib.ERR_INVALID_ARG
+    assert call(dt=2) == _lib.ERR_INVALID_ARG                  # append: fp32 input
+    assert call(k=FAKE + 8) == _lib.ERR_INVALID_ARG            # append: misaligned rows
+    assert call(ts=1020) == _lib.ERR_INVALID_ARG               # append: token stride below Hkv*D
+    assert call(t=-1) == _lib.ERR_INVALID_ARG
+    assert call(nn=FAKE + 2) == _lib.ERR_INVALID_ARG
+    assert call(lens=None) == _lib.ERR_INVALID_ARG
+    assert call(qd=2) == _lib.ERR_INVALID_ARG                  # decode: bad query dtype
+    assert call(out=FAKE + 4) == _lib.ERR_INVALID_ARG          # decode: misaligned output
+    assert call(ws=0) == _lib.ERR_WORKSPACE                    # decode: missing workspace
+    assert call(pool=_pool(n_kv_heads=4)) == _lib.ERR_INVALID_ARG
+    bad = _lib.DecodePlan.from_buffer_copy(plan)
+    bad.kernel = 3
+    assert call(pl=bad) == _lib.ERR_INVALID_ARG
+    st, empty = _plan(0, 32, 8, 128, 4, 0, 148)
+    assert st == 0 and call(pl=empty, ws=0, wsb=0) == 0        # batch 0: nothing to do
 
 
 def test_selftest_rejects_bad_arguments():

@@ -115,3 +115,89 @@ def test_generation_step_append_then_decode():
     qh, dt = host(q)
     want = O.decode_attention(ref, qh, dt, tables, grown)
     assert_close(out, want, what="append + decode")
+
+
+def _prefilled(d, hkv, dtype, rotated, n_q4, n_q8, lens, tables, seed):
+    """Two GPU pools and an oracle pool holding each sequence's first lens[b] tokens."""
+    dev = cuda()
+    name = "fp16" if dtype == torch.float16 else "bf16"
+    pools = [q4.Q4KVPool(hkv, d, n_q4, n_q8, k_rotated=rotated, device=dev) for _ in range(2)]
+    ref = O.OraclePool(hkv, d, n_q4, n_q8, k_rotated=rotated)
+    for b, n in enumerate(lens):
+        if n == 0:
+            continue
+        k, v = W.random_small(n, hkv, d, name, seed=seed + 10 * b)
+        ids = tables[b][: -(-n // 256)].tolist()
+        for p in pools:
+            p.quantize(k.to(dev), v.to(dev), torch.tensor(ids, dtype=torch.int32, device=dev))
+        kh, dt = host(k)
+        vh, _ = host(v)
+        ref.quantize_blocks(kh, vh, dt, ids)
+    return pools, ref
+
+
+# (D, Hq, Hkv, input dtype, rotated K, 8-bit blocks): both column layouts, both
+# head sizes, 4-bit-only and mixed pools
+@pytest.mark.parametrize("d,hq,hkv,dtype,rotated,n_q8", [(128, 40, 8, torch.float16, True, 0),
+                                                         (128, 32, 8, torch.bfloat16, False, 6),
+                                                         (256, 16, 8, torch.bfloat16, True, 0),
+                                                         (256, 8, 4, torch.float16, True, 6)])
+@pytest.mark.parametrize("n_splits", [0, 1, 3])
+def test_append_decode_matches_separate_calls_and_oracle(d, hq, hkv, dtype, rotated, n_q8, n_splits):
+    """The fused generation step (the decode overlapping the append, waiting
+    for it only before the blocks it writes) gives exactly the output of an
+    append followed by a decode over the grown lengths, and the oracle's."""
+    dev = cuda()
+    lens = [0, 100, 255, 256, 700, 1023]        # empty, mid-block, a block boundary crossed, full blocks
+    new = [3, 1, 3, 0, 2, 1]
+    B, max_new, mb = len(lens), 3, 5
+    g = torch.Generator().manual_seed(d + hq + n_splits)
+    tables = torch.randperm(B * mb, generator=g).to(torch.int32).view(B, mb).numpy()
+    (fused, sep), ref = _prefilled(d, hkv, dtype, rotated, B * mb - n_q8, n_q8, lens, tables, seed=d + n_q8)
+    name = "fp16" if dtype == torch.float16 else "bf16"
+    kn, vn = W.random_small(B * max_new, hkv, d, name, seed=77)
+    kn, vn = kn.view(B, max_new, hkv, d), vn.view(B, max_new, hkv, d)
+    q = torch.randn(B, hq, d, generator=g).to(dtype)
+    tab = torch.as_tensor(tables).to(dev)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device=dev)
+    nn = torch.tensor(new, dtype=torch.int32, device=dev)
+    grown = [n + a for n, a in zip(lens, new)]
+    plan = q4.DecodePlan(B, hq, hkv, d, mb, n_splits=n_splits)
+    out = q4.append_decode(fused, kn.to(dev), vn.to(dev), q.to(dev), tab, lens_d, nn, out_dtype=torch.float32,
+                           plan=plan)
+    sep.append(kn.to(dev), vn.to(dev), tab, lens_d, nn)
+    want_gpu = q4.decode_attention(sep, q.to(dev), tab, torch.tensor(grown, dtype=torch.int32, device=dev),
+                                   out_dtype=torch.float32, plan=plan)
+    torch.cuda.synchronize()
+    assert fused.read_device_error() == 0
+    assert torch.equal(out, want_gpu)
+    kh, dt = host(kn.reshape(B * max_new, hkv, d))
+    vh, _ = host(vn.reshape(B * max_new, hkv, d))
+    ref.append_tokens(kh.reshape(B, max_new, hkv, d), vh.reshape(B, max_new, hkv, d), dt, tables, lens, new)
+    assert_pool_equal(fused, ref)
+    qh, qdt = host(q)
+    assert_close(out, O.decode_attention(ref, qh, qdt, tables, grown), what=f"append + decode {d}/{hq}/{hkv}")
+
+
+def test_append_decode_all_new_tokens_and_no_new_tokens():
+    """n_new omitted: every sequence appends max_new; max_new = 0: a plain decode."""
+    dev = cuda()
+    d, hq, hkv = 128, 32, 8
+    lens = [300, 511]
+    B, mb = len(lens), 3
+    tables = np.array([[4, 0, 2], [1, 5, 3]], dtype=np.int32)
+    (fused, sep), ref = _prefilled(d, hkv, torch.float16, True, 6, 0, lens, tables, seed=9)
+    kn, vn = W.random_small(B * 2, hkv, d, "fp16", seed=8)
+    kn, vn = kn.view(B, 2, hkv, d).to(dev), vn.view(B, 2, hkv, d).to(dev)
+    q = torch.randn(B, hq, d, generator=torch.Generator().manual_seed(2)).to(torch.float16).to(dev)
+    tab = torch.as_tensor(tables).to(dev)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device=dev)
+    none = q4.append_decode(fused, kn[:, :0], vn[:, :0], q, tab, lens_d, out_dtype=torch.float32)
+    plain = q4.decode_attention(sep, q, tab, lens_d, out_dtype=torch.float32)
+    assert torch.equal(none, plain)
+    out = q4.append_decode(fused, kn, vn, q, tab, lens_d, out_dtype=torch.float32)
+    sep.append(kn, vn, tab, lens_d)
+    want = q4.decode_attention(sep, q, tab, lens_d + 2, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert fused.read_device_error() == 0
+    assert torch.equal(out, want)
