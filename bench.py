@@ -656,10 +656,11 @@ def measure_paging(job, dev, reps, decode_ms):
     d2h_ms = timed(lambda: flat.copy_(dev_buf, non_blocking=True))
     s_dec, s_copy = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def beside(import_ids):
+    def beside(import_ids, move=None):
         # The GPU first spins ~50 us in a gate kernel while the host enqueues
         # the decode and the import on their streams, so both start together
-        # and neither span includes the host's own launch time.
+        # and neither span includes the host's own launch time.  move: another
+        # transfer in place of the import (a plain pinned copy, as reference).
         spans = []
         for _ in range(reps):
             torch.cuda._sleep(100000)
@@ -674,7 +675,10 @@ def measure_paging(job, dev, reps, decode_ms):
             e[1].record(s_dec)
             e[2].record(s_copy)
             with torch.cuda.stream(s_copy):
-                other.import_blocks(images, import_ids)
+                if move is None:
+                    other.import_blocks(images, import_ids)
+                else:
+                    move()
             e[3].record(s_copy)
             spans.append(e)
         torch.cuda.synchronize()
@@ -685,7 +689,8 @@ def measure_paging(job, dev, reps, decode_ms):
     out = {"blocks": nb, "bytes": moved, "image_stride": stride,
            "copy_engine_h2d_gbps": round(flat.numel() / (h2d_ms * 1e-3) / 1e9, 2),
            "copy_engine_d2h_gbps": round(flat.numel() / (d2h_ms * 1e-3) / 1e9, 2),
-           "decode_us_alone": round(decode_ms * 1e3, 2)}
+           "decode_us_alone": round(decode_ms * 1e3, 2),
+           "decode_us_beside_plain_h2d": beside(None, lambda: dev_buf.copy_(flat, non_blocking=True))[0]}
     for tag, the_ids in (("kernel", ids), ("copy_engine", host_ids)):
         exp_ms = timed(lambda: pool.export_blocks(the_ids, images))
         imp_ms = timed(lambda: other.import_blocks(images, the_ids))
