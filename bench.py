@@ -209,7 +209,7 @@ class Job:
                 e = min(s + n_src, t.shape[0])
                 t[s:e].copy_(t[: e - s])
 
-    def quantize_layer(self, L):
+    def quantize_layer(self, L, mark=None):
         w, q4 = self.w, self.q4
         if w.q8_fraction and not self.fp8:
             am = q4.block_absmean(L["k"])
@@ -222,6 +222,8 @@ class Job:
         else:
             ids = self.ids
         L["pool"].quantize(L["k"], L["v"], ids)
+        if mark is not None:
+            mark.record()   # the encoder's span ends here; the remap of evicted slots follows
         if self.evict is not None:
             L["pool"].invalidate(self.evict)
 
@@ -263,9 +265,9 @@ class Job:
     def step(self, events=None):
         for L in self.layers:
             if events is not None:
-                e0, e1, e2 = events.pop()
+                e0, eq, e1, e2 = events.pop()
                 e0.record()
-            self.quantize_layer(L)
+            self.quantize_layer(L, eq if events is not None else None)
             if events is not None:
                 e1.record()
             self.decode_layer(L)
@@ -382,7 +384,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     # timed region: K steps, events around every quantise and decode launch
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
           for _ in range(args.steps * job.n_layers)]
     todo = list(reversed(ev))
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -398,8 +400,9 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     elapsed = reduce_max(start.elapsed_time(stop) / 1e3, dev)
-    q_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
-    d_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    q_ms = statistics.mean(a.elapsed_time(b) for a, b, _, _ in ev)
+    inv_ms = statistics.mean(b.elapsed_time(c) for _, b, c, _ in ev)   # remap of evicted slots (0 if none)
+    d_ms = statistics.mean(b.elapsed_time(c) for _, _, b, c in ev)
 
     # decode alone over all layers, cold (each layer's pool untouched for a full sweep)
     reps = max(3, min(20, args.steps))
@@ -495,6 +498,9 @@ def run_gpu(args):
             "kernels": {
                 "quantize": {"gbps": round(q_gbps, 1), "us_per_launch": round(q_ms * 1e3, 2),
                              "bytes_per_launch": job.quant_bytes},
+                "invalidate": {"us_per_launch_in_step": round(inv_ms * 1e3, 2),
+                               "slots_per_launch": 0 if job.evict is None else int(job.evict.numel()),
+                               "note": "remap of the evicted slots after each layer's encode (evicted workload only)"},
                 "decode": {"gbps_in_step": round(d_gbps, 1), "us_per_launch_in_step": round(d_ms * 1e3, 2),
                            "gbps_cold": round(d_cold_gbps, 1), "us_per_launch_cold": round(d_cold_ms * 1e3, 2),
                            "bytes_per_launch": job.decode_bytes,
