@@ -34,10 +34,16 @@ def oracle_pool(k: torch.Tensor, v: torch.Tensor, ids, n_q4: int, n_q8: int = 0,
 
 
 def assert_pool_equal(gpu, ref: O.OraclePool, blocks=None):
-    """Codes, scale/zero bits and remap mask bit-identical for `blocks`."""
+    """Codes, scale/zero bits and remap mask bit-identical for `blocks` (an
+    FP8 pool has E4M3 codes and the mask only)."""
     blocks = range(ref.n_blocks) if blocks is None else blocks
     for blk in blocks:
         blk = int(blk)
+        if ref.fp8:
+            for name in "kv":
+                np.testing.assert_array_equal(getattr(gpu, f"{name}_codes8")[blk].cpu().numpy(),
+                                              ref.codes8[name][blk], err_msg=f"{name} E4M3 codes, block {blk}")
+            continue
         for name in "kv":
             if blk < ref.n_q4:
                 g_codes = getattr(gpu, f"{name}_codes4")[blk].cpu().numpy()

@@ -117,12 +117,13 @@ def test_generation_step_append_then_decode():
     assert_close(out, want, what="append + decode")
 
 
-def _prefilled(d, hkv, dtype, rotated, n_q4, n_q8, lens, tables, seed):
+def _prefilled(d, hkv, dtype, rotated, n_q4, n_q8, lens, tables, seed, n_q2=0, fp8=False):
     """Two GPU pools and an oracle pool holding each sequence's first lens[b] tokens."""
     dev = cuda()
     name = "fp16" if dtype == torch.float16 else "bf16"
-    pools = [q4.Q4KVPool(hkv, d, n_q4, n_q8, k_rotated=rotated, device=dev) for _ in range(2)]
-    ref = O.OraclePool(hkv, d, n_q4, n_q8, k_rotated=rotated)
+    pools = [q4.Q4KVPool(hkv, d, n_q4, n_q8, k_rotated=rotated, device=dev, n_q2_blocks=n_q2, fp8=fp8)
+             for _ in range(2)]
+    ref = O.OraclePool(hkv, d, n_q4, n_q8, k_rotated=rotated, n_q2=n_q2, fp8=fp8)
     for b, n in enumerate(lens):
         if n == 0:
             continue
@@ -201,3 +202,39 @@ def test_append_decode_all_new_tokens_and_no_new_tokens():
     torch.cuda.synchronize()
     assert fused.read_device_error() == 0
     assert torch.equal(out, want)
+
+
+@pytest.mark.parametrize("kind", ["q2mix", "fp8"])
+def test_append_decode_other_block_classes(kind):
+    """The generation step over a pool mixing 2-, 4- and 8-bit blocks, and
+    over the FP8 comparison cache: equal to the two calls, and to the oracle."""
+    dev = cuda()
+    d, hq, hkv = 128, 32, 8
+    lens = [0, 255, 300, 1000]
+    new = [2, 3, 1, 2]
+    B, max_new, mb = len(lens), 3, 4
+    tables = torch.randperm(B * mb, generator=torch.Generator().manual_seed(5)).to(torch.int32).view(B, mb).numpy()
+    if kind == "q2mix":
+        (fused, sep), ref = _prefilled(d, hkv, torch.float16, True, 6, 4, lens, tables, seed=31, n_q2=6)
+    else:
+        (fused, sep), ref = _prefilled(d, hkv, torch.float16, False, 0, B * mb, lens, tables, seed=31, fp8=True)
+    kn, vn = W.random_small(B * max_new, hkv, d, "fp16", seed=32)
+    kn, vn = kn.view(B, max_new, hkv, d), vn.view(B, max_new, hkv, d)
+    q = torch.randn(B, hq, d, generator=torch.Generator().manual_seed(6)).to(torch.float16)
+    tab = torch.as_tensor(tables).to(dev)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device=dev)
+    nn = torch.tensor(new, dtype=torch.int32, device=dev)
+    grown = [n + a for n, a in zip(lens, new)]
+    out = q4.append_decode(fused, kn.to(dev), vn.to(dev), q.to(dev), tab, lens_d, nn, out_dtype=torch.float32)
+    sep.append(kn.to(dev), vn.to(dev), tab, lens_d, nn)
+    want_gpu = q4.decode_attention(sep, q.to(dev), tab, torch.tensor(grown, dtype=torch.int32, device=dev),
+                                   out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert fused.read_device_error() == 0
+    assert torch.equal(out, want_gpu)
+    kh, dt = host(kn.reshape(B * max_new, hkv, d))
+    vh, _ = host(vn.reshape(B * max_new, hkv, d))
+    ref.append_tokens(kh.reshape(B, max_new, hkv, d), vh.reshape(B, max_new, hkv, d), dt, tables, lens, new)
+    assert_pool_equal(fused, ref)
+    qh, qdt = host(q)
+    assert_close(out, O.decode_attention(ref, qh, qdt, tables, grown), what=f"append + decode, {kind}")
