@@ -1348,6 +1348,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   // -------------------------------------------------------------------------
   if (warp == C::kProducer) {
     if (lane != 0) return;
+    // the first copies need the tensor maps: fetch their descriptors now
+    const CUtensorMap* used[2] = {FP8 ? &maps.k8 : &maps.k4, FP8 ? &maps.v8 : &maps.v4};
+    for (int m = 0; m < 2; ++m)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(used[m])) : "memory");
     uint32_t it = 0;
     bool gave_up = false;
     // Global reads are issued ahead of the waits that follow them: the next
@@ -1377,7 +1381,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       int tok = t0;
       do {
         const int s = it % kNS;
-        const int32_t blk_read = tok < t1 ? a.tables[static_cast<int64_t>(b) * mb + tok / kBlockTokens] : -1;
+        // (read whenever the position is inside the table row, so the load
+        // does not wait for the sequence length it is checked against)
+        const int32_t blk_read =
+            tok < mb * kBlockTokens ? a.tables[static_cast<int64_t>(b) * mb + tok / kBlockTokens] : -1;
         // A stage that stays taken past the limit ends production: writing
         // the stage or arriving on its full barrier could then land in a
         // phase the consumers have not finished.  Their own bounded waits
@@ -1498,7 +1505,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     for (int item = i0; item < n_items; item += gridDim.x, ++k) {
       const int buf = k & 1;
       bool late = false;
-      if (!timed_out && !mbar_wait_idle(&done[buf], (k >> 1) & 1, 128, 1024)) {
+      // back-off capped at 256 ns: the wait after the CTA's last item is on
+      // the kernel's critical path
+      if (!timed_out && !mbar_wait_idle(&done[buf], (k >> 1) & 1, 64, 256)) {
         timed_out = late = true;
         if (lane == 0) raise_error(P.error_word, Q4KV_DEVERR_TIMEOUT);
       }
