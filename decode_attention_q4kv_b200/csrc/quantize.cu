@@ -33,6 +33,20 @@ __device__ __forceinline__ void red_and_if(bool p, uint32_t* addr, uint32_t v) {
   asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q red.global.and.b32 [%1], %2;\n}"
                :: "r"(static_cast<uint32_t>(p)), "l"(addr), "r"(v) : "memory");
 }
+
+// Stores predicated on p (one instruction each, no branch around them).
+__device__ __forceinline__ void st_if(bool p, void* a, uint32_t x) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q st.global.u32 [%1], %2;\n}"
+               :: "r"(static_cast<uint32_t>(p)), "l"(a), "r"(x) : "memory");
+}
+__device__ __forceinline__ void st_if(bool p, void* a, uint2 x) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q st.global.v2.u32 [%1], {%2, %3};\n}"
+               :: "r"(static_cast<uint32_t>(p)), "l"(a), "r"(x.x), "r"(x.y) : "memory");
+}
+__device__ __forceinline__ void st_if(bool p, void* a, uint4 x) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q st.global.v4.u32 [%1], {%2, %3, %4, %5};\n}"
+               :: "r"(static_cast<uint32_t>(p)), "l"(a), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w) : "memory");
+}
 constexpr int kEPL = 16;  // channels held by one lane
 
 template <int D>
@@ -251,7 +265,7 @@ __device__ __forceinline__ void clamped_codes(const float2 (&x)[8], float xs, co
 template <int BITS>
 __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupParams& g, int j,
                                             uint8_t* __restrict__ code_dst,
-                                            __half2* __restrict__ param_dst) {
+                                            __half2* __restrict__ param_dst, bool valid) {
   if (BITS == 2) {
     // element e (pair e % 8, half e / 8) at bits 2e of the lane's word: four
     // codes per byte, element 4i + m at bits 2m of byte i
@@ -261,7 +275,7 @@ __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupPar
       w |= (__float_as_uint(c[p].x) & 3u) << (2 * p);
       w |= (__float_as_uint(c[p].y) & 3u) << (2 * (p + 8));
     }
-    *reinterpret_cast<uint32_t*>(code_dst + j * 4) = w;
+    st_if(valid, code_dst + j * 4, w);
   } else if (BITS == 4) {
     // byte b holds elements 2b (low nibble) and 2b+1 (high nibble); the sums
     // are exact (integers below 2^24)
@@ -274,7 +288,7 @@ __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupPar
     }
     const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
-    *reinterpret_cast<uint2*>(code_dst + j * 8) = make_uint2(lo, hi);
+    st_if(valid, code_dst + j * 8, make_uint2(lo, hi));
   } else {
     // element e: pair e % 8, half e / 8
     uint32_t q[kEPL];
@@ -288,11 +302,12 @@ __device__ __forceinline__ void store_codes(const float2 (&c)[8], const GroupPar
     w.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
     w.z = __byte_perm(__byte_perm(q[8], q[9], 0x0040), __byte_perm(q[10], q[11], 0x0040), 0x5410);
     w.w = __byte_perm(__byte_perm(q[12], q[13], 0x0040), __byte_perm(q[14], q[15], 0x0040), 0x5410);
-    *reinterpret_cast<uint4*>(code_dst + j * 16) = w;
+    st_if(valid, code_dst + j * 16, w);
   }
   // the four lanes of a group hold the same parameters and all store them:
   // one branch fewer, and the stores merge in the same sector
-  param_dst[j >> 2] = __halves2half2(g.sh, g.zh);
+  const __half2 pv = __halves2half2(g.sh, g.zh);
+  st_if(valid, param_dst + (j >> 2), *reinterpret_cast<const uint32_t*>(&pv));
 }
 
 // FP8 comparison cache: the lane's 16 values as OCP E4M3 bytes (round to
@@ -324,10 +339,8 @@ __device__ __forceinline__ void encode_kv(const float2 (&xk)[8], float ks, const
   fast_codes<BITS>(xv, 1.0f, gv, cv);
   if (!gk.fast) clamped_codes<BITS>(xk, ks, gk, ck);
   if (!gv.fast) clamped_codes<BITS>(xv, 1.0f, gv, cv);
-  if (valid) {
-    store_codes<BITS>(ck, gk, j, kc, kp);
-    store_codes<BITS>(cv, gv, j, vc, vp);
-  }
+  store_codes<BITS>(ck, gk, j, kc, kp, valid);
+  store_codes<BITS>(cv, gv, j, vc, vp, valid);
 }
 
 // ---------------------------------------------------------------------------
