@@ -238,3 +238,29 @@ def test_append_decode_other_block_classes(kind):
     assert_pool_equal(fused, ref)
     qh, qdt = host(q)
     assert_close(out, O.decode_attention(ref, qh, qdt, tables, grown), what=f"append + decode, {kind}")
+
+
+def test_append_decode_past_the_table_raises_and_completes():
+    """An append that lands past the block table: the append skips the token
+    and raises Q4KV_DEVERR_SEQ_LEN, the decode over the grown length (beyond
+    the table) writes a zero row and raises the same bit; the other
+    sequence is unaffected, and the call completes (the decode then never
+    reads a block the append writes, so only its final grid wait orders them)."""
+    dev = cuda()
+    d, hq, hkv = 128, 16, 4
+    lens = [256, 100]
+    tables = np.array([[0], [1]], dtype=np.int32)
+    (fused, sep), ref = _prefilled(d, hkv, torch.float16, True, 2, 0, lens, tables, seed=41)
+    kn, vn = W.random_small(2, hkv, d, "fp16", seed=42)
+    kn, vn = kn.view(2, 1, hkv, d).to(dev), vn.view(2, 1, hkv, d).to(dev)
+    q = torch.randn(2, hq, d, generator=torch.Generator().manual_seed(43)).to(torch.float16).to(dev)
+    tab = torch.as_tensor(tables).to(dev)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device=dev)
+    out = q4.append_decode(fused, kn, vn, q, tab, lens_d, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert fused.read_device_error() & _lib.DEVERR_SEQ_LEN
+    assert torch.count_nonzero(out[0]) == 0
+    sep.append(kn[1:], vn[1:], tab[1:], lens_d[1:])
+    want = q4.decode_attention(sep, q[1:], tab[1:].clone(), lens_d[1:] + 1, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(out[1:], want)
