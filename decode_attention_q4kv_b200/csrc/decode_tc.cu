@@ -187,6 +187,14 @@ __device__ __forceinline__ uint32_t movtrans(uint32_t x) {
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
+// Four 8x8 b16 matrices from shared memory, transposed: lane 4 g + q gets
+// column g of rows 2 q and 2 q + 1 (low and high half) of matrix m in r[m];
+// lanes 8 m .. 8 m + 7 give the row addresses of matrix m.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -436,6 +444,7 @@ struct PairOffsets {
   static constexpr int NQ = KC >= 16 ? KC / 16 : 1;         // key loads per chunk (16 bytes, or one of 8)
   int k[2][NC * NQ];   // key rows pi(g), pi(g + 8)
   int v[4];            // value rows pi(2t), pi(2t+1), pi(2t+8), pi(2t+9) (thread g's bytes)
+  int lv[G::NG];       // ldmatrix row address of the lane, per group (4-bit values)
   int p[2];            // parameter rows pi(g), pi(g + 8) (the thread's two groups)
   int row[2];          // pi(g), pi(g + 8), relative to the base row
 
@@ -456,6 +465,12 @@ struct PairOffsets {
     const int vr[4] = {tok_perm(2 * t), tok_perm(2 * t + 1), tok_perm(2 * t + 8), tok_perm(2 * t + 9)};
 #pragma unroll
     for (int x = 0; x < 4; ++x) v[x] = swz<G::RB, G::SW>(base + vr[x], g * G::VB);
+    // matrix m = lane / 8: tokens 8 (m & 1) + [0, 8), channel half m >> 1 of
+    // the group (16 bytes); row i of a matrix is token pi(i) of its half tile
+    const int m = lane >> 3, i = lane & 7;
+#pragma unroll
+    for (int gr = 0; gr < G::NG; ++gr)
+      lv[gr] = swz<G::RB, G::SW>(base + tok_perm(8 * (m & 1) + i), gr * G::GB + 16 * (m >> 1));
   }
 };
 
@@ -470,7 +485,7 @@ constexpr float kLazy = 2.0f;
 // key-MMA chains and halve the softmax bookkeeping.  Thread t owns channels
 // 128c + 32t + [0, 32) of each key row; step kk uses chunk c = kk / 4, word
 // kk % 4.
-template <int D, int CB, int NTL, class BQ>
+template <int D, int CB, int NTL, bool VT, class BQ>
 __device__ __forceinline__ void pair_tiles(PairState<D>& st, const TileAt (&ta)[NTL],
                                            const PairOffsets<D, CB>& o, const BQ& bq, const PairConst& qc) {
   using G = Geo<D, CB>;
@@ -581,8 +596,31 @@ __device__ __forceinline__ void pair_tiles(PairState<D>& st, const TileAt (&ta)[
   for (int i = 0; i < NTL; ++i) {
     const uint32_t bw0 = movtrans(wb[i][0]);   // tokens pi(2t), pi(2t+1)
     const uint32_t bw1 = movtrans(wb[i][1]);   // tokens pi(8+2t), pi(9+2t)
-    uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
     const uint8_t* vc = ta[i].stg + Stg<D>::kOffV + ta[i].dr * G::RB;
+    if (VT && CB == 4) {
+      // as in the heads layout: tile 4 gr + j holds channels 64 gr + 4 g + j
+      // (rows g) and 64 gr + 32 + 4 g + j (rows g + 8)
+      const uint32_t vs = static_cast<uint32_t>(__cvta_generic_to_shared(vc));
+#pragma unroll
+      for (int gr = 0; gr < G::NG; ++gr) {
+        uint32_t r[4];
+        ldsm_x4_trans(vs + o.lv[gr], r);
+        const uint32_t s[4] = {r[0] >> 8, r[1] >> 8, r[2] >> 8, r[3] >> 8};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t* w = j < 2 ? r : s;
+          uint32_t a[4];
+          if (j % 2 == 0) {
+            a[0] = lo_nib(w[0]); a[1] = lo_nib(w[2]); a[2] = lo_nib(w[1]); a[3] = lo_nib(w[3]);
+          } else {
+            a[0] = hi_nib(w[0]); a[1] = hi_nib(w[2]); a[2] = hi_nib(w[1]); a[3] = hi_nib(w[3]);
+          }
+          mma16816(st.o[4 * gr + j], a, bw0, bw1);
+        }
+      }
+      continue;
+    }
+    uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
     if (VW == 1) {
       v0[0] = lds<uint32_t>(vc + o.v[0]);
       v1[0] = lds<uint32_t>(vc + o.v[1]);
@@ -658,6 +696,7 @@ struct HeadOffsets {
   static constexpr int NG = G::NG;
   int k[2][NG];
   int v[4][NG];
+  int lv[NG];   // ldmatrix row address of the lane, per group (4-bit values)
   int p[2];
   int row[2];   // relative to the base row
 
@@ -677,11 +716,22 @@ struct HeadOffsets {
     for (int x = 0; x < 4; ++x)
 #pragma unroll
       for (int gr = 0; gr < NG; ++gr) v[x][gr] = swz<G::RB, G::SW>(base + vr[x], gr * G::GB + g * vb);
+    // matrix m = lane / 8: tokens 8 (m & 1) + [0, 8), channel half m >> 1 of
+    // the group (16 bytes); row i of a matrix is token pi(i) of its half tile
+    const int m = lane >> 3, i = lane & 7;
+#pragma unroll
+    for (int gr = 0; gr < NG; ++gr)
+      lv[gr] = swz<G::RB, G::SW>(base + tok_perm(8 * (m & 1) + i), gr * G::GB + 16 * (m >> 1));
   }
 };
 
 // NTL tiles in the heads layout, one online-softmax update over all of them.
-template <int D, int CB, int NTL, class BQ>
+// VT (4-bit values only): the value codes come in by transposed ldmatrix and
+// value tile 4 gr + j holds channels 64 gr + 4 g + j (rows g) and
+// 64 gr + 32 + 4 g + j (rows g + 8), scaled 2^-24 for even j, 2^-20 for odd;
+// otherwise tile 4 gr + bp holds 64 gr + 8 g + 2 bp (rows g) and that + 1
+// (rows g + 8), the mapping every block width shares.
+template <int D, int CB, int NTL, bool VT, class BQ>
 __device__ __forceinline__ void head_tiles(HeadState<D>& st, const TileAt (&ta)[NTL],
                                            const HeadOffsets<D, CB>& o, const BQ& bq, const HeadConst<D>& qc) {
   using G = Geo<D, CB>;
@@ -828,6 +878,25 @@ __device__ __forceinline__ void head_tiles(HeadState<D>& st, const TileAt (&ta)[
           movtrans(h2u(__floats2half2_rn(q[i][0][0] * sv[i][0][gr], q[i][0][1] * sv[i][0][gr])));
       const uint32_t bw1 =
           movtrans(h2u(__floats2half2_rn(q[i][1][0] * sv[i][1][gr], q[i][1][1] * sv[i][1][gr])));
+      if (VT && CB == 4) {
+        // r[0], r[1]: tokens 2 t, 2 t + 1 and 2 t + 8, 2 t + 9 of channels
+        // 64 gr + 4 g + [0, 4); r[2], r[3]: the same 32 channels up
+        uint32_t r[4];
+        ldsm_x4_trans(static_cast<uint32_t>(__cvta_generic_to_shared(vc)) + o.lv[gr], r);
+        const uint32_t s[4] = {r[0] >> 8, r[1] >> 8, r[2] >> 8, r[3] >> 8};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t* w = j < 2 ? r : s;
+          uint32_t a[4];
+          if (j % 2 == 0) {
+            a[0] = lo_nib(w[0]); a[1] = lo_nib(w[2]); a[2] = lo_nib(w[1]); a[3] = lo_nib(w[3]);
+          } else {
+            a[0] = hi_nib(w[0]); a[1] = hi_nib(w[2]); a[2] = hi_nib(w[1]); a[3] = hi_nib(w[3]);
+          }
+          mma16816(st.o[4 * gr + j], a, bw0, bw1);
+        }
+        continue;
+      }
       constexpr int VW = CB == 8 ? 2 : 1;
       uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
       if (CB == 4) {
@@ -1527,6 +1596,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   uint32_t it = 0;
   bool dead = false;
   const int row0 = warp * 16;   // the warp's base row: its first tile of a whole stage
+  // a pool of 4-bit blocks only reads its value codes by transposed ldmatrix
+  constexpr bool kVT = !MIXED && !FP8;
   PairOffsets<D, 4> poff4;
   HeadOffsets<D, 4> hoff4;
   PairOffsets<D, 8> off8f;
@@ -1577,27 +1648,27 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
 #pragma unroll
         for (int x = 0; x < NTL; ++x) fp8_tile<D>(fst, ta[x], off8f, qtab_t);
       } else if (!MIXED || cb == 4) {
-        if (LAY == kPairs) pair_tiles<D, 4, NTL>(pst, ta, poff4, bq, pc);
-        else head_tiles<D, 4, NTL>(hst, ta, hoff4, bq, hc);
+        if (LAY == kPairs) pair_tiles<D, 4, NTL, kVT>(pst, ta, poff4, bq, pc);
+        else head_tiles<D, 4, NTL, kVT>(hst, ta, hoff4, bq, hc);
       } else if (cb == 8) {
         if (LAY == kPairs) {
           PairOffsets<D, 8> o8;
           o8.init(lane, row0);
-          pair_tiles<D, 8, NTL>(pst, ta, o8, bq, pc);
+          pair_tiles<D, 8, NTL, false>(pst, ta, o8, bq, pc);
         } else {
           HeadOffsets<D, 8> o8;
           o8.init(lane, row0);
-          head_tiles<D, 8, NTL>(hst, ta, o8, bq, hc);
+          head_tiles<D, 8, NTL, false>(hst, ta, o8, bq, hc);
         }
       } else {
         if (LAY == kPairs) {
           PairOffsets<D, 2> o2;
           o2.init(lane, row0);
-          pair_tiles<D, 2, NTL>(pst, ta, o2, bq, pc);
+          pair_tiles<D, 2, NTL, false>(pst, ta, o2, bq, pc);
         } else {
           HeadOffsets<D, 2> o2;
           o2.init(lane, row0);
-          head_tiles<D, 2, NTL>(hst, ta, o2, bq, hc);
+          head_tiles<D, 2, NTL, false>(hst, ta, o2, bq, hc);
         }
       }
     };
@@ -1724,11 +1795,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       for (int mv = 0; mv < D / 16; ++mv) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int ch = (D / 8) * g + 2 * mv + (e >> 1);
+          const int ch = kVT ? kGroup * (mv / 4) + 32 * (e >> 1) + 4 * g + mv % 4 : (D / 8) * g + 2 * mv + (e >> 1);
           const int col = c0 + (e & 1);
           const int hh = col / NG, gr = col % NG;
-          if (hh < G && gr == ch / kGroup)
-            mo[ch * C::HP + hh] = __fmaf_rn(pst.o[mv][e], e < 2 ? kEvenScale : kOddScale, zz[e & 1]);
+          const float sc = (kVT ? mv % 2 : e >> 1) == 0 ? kEvenScale : kOddScale;
+          if (hh < G && gr == ch / kGroup) mo[ch * C::HP + hh] = __fmaf_rn(pst.o[mv][e], sc, zz[e & 1]);
         }
       }
     } else {
@@ -1762,8 +1833,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           const int gr = mv / 4;
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const int ch = kGroup * gr + 8 * g + 2 * (mv % 4) + r;
-            const float sc = r == 0 ? kEvenScale : kOddScale;
+            const int ch = kVT ? kGroup * gr + 32 * r + 4 * g + mv % 4 : kGroup * gr + 8 * g + 2 * (mv % 4) + r;
+            const float sc = (kVT ? mv % 2 : r) == 0 ? kEvenScale : kOddScale;
             *reinterpret_cast<float2*>(mo + ch * C::HP + 2 * t) =
                 make_float2(__fmaf_rn(hst.o[mv][2 * r], sc, zz[0][gr]),
                             __fmaf_rn(hst.o[mv][2 * r + 1], sc, zz[1][gr]));
