@@ -205,10 +205,10 @@ __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__
 
 // Value codes enter the fp16 MMA as exact fp16 numbers with no offset: a
 // nibble or byte c masked into the low mantissa bits of a zero-exponent fp16
-// is the subnormal c * 2^-24.  Rows of the value MMA for even channels carry
-// c * 2^-24, rows for odd channels c * 2^-20 (a 4-bit high nibble masked in
-// place is 16 c * 2^-24); each output channel therefore has one power-of-two
-// scale, undone exactly in the epilogue.
+// is the subnormal c * 2^-24.  Value tiles 4 gr + j of even j (even
+// channels, group_values) carry c * 2^-24, those of odd j c * 2^-20 (a 4-bit
+// high nibble masked in place is 16 c * 2^-24); each output channel therefore
+// has one power-of-two scale, undone exactly in the epilogue.
 __device__ __forceinline__ uint32_t lo_nib(uint32_t x) { return x & 0x000F000Fu; }   // c * 2^-24
 __device__ __forceinline__ uint32_t hi_nib(uint32_t x) { return x & 0x00F000F0u; }   // c * 2^-20
 __device__ __forceinline__ uint32_t byte_lo(uint32_t x) { return x & 0x00FF00FFu; }  // c * 2^-24
@@ -308,37 +308,85 @@ __device__ __forceinline__ void key_a2(uint32_t x0, uint32_t x1, uint32_t (&a)[4
   a[3] = (y1 >> 2) & 0x03030303u;
 }
 
-// Value A operand from a token pair's words: byte bp of each (4-bit: low
-// nibble = even channel, high nibble = odd channel; 8-bit: bytes 2bp, 2bp+1;
-// 2-bit: element pair 2 (bp % 2), +1 of byte bp / 2).  Every width lands on
-// the same per-channel scale: even channels c * 2^-24, odd channels
-// c * 2^-20, so blocks of all widths add into the same accumulators.
-template <int CB>
-__device__ __forceinline__ void value_pair(const uint32_t* w0, const uint32_t* w1, const uint32_t* w8,
-                                           const uint32_t* w9, int bp, uint32_t (&a)[4]) {
-  if (CB == 4) {
-    const int wi = bp / 4, b = bp % 4;
-    const uint32_t sel = b | ((b + 4) << 8);             // [T1.b, -, T2.b, -]
-    const uint32_t x01 = __byte_perm(w0[wi], w1[wi], sel);
-    const uint32_t x89 = __byte_perm(w8[wi], w9[wi], sel);
-    a[0] = lo_nib(x01); a[1] = hi_nib(x01); a[2] = lo_nib(x89); a[3] = hi_nib(x89);
-  } else if (CB == 8) {
-    const int wi = (2 * bp) / 4, b = (2 * bp) % 4;
-    const uint32_t sa = b | ((b + 4) << 8), sb = (b + 1) | ((b + 5) << 8);
-    a[0] = byte_lo(__byte_perm(w0[wi], w1[wi], sa));
-    a[1] = byte_hi(__byte_perm(w0[wi], w1[wi], sb));
-    a[2] = byte_lo(__byte_perm(w8[wi], w9[wi], sa));
-    a[3] = byte_hi(__byte_perm(w8[wi], w9[wi], sb));
+// 8- and 2-bit value operands in the transposed mapping (value tile 4 gr + j:
+// channel 64 gr + 4 g + j in rows g, that + 32 in rows g + 8; even j scaled
+// 2^-24, odd j 2^-20), from plain 32-bit loads.  8-bit: x and y hold
+// channels 4g .. 4g + 3 of a half group for two tokens; the operand pairs
+// their bytes j.
+__device__ __forceinline__ uint32_t vt_a8(uint32_t x, uint32_t y, int j) {
+  const uint32_t p = __byte_perm(x, y, j | ((j + 4) << 8));
+  return j % 2 == 0 ? byte_lo(p) : byte_hi(p);
+}
+// 2-bit: p holds in bytes 0 and 2 the code byte of channels 4g .. 4g + 3 for
+// two tokens (channel 4g + j at bits 2j); even j go to bits 0-1, odd j to
+// bits 4-5 (16 c * 2^-24).
+__device__ __forceinline__ uint32_t vt_a2(uint32_t p, int j) {
+  if (j == 0) return p & 0x00030003u;
+  if (j == 1) return (p << 2) & 0x00300030u;
+  if (j == 2) return (p >> 4) & 0x00030003u;
+  return (p >> 2) & 0x00300030u;
+}
+// One group's four value MMAs of a tile (B operand bw0, bw1: the weights of
+// tokens pi(2t), pi(2t+1) and pi(8+2t), pi(9+2t)).  Value tile 4 gr + j holds
+// channels 64 gr + 4 g + j (rows g) and 64 gr + 32 + 4 g + j (rows g + 8),
+// scaled 2^-24 for even j and 2^-20 for odd j, for every code width, so
+// blocks of all widths add into the same accumulators.
+//
+// 4-bit: one ldmatrix.x4.trans (b16 elements; matrices: tokens 0-7 and 8-15
+// of the tile x the two 16-byte halves of the group, row addresses off.lv)
+// gives lane (g, t) tokens (2t, 2t+1) and (2t+8, 2t+9) of channels
+// 64 gr + 4 g + [0, 4) and of the same channels + 32; nibble masks and one
+// 8-bit shift make the operands.  8- and 2-bit: plain 32-bit loads,
+// off.vt[x][h] ^ (gr * GB) being the word of token pi(2t), pi(2t+1),
+// pi(2t+8) or pi(2t+9) (x) that holds channels 64 gr + 32 h + 4 g .. (8-bit)
+// or their byte (2-bit: byte g % 4 of the word, picked by off.sel2).  A group
+// is a power-of-two byte span of the row and the swizzle XORs only bits inside
+// the row, so group gr's offset is group 0's with gr * GB XORed in.
+template <int D, int CB, class O>
+__device__ __forceinline__ void group_values(float (&acc)[D / 16][4], const uint8_t* vc, const O& off, int gr,
+                                             uint32_t bw0, uint32_t bw1) {
+  if constexpr (CB == 4) {
+    uint32_t r[4];
+    ldsm_x4_trans(static_cast<uint32_t>(__cvta_generic_to_shared(vc)) + off.lv[gr], r);
+    const uint32_t s[4] = {r[0] >> 8, r[1] >> 8, r[2] >> 8, r[3] >> 8};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t* x = j < 2 ? r : s;
+      uint32_t a[4];
+      if (j % 2 == 0) {
+        a[0] = lo_nib(x[0]); a[1] = lo_nib(x[2]); a[2] = lo_nib(x[1]); a[3] = lo_nib(x[3]);
+      } else {
+        a[0] = hi_nib(x[0]); a[1] = hi_nib(x[2]); a[2] = hi_nib(x[1]); a[3] = hi_nib(x[3]);
+      }
+      mma16816(acc[4 * gr + j], a, bw0, bw1);
+    }
   } else {
-    const int byte = bp / 2, wi = byte / 4, b = byte % 4, m = 2 * (bp % 2);
-    const uint32_t sel = b | ((b + 4) << 8);
-    const uint32_t x01 = __byte_perm(w0[wi], w1[wi], sel);
-    const uint32_t x89 = __byte_perm(w8[wi], w9[wi], sel);
-    // element m (even channel) to bits 0-1, element m + 1 (odd) to bits 4-5
-    a[0] = (x01 >> (2 * m)) & 0x00030003u;
-    a[2] = (x89 >> (2 * m)) & 0x00030003u;
-    a[1] = (m == 0 ? (x01 << 2) : (x01 >> 2)) & 0x00300030u;
-    a[3] = (m == 0 ? (x89 << 2) : (x89 >> 2)) & 0x00300030u;
+    uint32_t w[4][2];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) w[x][h] = lds<uint32_t>(vc + (off.vt[x][h] ^ (gr * Geo<D, CB>::GB)));
+    uint32_t p[4];
+    if (CB == 2) {
+      p[0] = __byte_perm(w[0][0], w[1][0], off.sel2);
+      p[1] = __byte_perm(w[0][1], w[1][1], off.sel2);
+      p[2] = __byte_perm(w[2][0], w[3][0], off.sel2);
+      p[3] = __byte_perm(w[2][1], w[3][1], off.sel2);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t a[4];
+      if (CB == 8) {
+        a[0] = vt_a8(w[0][0], w[1][0], j);
+        a[1] = vt_a8(w[0][1], w[1][1], j);
+        a[2] = vt_a8(w[2][0], w[3][0], j);
+        a[3] = vt_a8(w[2][1], w[3][1], j);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) a[k] = vt_a2(p[k], j);
+      }
+      mma16816(acc[4 * gr + j], a, bw0, bw1);
+    }
   }
 }
 
@@ -436,6 +484,21 @@ __device__ __forceinline__ void reset(PairState<D>& st) {
 // Per-thread byte offsets of tile 0 of a stage.  Tiles start at multiples of
 // 16 rows, so the token permutation and the TMA swizzle depend only on the
 // row's low four bits, and tile i sits i * 16 rows further on.
+// Group-0 word offsets for group_values_vt (8- and 2-bit codes; 4-bit leaves them unset).
+template <class G>
+__device__ __forceinline__ void init_vt(int (&vt)[4][2], uint32_t& sel2, int base, const int (&vr)[4], int g) {
+  constexpr int CB = G::GB * 8 / kGroup;
+  static_assert((G::GB & (G::GB - 1)) == 0 && G::RB % G::GB == 0, "groups are power-of-two spans of a row");
+  sel2 = static_cast<uint32_t>((g & 3) | (((g & 3) + 4) << 8));
+  if constexpr (CB != 4) {
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        vt[x][h] = swz<G::RB, G::SW>(base + vr[x], CB == 8 ? 32 * h + 4 * g : 8 * h + 4 * (g >> 2));
+  }
+}
+
 template <int D, int CB>
 struct PairOffsets {
   using G = Geo<D, CB>;
@@ -445,6 +508,8 @@ struct PairOffsets {
   int k[2][NC * NQ];   // key rows pi(g), pi(g + 8)
   int v[4];            // value rows pi(2t), pi(2t+1), pi(2t+8), pi(2t+9) (thread g's bytes)
   int lv[G::NG];       // ldmatrix row address of the lane, per group (4-bit values)
+  int vt[4][2];        // 8- and 2-bit value words of group 0 in the transposed mapping (group_values_vt)
+  uint32_t sel2;       // 2-bit: byte g % 4 of two words into bytes 0 and 2
   int p[2];            // parameter rows pi(g), pi(g + 8) (the thread's two groups)
   int row[2];          // pi(g), pi(g + 8), relative to the base row
 
@@ -471,6 +536,7 @@ struct PairOffsets {
 #pragma unroll
     for (int gr = 0; gr < G::NG; ++gr)
       lv[gr] = swz<G::RB, G::SW>(base + tok_perm(8 * (m & 1) + i), gr * G::GB + 16 * (m >> 1));
+    init_vt<G>(vt, sel2, base, vr, g);
   }
 };
 
@@ -485,7 +551,7 @@ constexpr float kLazy = 2.0f;
 // key-MMA chains and halve the softmax bookkeeping.  Thread t owns channels
 // 128c + 32t + [0, 32) of each key row; step kk uses chunk c = kk / 4, word
 // kk % 4.
-template <int D, int CB, int NTL, bool VT, class BQ>
+template <int D, int CB, int NTL, class BQ>
 __device__ __forceinline__ void pair_tiles(PairState<D>& st, const TileAt (&ta)[NTL],
                                            const PairOffsets<D, CB>& o, const BQ& bq, const PairConst& qc) {
   using G = Geo<D, CB>;
@@ -590,65 +656,14 @@ __device__ __forceinline__ void pair_tiles(PairState<D>& st, const TileAt (&ta)[
       st.z[1] = __fmaf_rn(q, wz[i][r][1], st.z[1]);
       wb[i][r] = h2u(__floats2half2_rn(q * ws[i][r][0], q * ws[i][r][1]));
     }
-  // ---- values ----
-  constexpr int VW = G::VB / 4;           // words of value codes per token row
+  // ---- values: every group with the tile's weights ----
 #pragma unroll
   for (int i = 0; i < NTL; ++i) {
     const uint32_t bw0 = movtrans(wb[i][0]);   // tokens pi(2t), pi(2t+1)
     const uint32_t bw1 = movtrans(wb[i][1]);   // tokens pi(8+2t), pi(9+2t)
     const uint8_t* vc = ta[i].stg + Stg<D>::kOffV + ta[i].dr * G::RB;
-    if (VT && CB == 4) {
-      // as in the heads layout: tile 4 gr + j holds channels 64 gr + 4 g + j
-      // (rows g) and 64 gr + 32 + 4 g + j (rows g + 8)
-      const uint32_t vs = static_cast<uint32_t>(__cvta_generic_to_shared(vc));
 #pragma unroll
-      for (int gr = 0; gr < G::NG; ++gr) {
-        uint32_t r[4];
-        ldsm_x4_trans(vs + o.lv[gr], r);
-        const uint32_t s[4] = {r[0] >> 8, r[1] >> 8, r[2] >> 8, r[3] >> 8};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t* w = j < 2 ? r : s;
-          uint32_t a[4];
-          if (j % 2 == 0) {
-            a[0] = lo_nib(w[0]); a[1] = lo_nib(w[2]); a[2] = lo_nib(w[1]); a[3] = lo_nib(w[3]);
-          } else {
-            a[0] = hi_nib(w[0]); a[1] = hi_nib(w[2]); a[2] = hi_nib(w[1]); a[3] = hi_nib(w[3]);
-          }
-          mma16816(st.o[4 * gr + j], a, bw0, bw1);
-        }
-      }
-      continue;
-    }
-    uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
-    if (VW == 1) {
-      v0[0] = lds<uint32_t>(vc + o.v[0]);
-      v1[0] = lds<uint32_t>(vc + o.v[1]);
-      v8[0] = lds<uint32_t>(vc + o.v[2]);
-      v9[0] = lds<uint32_t>(vc + o.v[3]);
-    } else if (VW == 2) {
-      const uint2 a0 = lds<uint2>(vc + o.v[0]), a1 = lds<uint2>(vc + o.v[1]);
-      const uint2 a8 = lds<uint2>(vc + o.v[2]), a9 = lds<uint2>(vc + o.v[3]);
-      v0[0] = a0.x; v0[VW - 1] = a0.y; v1[0] = a1.x; v1[VW - 1] = a1.y;
-      v8[0] = a8.x; v8[VW - 1] = a8.y; v9[0] = a9.x; v9[VW - 1] = a9.y;
-    } else {
-#pragma unroll
-      for (int q = 0; q < VW; q += 4) {   // 16-byte pieces of the thread's bytes (never swizzle-split)
-        const uint4 a0 = lds<uint4>(vc + o.v[0] + 4 * q), a1 = lds<uint4>(vc + o.v[1] + 4 * q);
-        const uint4 a8 = lds<uint4>(vc + o.v[2] + 4 * q), a9 = lds<uint4>(vc + o.v[3] + 4 * q);
-        v0[q] = a0.x; v0[q + 1] = a0.y; v0[q + 2] = a0.z; v0[q + 3] = a0.w;
-        v1[q] = a1.x; v1[q + 1] = a1.y; v1[q + 2] = a1.z; v1[q + 3] = a1.w;
-        v8[q] = a8.x; v8[q + 1] = a8.y; v8[q + 2] = a8.z; v8[q + 3] = a8.w;
-        v9[q] = a9.x; v9[q + 1] = a9.y; v9[q + 2] = a9.z; v9[q + 3] = a9.w;
-      }
-    }
-    // tile mv uses rows g -> channel cb + 2 mv and g + 8 -> cb + 2 mv + 1, cb = g D / 8
-#pragma unroll
-    for (int mv = 0; mv < D / 16; ++mv) {
-      uint32_t a[4];
-      value_pair<CB>(v0, v1, v8, v9, mv, a);
-      mma16816(st.o[mv], a, bw0, bw1);
-    }
+    for (int gr = 0; gr < G::NG; ++gr) group_values<D, CB>(st.o, vc, o, gr, bw0, bw1);
   }
 }
 
@@ -695,8 +710,9 @@ struct HeadOffsets {
   using G = Geo<D, CB>;
   static constexpr int NG = G::NG;
   int k[2][NG];
-  int v[4][NG];
   int lv[NG];   // ldmatrix row address of the lane, per group (4-bit values)
+  int vt[4][2];       // 8- and 2-bit value words of group 0 in the transposed mapping (group_values_vt)
+  uint32_t sel2;      // 2-bit: byte g % 4 of two words into bytes 0 and 2
   int p[2];
   int row[2];   // relative to the base row
 
@@ -704,7 +720,7 @@ struct HeadOffsets {
     const int g = lane >> 2, t = lane & 3;
     row[0] = tok_perm(g);
     row[1] = tok_perm(g + 8);
-    const int kb = 2 * CB, vb = CB;   // bytes of 16 and 8 channels
+    const int kb = 2 * CB;   // bytes of 16 channels
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
 #pragma unroll
@@ -712,26 +728,18 @@ struct HeadOffsets {
       p[x] = (base + row[x]) * G::PB;
     }
     const int vr[4] = {tok_perm(2 * t), tok_perm(2 * t + 1), tok_perm(2 * t + 8), tok_perm(2 * t + 9)};
-#pragma unroll
-    for (int x = 0; x < 4; ++x)
-#pragma unroll
-      for (int gr = 0; gr < NG; ++gr) v[x][gr] = swz<G::RB, G::SW>(base + vr[x], gr * G::GB + g * vb);
     // matrix m = lane / 8: tokens 8 (m & 1) + [0, 8), channel half m >> 1 of
     // the group (16 bytes); row i of a matrix is token pi(i) of its half tile
     const int m = lane >> 3, i = lane & 7;
 #pragma unroll
     for (int gr = 0; gr < NG; ++gr)
       lv[gr] = swz<G::RB, G::SW>(base + tok_perm(8 * (m & 1) + i), gr * G::GB + 16 * (m >> 1));
+    init_vt<G>(vt, sel2, base, vr, g);
   }
 };
 
 // NTL tiles in the heads layout, one online-softmax update over all of them.
-// VT (4-bit values only): the value codes come in by transposed ldmatrix and
-// value tile 4 gr + j holds channels 64 gr + 4 g + j (rows g) and
-// 64 gr + 32 + 4 g + j (rows g + 8), scaled 2^-24 for even j, 2^-20 for odd;
-// otherwise tile 4 gr + bp holds 64 gr + 8 g + 2 bp (rows g) and that + 1
-// (rows g + 8), the mapping every block width shares.
-template <int D, int CB, int NTL, bool VT, class BQ>
+template <int D, int CB, int NTL, class BQ>
 __device__ __forceinline__ void head_tiles(HeadState<D>& st, const TileAt (&ta)[NTL],
                                            const HeadOffsets<D, CB>& o, const BQ& bq, const HeadConst<D>& qc) {
   using G = Geo<D, CB>;
@@ -878,50 +886,7 @@ __device__ __forceinline__ void head_tiles(HeadState<D>& st, const TileAt (&ta)[
           movtrans(h2u(__floats2half2_rn(q[i][0][0] * sv[i][0][gr], q[i][0][1] * sv[i][0][gr])));
       const uint32_t bw1 =
           movtrans(h2u(__floats2half2_rn(q[i][1][0] * sv[i][1][gr], q[i][1][1] * sv[i][1][gr])));
-      if (VT && CB == 4) {
-        // r[0], r[1]: tokens 2 t, 2 t + 1 and 2 t + 8, 2 t + 9 of channels
-        // 64 gr + 4 g + [0, 4); r[2], r[3]: the same 32 channels up
-        uint32_t r[4];
-        ldsm_x4_trans(static_cast<uint32_t>(__cvta_generic_to_shared(vc)) + o.lv[gr], r);
-        const uint32_t s[4] = {r[0] >> 8, r[1] >> 8, r[2] >> 8, r[3] >> 8};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t* w = j < 2 ? r : s;
-          uint32_t a[4];
-          if (j % 2 == 0) {
-            a[0] = lo_nib(w[0]); a[1] = lo_nib(w[2]); a[2] = lo_nib(w[1]); a[3] = lo_nib(w[3]);
-          } else {
-            a[0] = hi_nib(w[0]); a[1] = hi_nib(w[2]); a[2] = hi_nib(w[1]); a[3] = hi_nib(w[3]);
-          }
-          mma16816(st.o[4 * gr + j], a, bw0, bw1);
-        }
-        continue;
-      }
-      constexpr int VW = CB == 8 ? 2 : 1;
-      uint32_t v0[VW], v1[VW], v8[VW], v9[VW];
-      if (CB == 4) {
-        v0[0] = lds<uint32_t>(vc + o.v[0][gr]);
-        v1[0] = lds<uint32_t>(vc + o.v[1][gr]);
-        v8[0] = lds<uint32_t>(vc + o.v[2][gr]);
-        v9[0] = lds<uint32_t>(vc + o.v[3][gr]);
-      } else if (CB == 2) {   // 2 bytes: channels 64 gr + 8 g + [0, 8)
-        v0[0] = lds<uint16_t>(vc + o.v[0][gr]);
-        v1[0] = lds<uint16_t>(vc + o.v[1][gr]);
-        v8[0] = lds<uint16_t>(vc + o.v[2][gr]);
-        v9[0] = lds<uint16_t>(vc + o.v[3][gr]);
-      } else {
-        const uint2 a0 = lds<uint2>(vc + o.v[0][gr]), a1 = lds<uint2>(vc + o.v[1][gr]);
-        const uint2 a8 = lds<uint2>(vc + o.v[2][gr]), a9 = lds<uint2>(vc + o.v[3][gr]);
-        v0[0] = a0.x; v0[VW - 1] = a0.y; v1[0] = a1.x; v1[VW - 1] = a1.y;
-        v8[0] = a8.x; v8[VW - 1] = a8.y; v9[0] = a9.x; v9[VW - 1] = a9.y;
-      }
-      // tile 4 gr + bp: rows g -> channel 64 gr + 8 g + 2 bp, g + 8 -> + 1
-#pragma unroll
-      for (int bp = 0; bp < 4; ++bp) {
-        uint32_t a[4];
-        value_pair<CB>(v0, v1, v8, v9, bp, a);
-        mma16816(st.o[4 * gr + bp], a, bw0, bw1);
-      }
+      group_values<D, CB>(st.o, vc, o, gr, bw0, bw1);
     }
   }
 }
@@ -1392,7 +1357,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   const PoolView& P = a.pool;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hkv = P.n_kv_heads, hq = a.plan.n_q_heads, G = hq / hkv;
-  const int S = a.plan.n_splits, tps = a.plan.tokens_per_split, mb = a.plan.max_blocks_per_seq;
+  const int tps = a.plan.tokens_per_split, mb = a.plan.max_blocks_per_seq;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNS; ++i) {
@@ -1596,8 +1561,6 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   uint32_t it = 0;
   bool dead = false;
   const int row0 = warp * 16;   // the warp's base row: its first tile of a whole stage
-  // a pool of 4-bit blocks only reads its value codes by transposed ldmatrix
-  constexpr bool kVT = !MIXED && !FP8;
   PairOffsets<D, 4> poff4;
   HeadOffsets<D, 4> hoff4;
   PairOffsets<D, 8> off8f;
@@ -1644,31 +1607,31 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     // Tile places are row deltas from the warp's base row (warp * 16).
     auto run = [&](auto ntl, const TileAt (&ta)[decltype(ntl)::value], int cb) {
       constexpr int NTL = decltype(ntl)::value;
-      if (FP8) {
+      if constexpr (FP8) {
 #pragma unroll
         for (int x = 0; x < NTL; ++x) fp8_tile<D>(fst, ta[x], off8f, qtab_t);
       } else if (!MIXED || cb == 4) {
-        if (LAY == kPairs) pair_tiles<D, 4, NTL, kVT>(pst, ta, poff4, bq, pc);
-        else head_tiles<D, 4, NTL, kVT>(hst, ta, hoff4, bq, hc);
+        if (LAY == kPairs) pair_tiles<D, 4, NTL>(pst, ta, poff4, bq, pc);
+        else head_tiles<D, 4, NTL>(hst, ta, hoff4, bq, hc);
       } else if (cb == 8) {
         if (LAY == kPairs) {
           PairOffsets<D, 8> o8;
           o8.init(lane, row0);
-          pair_tiles<D, 8, NTL, false>(pst, ta, o8, bq, pc);
+          pair_tiles<D, 8, NTL>(pst, ta, o8, bq, pc);
         } else {
           HeadOffsets<D, 8> o8;
           o8.init(lane, row0);
-          head_tiles<D, 8, NTL, false>(hst, ta, o8, bq, hc);
+          head_tiles<D, 8, NTL>(hst, ta, o8, bq, hc);
         }
       } else {
         if (LAY == kPairs) {
           PairOffsets<D, 2> o2;
           o2.init(lane, row0);
-          pair_tiles<D, 2, NTL, false>(pst, ta, o2, bq, pc);
+          pair_tiles<D, 2, NTL>(pst, ta, o2, bq, pc);
         } else {
           HeadOffsets<D, 2> o2;
           o2.init(lane, row0);
-          head_tiles<D, 2, NTL, false>(hst, ta, o2, bq, hc);
+          head_tiles<D, 2, NTL>(hst, ta, o2, bq, hc);
         }
       }
     };
@@ -1795,10 +1758,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       for (int mv = 0; mv < D / 16; ++mv) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int ch = kVT ? kGroup * (mv / 4) + 32 * (e >> 1) + 4 * g + mv % 4 : (D / 8) * g + 2 * mv + (e >> 1);
+          const int ch = kGroup * (mv / 4) + 32 * (e >> 1) + 4 * g + mv % 4;   // value tile mv = 4 gr + j
           const int col = c0 + (e & 1);
           const int hh = col / NG, gr = col % NG;
-          const float sc = (kVT ? mv % 2 : e >> 1) == 0 ? kEvenScale : kOddScale;
+          const float sc = mv % 2 == 0 ? kEvenScale : kOddScale;
           if (hh < G && gr == ch / kGroup) mo[ch * C::HP + hh] = __fmaf_rn(pst.o[mv][e], sc, zz[e & 1]);
         }
       }
@@ -1833,8 +1796,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           const int gr = mv / 4;
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const int ch = kVT ? kGroup * gr + 32 * r + 4 * g + mv % 4 : kGroup * gr + 8 * g + 2 * (mv % 4) + r;
-            const float sc = (kVT ? mv % 2 : r) == 0 ? kEvenScale : kOddScale;
+            const int ch = kGroup * gr + 32 * r + 4 * g + mv % 4;   // value tile mv = 4 gr + j
+            const float sc = mv % 2 == 0 ? kEvenScale : kOddScale;
             *reinterpret_cast<float2*>(mo + ch * C::HP + 2 * t) =
                 make_float2(__fmaf_rn(hst.o[mv][2 * r], sc, zz[0][gr]),
                             __fmaf_rn(hst.o[mv][2 * r + 1], sc, zz[1][gr]));
