@@ -258,7 +258,7 @@ class Job:
         L["pool"].append(self.k_new, self.v_new, L.get("tables", self.tables), self.lens_before)
 
     def append_decode_layer(self, L):
-        """The generation step as one call: append, with the decode overlapping it."""
+        """The generation step as one call (q4kv_append_decode)."""
         self.q4.append_decode(L["pool"], self.k_new, self.v_new, L["q"], L.get("tables", self.tables),
                               self.lens_before, plan=self.plan, workspace=self.ws, out=L["out"])
 
@@ -317,8 +317,8 @@ def job_throughput(world: int, bytes_per_step: float, steps: int, elapsed_s: flo
 # host code that picks the split count (the partials it writes depend on it).
 _CSRC = os.path.join("decode_attention_q4kv_b200", "csrc")
 KERNEL_SOURCES = {
-    "quantize": ("quantize.cu", "async_copy.cuh", "q4kv_internal.cuh"),
-    "decode": ("decode_tc.cu", "decode.cu", "api.cu", "async_copy.cuh", "q4kv_internal.cuh"),
+    "quantize": ("quantize.cu", "encode.cuh", "async_copy.cuh", "q4kv_internal.cuh"),
+    "decode": ("decode_tc.cu", "decode.cu", "api.cu", "encode.cuh", "async_copy.cuh", "q4kv_internal.cuh"),
 }
 
 
@@ -511,8 +511,8 @@ def run_gpu(args):
                            "append_then_decode_us": round(gen_ms * 1e3, 2),
                            "append_then_decode_separate_us": round(sep_ms * 1e3, 2),
                            "note": "one new token per sequence written over its last slot, then decode over "
-                                   "the grown cache: append_then_decode_us = q4kv_append_decode (the decode "
-                                   "overlaps the append), _separate_us = the two calls back to back"},
+                                   "the grown cache: append_then_decode_us = q4kv_append_decode (one decode launch "
+                                   "that encodes the new rows itself), _separate_us = the two calls back to back"},
                 "paging": paging,
                 "card": card,
                 "q2mix": q2mix,

@@ -384,7 +384,9 @@ def append_decode(pool: Q4KVPool, k_new: torch.Tensor, v_new: torch.Tensor, q: t
     sequence's position seq_lens[b] (lengths before the append, not
     modified), then decode q [B][Hq][D] over seq_lens[b] + n_new[b] tokens
     (+ T when n_new is None).  Same result as pool.append then
-    decode_attention with the grown lengths; the decode overlaps the append."""
+    decode_attention with the grown lengths, in one decode launch that
+    encodes the new rows itself (FP8 pools and plan kernel 0: the append
+    kernel, then a decode that overlaps it)."""
     dev = _require_cuda(k_new, v_new, q, block_tables, seq_lens)
     if k_new.dtype != v_new.dtype or k_new.dtype not in _IN_DTYPES:
         raise ValueError("k_new and v_new must share dtype float16 or bfloat16")

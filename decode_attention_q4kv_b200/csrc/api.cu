@@ -442,6 +442,11 @@ static q4kv_status prepare_decode(const q4kv_pool* pool, const q4kv_decode_plan*
   a->add_lens = nullptr;
   a->add_const = 0;
   a->defer_wait = 0;
+  a->app_k = nullptr;
+  a->app_v = nullptr;
+  a->app_dtype = 0;
+  a->app_seq_stride = 0;
+  a->app_token_stride = 0;
   a->scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(plan->head_dim));
   a->out = out;
   a->out_dtype = out_dtype;
@@ -485,13 +490,22 @@ q4kv_status q4kv_append_decode(const q4kv_pool* pool, const q4kv_decode_plan* pl
   if (st != Q4KV_OK || empty) return st;
   cudaStream_t s = as_stream(stream);
   if (rows > 0) {
-    const cudaError_t e = launch_append(view_of(*pool), k_new, v_new, in_dtype, plan->batch, max_new, n_new,
-                                        seq_stride, token_stride, block_tables, plan->max_blocks_per_seq,
-                                        seq_lens, s);
-    if (e != cudaSuccess) return from_cuda(e);
     a.add_lens = n_new;
     a.add_const = max_new;
-    a.defer_wait = 1;
+    if (!a.pool.fp8 && plan->kernel == 1) {
+      // one launch: the tensor-core kernel encodes the new rows itself
+      a.app_k = k_new;
+      a.app_v = v_new;
+      a.app_dtype = in_dtype;
+      a.app_seq_stride = seq_stride;
+      a.app_token_stride = token_stride;
+    } else {
+      const cudaError_t e = launch_append(view_of(*pool), k_new, v_new, in_dtype, plan->batch, max_new, n_new,
+                                          seq_stride, token_stride, block_tables, plan->max_blocks_per_seq,
+                                          seq_lens, s);
+      if (e != cudaSuccess) return from_cuda(e);
+      a.defer_wait = 1;
+    }
   }
   return from_cuda(launch_decode(a, s));
 }

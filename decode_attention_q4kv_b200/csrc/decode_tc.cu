@@ -61,6 +61,7 @@
 #include <type_traits>
 
 #include "async_copy.cuh"
+#include "encode.cuh"
 #include "q4kv_internal.cuh"
 
 namespace q4kv {
@@ -105,6 +106,7 @@ struct Cfg {
   static constexpr int kThreads = (CW + 2) * 32; // + producer + aux
   static constexpr int kProducer = CW;
   static constexpr int kAux = CW + 1;
+  static constexpr int kAppender = CW + 2;   // fused-append instantiations only
   static constexpr int NG = D / kGroup;
   static constexpr int KK = D / 32;              // key MMA steps (32 channels each)
   static constexpr int HP = 1024 / D;            // heads per merge row (g * D <= 1024)
@@ -176,6 +178,27 @@ __device__ __forceinline__ bool mbar_wait_hot(uint64_t* bar, uint32_t parity) {
   for (int i = 0; i < Q4KV_DEC_SPIN; ++i)
     if (mbar_try(bar, parity)) return true;
   return mbar_wait(bar, parity);
+}
+
+// A monotonic progress counter in shared memory: the writer publishes with
+// a release store, the reader waits (bounded, sleeping between tests) for a
+// value with acquire loads.
+__device__ __forceinline__ void st_release_cta(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_cta(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool wait_count(const uint32_t* p, uint32_t v) {
+  unsigned ns = 32;
+  for (unsigned i = 0; i < 4 * kSpinLimit; ++i) {
+    if (ld_acquire_cta(p) >= v) return true;
+    __nanosleep(ns);
+    ns = ns < 128 ? 2 * ns : 128;
+  }
+  return false;
 }
 
 // Barrier among the warps of the CTA that are not the producer.
@@ -1317,13 +1340,85 @@ __device__ void merge_item(const DecodeArgs& a, int item, const float* mrg_o, co
 }
 
 // ---------------------------------------------------------------------------
+// Fused append: the appender warp encodes the new rows of an item's (sequence, KV
+// head) whose positions fall in the item's split, with the append kernel's
+// encoding steps (encode.cuh): up to VPW tokens of one block per pass (a
+// lane holds 16 channels of one token), so the block and its code width are
+// the same for the whole warp and every shuffle runs converged.  Each such
+// item clears the new slots' mask bits (the bits are shared by the KV heads;
+// clearing is idempotent).  The proxy fence orders these stores before the
+// producer's bulk copies of the block, which follow the appender's count.
+// ---------------------------------------------------------------------------
+template <int D, bool MIXED>
+__device__ __forceinline__ void append_rows(const DecodeArgs& a, int item, int lane) {
+  using S = Shape<D>;
+  const PoolView& P = a.pool;
+  int b, kvh, split;
+  item_coords(a, item, b, kvh, split);
+  const int old = a.seq_lens[b];
+  const int nn = a.add_lens != nullptr ? a.add_lens[b] : a.add_const;
+  const int tps = a.plan.tokens_per_split, mb = a.plan.max_blocks_per_seq;
+  const int64_t cap = static_cast<int64_t>(mb) * kBlockTokens;
+  // new rows i whose position old + i lies in this split
+  const int64_t lo = max(static_cast<int64_t>(0), static_cast<int64_t>(split) * tps - old);
+  const int64_t hi = min(static_cast<int64_t>(nn), static_cast<int64_t>(split + 1) * tps - old);
+  if (old < 0 || lo >= hi) return;
+  const int r = lane / S::LPV, j = lane % S::LPV;
+  const bool rot = P.k_rotated != 0;
+  const float ks = rot ? kRotScale<D> : 1.0f;
+  for (int64_t i0 = lo; i0 < hi;) {
+    const int64_t p0 = old + i0;
+    const int64_t i1 = min(min(i0 + S::VPW, hi), i0 + (kBlockTokens - p0 % kBlockTokens));   // one block
+    const bool live = i0 + r < i1;
+    const int64_t i = live ? i0 + r : i1 - 1;   // lanes past the pass's rows read a real row, store nothing
+    const int32_t blk = p0 < cap ? __ldg(a.tables + static_cast<int64_t>(b) * mb + p0 / kBlockTokens) : -1;
+    const bool ok = blk >= 0 && blk < P.n_blocks();
+    if (!ok && lane == 0) raise_error(P.error_word, p0 < cap ? Q4KV_DEVERR_BLOCK_ID : Q4KV_DEVERR_SEQ_LEN);
+    const int bk = ok ? blk : 0;
+    const int slot = static_cast<int>((old + i) % kBlockTokens);
+    const int64_t src = b * a.app_seq_stride + i * a.app_token_stride + kvh * D + j * kEPL;
+    const uint4* kp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.app_k) + src);
+    const uint4* vp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.app_v) + src);
+    const uint4 k0 = __ldg(kp), k1 = __ldg(kp + 1), v0 = __ldg(vp), v1 = __ldg(vp + 1);
+    float2 xk[8], xv[8];
+    if (a.app_dtype == Q4KV_BF16) {
+      unpack16<__nv_bfloat16>(k0, k1, xk);
+      unpack16<__nv_bfloat16>(v0, v1, xv);
+    } else {
+      unpack16<__half>(k0, k1, xk);
+      unpack16<__half>(v0, v1, xv);
+    }
+    if (rot) rotate_pairs<D>(xk, j);
+    const bool valid = live && ok;
+    const int bits = MIXED ? P.bits_of(bk) : 4;   // the same for the whole pass
+    const int64_t phys = bits == 4 ? bk : (bits == 8 ? bk - P.n_q4 : bk - P.n_q4 - P.n_q8);
+    const int64_t row = (phys * P.n_kv_heads + kvh) * kBlockTokens + slot;   // (block, head, slot)
+    if (MIXED && bits == 8)
+      encode_kv<8>(xk, ks, xv, j, valid, P.k_codes8 + row * D, P.k_params8 + row * S::NG, P.v_codes8 + row * D,
+                   P.v_params8 + row * S::NG);
+    else if (MIXED && bits == 2)
+      encode_kv<2>(xk, ks, xv, j, valid, P.k_codes2 + row * (D / 4), P.k_params2 + row * S::NG,
+                   P.v_codes2 + row * (D / 4), P.v_params2 + row * S::NG);
+    else
+      encode_kv<4>(xk, ks, xv, j, valid, P.k_codes4 + row * (D / 2), P.k_params4 + row * S::NG,
+                   P.v_codes4 + row * (D / 2), P.v_params4 + row * S::NG);
+    if (valid && j == 0)
+      atomicAnd(P.mask + static_cast<int64_t>(bk) * kMaskWords + slot / 32, ~(1u << (slot % 32)));
+    i0 = i1;
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
 // MIXED: the pool may hold 8- or 2-bit blocks beside the 4-bit ones; a pool
 // of 4-bit blocks only runs an instantiation without those paths (fewer
-// registers held for them).
-template <int D, int LAY, bool FP8, bool MIXED>
-__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
+// registers held for them).  APP: a fused append (DecodeArgs::app_k), done by
+// one more warp (the appender); a plain decode runs an instantiation without
+// it.
+template <int D, int LAY, bool FP8, bool MIXED, bool APP>
+__global__ void __launch_bounds__(Cfg<D>::kThreads + (APP ? 32 : 0), 1)
     decode_tc_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ TileMaps maps,
                      int n_items) {
   using C = Cfg<D>;
@@ -1340,6 +1435,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   uint64_t* qready = empty + kNS;   // [2] aux -> consumers: query table of an item ready
   uint64_t* done = qready + 2;      // [2] consumers -> aux: item merged-in, its table free
   uint64_t* mfree = done + 2;       // aux -> consumers: merge buffer read
+  // appender -> producer: how many of the CTA's items have their appended rows in the pool
+  uint32_t* n_enc = reinterpret_cast<uint32_t*>(mfree + 1);
   uint8_t* qtab0 = smem + C::kOffQTab;
   int* qint = reinterpret_cast<int*>(smem + C::kOffQInt);
   int* gsum = reinterpret_cast<int*>(smem + C::kOffQAux);
@@ -1369,6 +1466,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       mbar_init(&done[i], CW);
     }
     mbar_init(mfree, 1);
+    *n_enc = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (FP8) {   // heads past G of the FP8 query tables stay zero
@@ -1402,10 +1500,16 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     // An append just before: its writes land in blocks at or past the old
     // length, which are read only after waiting for the append grid.
     bool waited = !a.defer_wait;
+    // A fused append: item k's rows are in the pool once the appender's count
+    // passes k, waited for before the item's first block at or past the old
+    // length.
+    constexpr bool fused = APP && !FP8;
     int2 seq_next = blockIdx.x < n_items ? seq_of(blockIdx.x) : make_int2(0, 0);
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int k = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
       int b, kvh, split;
       item_coords(a, item, b, kvh, split);
+      bool enc_wait = fused;
       const int seq = seq_next.y, fresh_blk = seq_next.x / kBlockTokens;
       if (item + static_cast<int>(gridDim.x) < n_items) seq_next = seq_of(item + gridDim.x);
       const bool bad_seq = seq < 0 || seq > mb * kBlockTokens;
@@ -1426,6 +1530,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         if (!mbar_wait_idle(&empty[s], ((it / kNS) & 1) ^ 1, 32, 128)) {
           gave_up = true;
           break;
+        }
+        if (enc_wait && tok < t1 && tok / kBlockTokens >= fresh_blk) {
+          if (!wait_count(n_enc, static_cast<uint32_t>(k + 1))) {
+            gave_up = true;
+            break;
+          }
+          enc_wait = false;
         }
         uint8_t* stg = stages + s * kStageBytes;
         StageMeta meta;
@@ -1495,6 +1606,21 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       if (!mbar_wait(&full[k % kNS], (k / kNS) & 1)) break;
     if (!waited) griddep_wait();   // this grid never completes before the append
     return;
+  }
+
+  // -------------------------------------------------------------------------
+  // appender warp (fused append): every item's new rows, in item order
+  // -------------------------------------------------------------------------
+  if constexpr (APP && !FP8) {
+    if (warp == C::kAppender) {
+      uint32_t k = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        append_rows<D, MIXED>(a, item, lane);
+        __syncwarp();
+        if (lane == 0) st_release_cta(n_enc, ++k);
+      }
+      return;
+    }
   }
 
   // -------------------------------------------------------------------------
@@ -1890,23 +2016,26 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
     return cudaErrorInvalidValue;
 
   cudaError_t e = cudaSuccess;
-#define Q4KV_TC(DD, LL, F8, MX)                                                                    \
+#define Q4KV_TC(DD, LL, F8, MX, AP)                                                                 \
   do {                                                                                             \
-    e = cudaFuncSetAttribute(decode_tc_kernel<DD, LL, F8, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(decode_tc_kernel<DD, LL, F8, MX, AP>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              static_cast<int>(smem));                                              \
     if (e == cudaSuccess)                                                                          \
-      e = launch_pdl(decode_tc_kernel<DD, LL, F8, MX>, dim3(grid), dim3(Cfg<DD>::kThreads), smem, stream, a, \
-                     maps, n_items);                                                               \
+      e = launch_pdl(decode_tc_kernel<DD, LL, F8, MX, AP>, dim3(grid), dim3(Cfg<DD>::kThreads + (AP ? 32 : 0)), \
+                     smem, stream, a, maps, n_items);                                              \
   } while (0)
-#define Q4KV_TCM(DD, LL)                    \
-  do {                                      \
-    if (mixed) Q4KV_TC(DD, LL, false, true); \
-    else Q4KV_TC(DD, LL, false, false);      \
+#define Q4KV_TCM(DD, LL)                           \
+  do {                                             \
+    if (mixed && app) Q4KV_TC(DD, LL, false, true, true);   \
+    else if (mixed) Q4KV_TC(DD, LL, false, true, false);    \
+    else if (app) Q4KV_TC(DD, LL, false, false, true);      \
+    else Q4KV_TC(DD, LL, false, false, false);              \
   } while (0)
   const int lay = decode_tc_layout(d, g);
   const bool mixed = a.pool.n_q8 > 0 || a.pool.n_q2 > 0;
-  if (a.pool.fp8 && d == 128) Q4KV_TC(128, kHeads, true, false);   // FP8 comparison cache: heads are the columns
-  else if (a.pool.fp8) Q4KV_TC(256, kHeads, true, false);
+  const bool app = a.app_k != nullptr;   // never set for FP8 pools (their appends run the append kernel)
+  if (a.pool.fp8 && d == 128) Q4KV_TC(128, kHeads, true, false, false);   // FP8 comparison cache: heads are the columns
+  else if (a.pool.fp8) Q4KV_TC(256, kHeads, true, false, false);
   else if (d == 128 && lay == kPairs) Q4KV_TCM(128, kPairs);
   else if (d == 128) Q4KV_TCM(128, kHeads);
   else if (lay == kPairs) Q4KV_TCM(256, kPairs);

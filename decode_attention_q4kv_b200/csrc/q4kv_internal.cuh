@@ -172,6 +172,15 @@ struct DecodeArgs {
   // all land at positions >= seq_lens[b]; the tensor-core kernel then waits
   // for it only before it reads those blocks (programmatic dependent launch).
   int defer_wait;
+  // Fused append (tensor-core kernel, pools of 4-, 8- and 2-bit blocks): when
+  // app_k is set, the kernel itself encodes new row i < (add_lens ? add_lens[b]
+  // : add_const) of sequence b -- element (b, i, h, c) at b * app_seq_stride +
+  // i * app_token_stride + h * D + c of app_k and app_v, 16-bit app_dtype --
+  // into the pool at position seq_lens[b] + i before it reads that block.
+  const void* app_k;
+  const void* app_v;
+  int app_dtype;
+  int64_t app_seq_stride, app_token_stride;
   float scale;
   void* out;
   int out_dtype;

@@ -320,10 +320,14 @@ q4kv_status q4kv_decode_attention(const q4kv_pool *pool, const q4kv_decode_plan 
  * One generation step: append each sequence's new tokens, then decode over
  * the grown cache ([AMBP] sec. 2.1 item 4: EXTEND grows the cache in place,
  * then attention reads it).  Equal to q4kv_append_tokens followed by
- * q4kv_decode_attention with lengths seq_lens[b] + n_new[b], but faster: the
- * decode starts while the append runs (programmatic dependent launch) and
- * waits for it only before it streams a block at or past position
- * seq_lens[b], the only blocks an append writes.
+ * q4kv_decode_attention with lengths seq_lens[b] + n_new[b] (the same pool
+ * bytes and the same output), but faster.  For pools of 4-, 8- and 2-bit
+ * blocks with plan->kernel == 1 it is one decode launch (plus the split
+ * merge): one extra warp per CTA encodes the new rows of the CTA's items, and
+ * the CTA reads a block at or past position seq_lens[b] -- the only blocks an
+ * append writes -- only after those rows are in.  For FP8 pools and plan
+ * kernel 0 the append kernel runs first and the decode starts while it runs
+ * (programmatic dependent launch), waiting for it only before such blocks.
  *   plan         as for q4kv_decode_attention; plan->batch sequences and
  *                plan->max_blocks_per_seq block-table columns for both steps
  *   k_new, v_new, in_dtype, max_new, n_new, seq_stride, token_stride
