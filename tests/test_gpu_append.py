@@ -145,9 +145,10 @@ def _prefilled(d, hkv, dtype, rotated, n_q4, n_q8, lens, tables, seed, n_q2=0, f
                                                          (256, 8, 4, torch.float16, True, 6)])
 @pytest.mark.parametrize("n_splits", [0, 1, 3])
 def test_append_decode_matches_separate_calls_and_oracle(d, hq, hkv, dtype, rotated, n_q8, n_splits):
-    """The fused generation step (the decode overlapping the append, waiting
-    for it only before the blocks it writes) gives exactly the output of an
-    append followed by a decode over the grown lengths, and the oracle's."""
+    """The generation step in one call (one decode launch whose extra warp
+    encodes the new rows before the producer reads their blocks) gives
+    exactly the pool and the output of an append followed by a decode over
+    the grown lengths, and the oracle's."""
     dev = cuda()
     lens = [0, 100, 255, 256, 700, 1023]        # empty, mid-block, a block boundary crossed, full blocks
     new = [3, 1, 3, 0, 2, 1]
@@ -178,6 +179,43 @@ def test_append_decode_matches_separate_calls_and_oracle(d, hq, hkv, dtype, rota
     assert_pool_equal(fused, ref)
     qh, qdt = host(q)
     assert_close(out, O.decode_attention(ref, qh, qdt, tables, grown), what=f"append + decode {d}/{hq}/{hkv}")
+
+
+@pytest.mark.parametrize("d,hq,hkv", [(128, 40, 8), (256, 16, 8)])
+def test_append_decode_rows_across_split_and_block_boundaries(d, hq, hkv):
+    """New rows of one sequence that fall in two splits (and two blocks of
+    different widths): each split's item encodes its own part, and the
+    result equals the two calls and the oracle."""
+    dev = cuda()
+    lens = [510, 0, 1020, 255]          # + new: 510..512 and 1020..1024 cross a split (512 tokens) and a block
+    new = [3, 2, 5, 1]
+    B, max_new, mb = len(lens), 5, 5
+    tables = torch.randperm(B * mb, generator=torch.Generator().manual_seed(d + 3)).to(torch.int32).view(B, mb).numpy()
+    n_q8 = 7
+    (fused, sep), ref = _prefilled(d, hkv, torch.bfloat16, True, B * mb - n_q8, n_q8, lens, tables, seed=d + 5)
+    kn, vn = W.random_small(B * max_new, hkv, d, "bf16", seed=41)
+    kn, vn = kn.view(B, max_new, hkv, d), vn.view(B, max_new, hkv, d)
+    q = torch.randn(B, hq, d, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    tab = torch.as_tensor(tables).to(dev)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device=dev)
+    nn = torch.tensor(new, dtype=torch.int32, device=dev)
+    grown = [n + a for n, a in zip(lens, new)]
+    plan = q4.DecodePlan(B, hq, hkv, d, mb, n_splits=3)
+    assert plan.c.tokens_per_split == 512
+    out = q4.append_decode(fused, kn.to(dev), vn.to(dev), q.to(dev), tab, lens_d, nn, out_dtype=torch.float32,
+                           plan=plan)
+    sep.append(kn.to(dev), vn.to(dev), tab, lens_d, nn)
+    want_gpu = q4.decode_attention(sep, q.to(dev), tab, torch.tensor(grown, dtype=torch.int32, device=dev),
+                                   out_dtype=torch.float32, plan=plan)
+    torch.cuda.synchronize()
+    assert fused.read_device_error() == 0
+    assert torch.equal(out, want_gpu)
+    kh, dt = host(kn.reshape(B * max_new, hkv, d))
+    vh, _ = host(vn.reshape(B * max_new, hkv, d))
+    ref.append_tokens(kh.reshape(B, max_new, hkv, d), vh.reshape(B, max_new, hkv, d), dt, tables, lens, new)
+    assert_pool_equal(fused, ref)
+    qh, qdt = host(q)
+    assert_close(out, O.decode_attention(ref, qh, qdt, tables, grown), what=f"rows across splits {d}")
 
 
 def test_append_decode_all_new_tokens_and_no_new_tokens():
