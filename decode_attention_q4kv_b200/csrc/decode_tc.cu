@@ -1356,7 +1356,8 @@ __device__ __forceinline__ void append_rows(const DecodeArgs& a, int item, int l
   int b, kvh, split;
   item_coords(a, item, b, kvh, split);
   const int old = a.seq_lens[b];
-  const int nn = a.add_lens != nullptr ? a.add_lens[b] : a.add_const;
+  // add_const is max_new here: rows past it are not read (as in the append kernel)
+  const int nn = a.add_lens != nullptr ? min(a.add_lens[b], a.add_const) : a.add_const;
   const int tps = a.plan.tokens_per_split, mb = a.plan.max_blocks_per_seq;
   const int64_t cap = static_cast<int64_t>(mb) * kBlockTokens;
   // new rows i whose position old + i lies in this split
