@@ -181,7 +181,7 @@ def test_append_decode_matches_separate_calls_and_oracle(d, hq, hkv, dtype, rota
     assert_close(out, O.decode_attention(ref, qh, qdt, tables, grown), what=f"append + decode {d}/{hq}/{hkv}")
 
 
-@pytest.mark.parametrize("d,hq,hkv", [(128, 40, 8), (256, 16, 8)])
+@pytest.mark.parametrize("d,hq,hkv", [(128, 40, 8), (256, 16, 8), (256, 16, 4)])   # heads, pairs, heads
 def test_append_decode_rows_across_split_and_block_boundaries(d, hq, hkv):
     """New rows of one sequence that fall in two splits (and two blocks of
     different widths): each split's item encodes its own part, and the
