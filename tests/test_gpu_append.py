@@ -182,16 +182,17 @@ def test_append_decode_matches_separate_calls_and_oracle(d, hq, hkv, dtype, rota
 
 
 @pytest.mark.parametrize("d,hq,hkv", [(128, 40, 8), (256, 16, 8), (256, 16, 4)])   # heads, pairs, heads
-def test_append_decode_rows_across_split_and_block_boundaries(d, hq, hkv):
-    """New rows of one sequence that fall in two splits (and two blocks of
-    different widths): each split's item encodes its own part, and the
-    result equals the two calls and the oracle."""
+@pytest.mark.parametrize("n_q8", [0, 7])
+def test_append_decode_rows_across_split_and_block_boundaries(d, hq, hkv, n_q8):
+    """New rows of one sequence that fall in two splits (and two blocks,
+    of different widths when the pool has 8-bit blocks): each split's item
+    encodes its own part, and the result equals the two calls and the
+    oracle."""
     dev = cuda()
     lens = [510, 0, 1020, 255]          # + new: 510..512 and 1020..1024 cross a split (512 tokens) and a block
     new = [3, 2, 5, 1]
     B, max_new, mb = len(lens), 5, 5
     tables = torch.randperm(B * mb, generator=torch.Generator().manual_seed(d + 3)).to(torch.int32).view(B, mb).numpy()
-    n_q8 = 7
     (fused, sep), ref = _prefilled(d, hkv, torch.bfloat16, True, B * mb - n_q8, n_q8, lens, tables, seed=d + 5)
     kn, vn = W.random_small(B * max_new, hkv, d, "bf16", seed=41)
     kn, vn = kn.view(B, max_new, hkv, d), vn.view(B, max_new, hkv, d)
